@@ -1,0 +1,123 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that the pins catch each.
+
+Each mutant replaces one oracle function with a subtly wrong version: a dropped term, a
+wrong sign or index, an off-by-one, a transposed operand.  The pin named beside it must
+then fail.  This shows the pins constrain the oracle, not just exercise it.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+import oracle.dsa_oracle as OD
+import tests.test_oracle_pins as P
+
+
+def _scores_no_relu(q_t, w_t, k, pos, pool=1):
+    S = k.shape[0]; n = min(S, pos // pool + 1)
+    out = np.full(S, -np.inf, dtype=np.float32)
+    out[:n] = ((k[:n] @ q_t.T) @ np.asarray(w_t, np.float64)).astype(np.float32)
+    return out
+
+
+def _scores_excl_self(q_t, w_t, k, pos, pool=1):
+    out = OD._orig["index_scores_row"](q_t, w_t, k, pos, pool)
+    if pos // pool < k.shape[0]:
+        out[pos // pool] = -np.inf
+    return out
+
+
+def _scores_weights_reversed(q_t, w_t, k, pos, pool=1):
+    return OD._orig["index_scores_row"](q_t, np.asarray(w_t)[::-1].copy(), k, pos, pool)
+
+
+def _scores_abs_instead_of_relu(q_t, w_t, k, pos, pool=1):
+    S = k.shape[0]; n = min(S, pos // pool + 1)
+    out = np.full(S, -np.inf, dtype=np.float32)
+    out[:n] = (np.abs(k[:n] @ q_t.T) @ np.asarray(w_t, np.float64)).astype(np.float32)
+    return out
+
+
+def _topk_ties_high_index(scores, n_valid, k):
+    n = int(min(n_valid, scores.shape[0])); out = np.full(k, -1, np.int32)
+    order = np.lexsort((-np.arange(n), -np.asarray(scores[:n], np.float64)))
+    out[: min(k, n)] = order[: min(k, n)]
+    return out
+
+
+def _topk_smallest(scores, n_valid, k):
+    n = int(min(n_valid, scores.shape[0])); out = np.full(k, -1, np.int32)
+    order = np.lexsort((np.arange(n), np.asarray(scores[:n], np.float64)))
+    out[: min(k, n)] = order[: min(k, n)]
+    return out
+
+
+def _attn_no_scale(q_t, K, V, idx_row, sm_scale):
+    return OD._orig["sparse_attn_row"](q_t, K, V, idx_row, 1.0)
+
+
+def _attn_k_as_v(q_t, K, V, idx_row, sm_scale):
+    return OD._orig["sparse_attn_row"](q_t, K, K[:, : V.shape[1]], idx_row, sm_scale)
+
+
+def _attn_drop_last(q_t, K, V, idx_row, sm_scale):
+    r = [i for i in idx_row if i >= 0]
+    return OD._orig["sparse_attn_row"](q_t, K, V, np.array(r[:-1] if len(r) > 1 else r), sm_scale)
+
+
+def _decode_bias8(codes):
+    v = OD._orig["e4m3_to_f64"](codes)
+    c = np.asarray(codes, np.uint8)
+    return np.where(((c >> 3) & 0xF) == 0, v, v / 2.0)
+
+
+def _encode_truncate(x):
+    x = np.asarray(x, np.float32)
+    codes = OD._orig["f32_to_e4m3"](x)
+    back = OD._orig["e4m3_to_f64"](codes)
+    over = np.abs(back) > np.abs(x.astype(np.float64))
+    return np.where(over & (codes & 0x7F > 0), codes - 1, codes).astype(np.uint8)
+
+
+def _pool_half(k_idx, pool=4):
+    kf = OD._orig["e4m3_to_f64"](k_idx).astype(np.float32)
+    S = kf.shape[-2]; g = kf.reshape(kf.shape[:-2] + (S // 4, 4, kf.shape[-1]))
+    return OD._orig["f32_to_e4m3"]((g[..., 0, :] + g[..., 1, :]) * np.float32(0.5))
+
+
+def _expand_no_mask(block_ids, pos, pool):
+    out = np.full(block_ids.shape[0] * pool, -1, np.int32)
+    for i, b in enumerate(block_ids):
+        if b >= 0:
+            out[i * pool:(i + 1) * pool] = [pool * int(b) + r for r in range(pool)]
+    return out
+
+
+MUTANTS = [
+    ("index_scores_row", _scores_no_relu, ["test_indexer_single_head_unit_weight_is_relu_dot", "test_indexer_hand_worked_example"]),
+    ("index_scores_row", _scores_excl_self, ["test_indexer_causal_rule_includes_self", "test_indexer_brute_force_tiny"]),
+    ("index_scores_row", _scores_weights_reversed, ["test_indexer_brute_force_tiny", "test_indexer_hand_worked_example"]),
+    ("index_scores_row", _scores_abs_instead_of_relu, ["test_indexer_single_head_unit_weight_is_relu_dot"]),
+    ("topk_row", _topk_ties_high_index, ["test_topk_brute_force_sort"]),
+    ("topk_row", _topk_smallest, ["test_topk_brute_force_sort", "test_indexer_hand_worked_example"]),
+    ("sparse_attn_row", _attn_no_scale, ["test_attention_dense_when_all_keys_selected_matches_torch_sdpa", "test_attention_brute_force_and_permutation"]),
+    ("sparse_attn_row", _attn_k_as_v, ["test_attention_dense_when_all_keys_selected_matches_torch_sdpa"]),
+    ("sparse_attn_row", _attn_drop_last, ["test_attention_zero_query_is_mean_of_v_and_duplicates_count", "test_attention_brute_force_and_permutation"]),
+    ("e4m3_to_f64", _decode_bias8, ["test_e4m3_decode_all_codes_match_torch", "test_e4m3_decode_format_values"]),
+    ("f32_to_e4m3", _encode_truncate, ["test_e4m3_encode_matches_torch_in_range"]),
+    ("index_pool", _pool_half, ["test_pool_brute_force_and_library_requantisation"]),
+    ("expand_blocks", _expand_no_mask, ["test_pool_validity_and_expansion"]),
+]
+
+if not hasattr(OD, "_orig"):
+    OD._orig = {n: getattr(OD, n) for n in
+                ["index_scores_row", "topk_row", "sparse_attn_row", "e4m3_to_f64", "f32_to_e4m3",
+                 "index_pool", "expand_blocks"]}
+
+
+@pytest.mark.parametrize("fn,mutant,pins", MUTANTS, ids=[m[1].__name__ for m in MUTANTS])
+def test_pins_catch_planted_mistake(monkeypatch, fn, mutant, pins):
+    monkeypatch.setattr(OD, fn, mutant)
+    monkeypatch.setattr(O, fn, mutant)
+    for pin in pins:
+        with pytest.raises(AssertionError):
+            getattr(P, pin)()
