@@ -1,0 +1,183 @@
+/*
+ * dsa.h - C ABI of the B200 (sm_100a) DSA layer-group library (libdsa_b200.so).
+ *
+ * The method (prose sources):
+ *   - "GLM 5.2: How Four Co-Designed Mechanisms Beat Raw Scale", section "DeepSeek Sparse
+ *     Attention": Stage 1, coarse scoring (an indexer scores every token of the context for
+ *     the current query); Stage 2, fine selection (the top-2,048 tokens get full attention).
+ *   - same page, section "IndexShare: Amortizing the Indexer": the indexer runs once per
+ *     block of 4 layers and the block shares its selection.
+ *   - twiscan.com post on GLM-5.2 (IndexShare): the indexer runs in FP8; one indexer is
+ *     shared by a group of 4 layers and the other 3 reuse its selection.
+ *   - "GLM-5.3-Flash hybrid sparse-linear attention with IndexPool", section "What
+ *     changed": IndexPool pools four indexer keys into one.
+ *
+ * Conventions shared by every entry point
+ *   Positions   Sequence b holds ctx_len[b] keys (rows 0..ctx_len[b]-1 of its caches) and T
+ *               new queries at its end: query t sits at position pos(b,t) = ctx_len[b]-T+t.
+ *               A key row s (or pooled block s when pool > 1) is visible to the query iff
+ *               pool*s <= pos(b,t).  ctx_len is a DEVICE array of B int32, and the caller
+ *               guarantees T <= ctx_len[b] <= S_max * pool.
+ *   Types       e4m3 = OCP FP8 E4M3 ("e4m3fn") codes stored as uint8, unit scale.
+ *               bf16 = bfloat16 stored as uint16.  Scores and weights are IEEE fp32.
+ *   Layouts     Row-major, innermost dimension last, as written in each comment.
+ *   Memory      Every pointer is a device pointer (unless stated) owned by the caller.  The
+ *               library allocates no memory; calls that need scratch take a caller
+ *               workspace and say how large it must be.  Pointers must be 16-byte aligned
+ *               and row strides multiples of 16 bytes.
+ *   Streams     `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *               Every call only enqueues work on that stream; none synchronises the host.
+ *   Errors      Every call returns a dsa_status.  On any non-zero status nothing was
+ *               enqueued (argument checks happen before the first launch), except
+ *               DSA_ERR_CUDA from a failed launch, after which dsa_last_cuda_error() gives
+ *               the cudaError_t.  Unsupported shapes are rejected, never emulated.
+ *   Threads     Calls are reentrant; concurrent calls must not share output or workspace
+ *               buffers.
+ */
+#ifndef DSA_B200_H
+#define DSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,         /* null pointer, negative or inconsistent size */
+  DSA_ERR_UNSUPPORTED_SHAPE = 2,   /* a head count / dim / k outside the supported set */
+  DSA_ERR_MISALIGNED = 3,          /* pointer or stride not 16-byte aligned */
+  DSA_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below the size the *_workspace_size call gives */
+  DSA_ERR_CUDA = 5,                /* a CUDA launch failed; see dsa_last_cuda_error() */
+  DSA_ERR_TIMEOUT = 6              /* a bounded device-side wait gave up (kernel exited early) */
+} dsa_status;
+
+/* Static, NUL-terminated description of a status code (thread-safe). */
+const char* dsa_status_string(int status);
+
+/* cudaError_t of the last failed launch on the calling thread (0 if none). */
+int dsa_last_cuda_error(void);
+
+/* Number of the library's kernel launches enqueued by the calling thread so far
+ * (a running counter, for accounting in benchmarks). */
+uint64_t dsa_launch_count(void);
+
+/* ------------------------------------------------------------------------------------
+ * dsa_index_scores - the lightning indexer (Stage 1, coarse scoring; FP8 per the
+ * IndexShare post).  For every query t in [t_begin, t_begin + t_count) of every sequence:
+ *
+ *     I[t,s] = sum_{j<H_I} w[t,j] * max(0, sum_{d<d_I} q_idx[t,j,d] * k_idx[s,d])
+ *
+ * over the visible key rows s (pool*s <= pos(b,t)).  FP8 products are exact in fp32;
+ * accumulation is fp32 on the tensor cores; the weighted ReLU reduction runs in fp32 in
+ * the epilogue, so the per-head logits never reach memory.
+ *
+ *   q_idx  [B, T, H_I, d_I] e4m3      w [B, T, H_I] fp32      k_idx [B, S_max, d_I] e4m3
+ *   scores [B, t_count, ld] fp32 out:  row (b, t - t_begin); entries s < n_valid hold I;
+ *          entries from n_valid up to the end of the 128-key tile that holds the last
+ *          visible key are -inf; entries beyond are not written.
+ *   pool   1, or 4 when k_idx holds IndexPool blocks (validity 4*s <= pos).
+ * Supported: (H_I, d_I) in {(4, 64), (64, 128)}; ld >= S_max, ld % 4 == 0.
+ * ------------------------------------------------------------------------------------ */
+int dsa_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                     const int32_t* ctx_len, int B, int T, int S_max, int H_I, int d_I,
+                     int pool, int t_begin, int t_count, float* scores, int64_t ld,
+                     void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * dsa_topk - Stage 2, fine selection: per query row, the k_eff = min(k, n_valid) keys with
+ * the largest scores, n_valid = min(S_max, pos/pool + 1).  Ties at the k-th score are
+ * broken toward lower key index.  The selected keys are written in ascending key order,
+ * followed by -1 padding.  With pool > 1 (IndexPool) the k selected blocks expand to
+ * pool*k token ids pool*blk .. pool*blk+pool-1 (ascending); tokens beyond pos become -1.
+ *
+ *   scores  [B, t_count, ld] fp32 (as written by dsa_index_scores for the same t_begin)
+ *   idx     [B, T, k*pool] int32 out; rows t_begin .. t_begin+t_count-1 are written.
+ * Supported: 1 <= k <= 2048, pool in {1, 4}, ld % 4 == 0.
+ * ------------------------------------------------------------------------------------ */
+int dsa_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, int T, int S_max,
+             int pool, int t_begin, int t_count, int k, int32_t* idx, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * dsa_sparse_attn - attention of every query over its selected keys only (Stage 2; the
+ * "China's First Frontier Model?" page, section "The Time has Come": attend only to the
+ * indexer's candidates).  All Hq query heads share one KV head (MQA; MLA latent form when
+ * V aliases the first d_v columns of the K row):
+ *
+ *     O[t,h,:] = sum_i p_i * V[idx[t,i], :],  p = softmax_i(sm_scale * q[t,h,:] . K[idx[t,i], :])
+ *     lse[t,h] = log sum_i exp(sm_scale * q[t,h,:] . K[idx[t,i], :])
+ *
+ * bf16 inputs, fp32 online softmax and accumulation, bf16 output.  Entries idx < 0 are
+ * skipped; a repeated index counts once per occurrence.  A row with no selected key gives
+ * O = 0 and lse = -inf.
+ *
+ *   q    [B, T, Hq, d_qk] bf16 (contiguous)
+ *   kv   K rows: element (b, s, c) at kv[b*kv_batch_stride + s*kv_row_stride + c], c < d_qk
+ *   v    V rows, same form with v_* strides; NULL means V = the first d_v columns of kv
+ *   idx  [B, T, k] int32, entries in [0, ctx_len[b]) or < 0
+ *   out  [B, T, Hq, d_v] bf16          lse  [B, T, Hq] fp32 or NULL
+ *   ws   scratch of at least dsa_sparse_attn_workspace_size(B, T, Hq, d_v, k) bytes
+ *        (zero for long prefill; split-key partials for few-query batches such as decode)
+ * Supported: (Hq, d_qk, d_v) in {(16, 128, 128), (128, 576, 512)}; 1 <= k <= 8192.
+ * ------------------------------------------------------------------------------------ */
+size_t dsa_sparse_attn_workspace_size(int B, int T, int Hq, int d_v, int k);
+int dsa_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v,
+                    int64_t kv_row_stride, int64_t kv_batch_stride, int64_t v_row_stride,
+                    int64_t v_batch_stride, const int32_t* idx, int B, int T, int Hq, int d_qk,
+                    int d_v, int k, float sm_scale, uint16_t* out, float* lse, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * dsa_index_pool - IndexPool ("What changed": four indexer keys pooled into one):
+ *     k_pool[b, g, :] = e4m3(((k[4g] + k[4g+1]) + (k[4g+2] + k[4g+3])) * 0.25)
+ * with the sum in fp32 on the decoded keys and the requantisation round-to-nearest-even,
+ * saturating at +-448.
+ *   k_idx [B, S_max, d_I] e4m3 -> k_pool [B, S_max/4, d_I] e4m3.
+ * Supported: pool == 4, S_max % 4 == 0, d_I % 16 == 0.
+ * ------------------------------------------------------------------------------------ */
+int dsa_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool, uint8_t* k_pool,
+                   void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * dsa_group_forward - one IndexShare group ("IndexShare: Amortizing the Indexer"): the
+ * indexer and the top-k run ONCE, and each of the group_size attention layers reads the
+ * same index buffer.  Equivalent to dsa_index_scores + dsa_topk over all queries
+ * (processed in query chunks sized to the workspace), then group_size x dsa_sparse_attn.
+ * With pool == 4 the indexer runs on dsa_index_pool's blocks and `topk` counts blocks
+ * (idx then holds 4*topk token ids per row).  The comparator without IndexShare is
+ * group_size calls with group_size = 1 and per-layer indexer tensors.
+ * ------------------------------------------------------------------------------------ */
+typedef struct dsa_group_args {
+  /* indexer, shared by the group */
+  const uint8_t* q_idx;    /* [B, T, H_I, d_I] e4m3 */
+  const float* w;          /* [B, T, H_I] fp32 */
+  const uint8_t* k_idx;    /* [B, S_max, d_I] e4m3 */
+  const int32_t* ctx_len;  /* device [B] */
+  int32_t B, T, S_max, H_I, d_I;
+  int32_t topk;            /* keys (pool 1) or blocks (pool 4) selected per query */
+  int32_t pool;            /* 1 or 4 (IndexPool) */
+  int32_t group_size;      /* attention layers sharing the selection, 1..16 */
+  /* attention, one entry per layer: HOST arrays of group_size DEVICE pointers */
+  const uint16_t* const* q;   /* [B, T, Hq, d_qk] bf16 */
+  const uint16_t* const* kv;  /* K (latent) rows, strides below */
+  const uint16_t* const* v;   /* NULL, or per-layer V (NULL entries alias kv) */
+  uint16_t* const* out;       /* [B, T, Hq, d_v] bf16 */
+  float* const* lse;          /* NULL, or per-layer [B, T, Hq] fp32 (NULL entries skip) */
+  int64_t kv_row_stride, kv_batch_stride, v_row_stride, v_batch_stride;
+  int32_t Hq, d_qk, d_v;
+  float sm_scale;
+  int32_t* idx;            /* [B, T, topk*pool] int32 out: the shared selection */
+} dsa_group_args;
+
+/* Workspace for dsa_group_forward when the indexer is run over chunks of t_chunk queries
+ * (t_chunk >= 1; larger chunks mean fewer launches).  dsa_group_forward uses the largest
+ * chunk that fits in the ws_bytes it is given. */
+size_t dsa_group_workspace_size(const dsa_group_args* args, int t_chunk);
+int dsa_group_forward(const dsa_group_args* args, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSA_B200_H */

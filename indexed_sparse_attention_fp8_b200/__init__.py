@@ -1,0 +1,230 @@
+"""B200 (sm_100a) DSA layer group: FP8 lightning indexer -> top-k -> sparse MQA/MLA attention,
+with IndexShare (one selection per group of layers) and IndexPool.
+
+This module is a thin ctypes binding over the C ABI of libdsa_b200.so (include/dsa.h): it
+only marshals torch tensors into pointers and sizes.  Every step of the computation runs in
+the library's CUDA kernels; there is no CPU or PyTorch fallback.  Functions keep the C names.
+PyTorch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdsa_b200.so")
+
+_c_int, _c_i64, _c_p, _c_sz, _c_f = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
+
+STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED_SHAPE", 3: "DSA_ERR_MISALIGNED",
+          4: "DSA_ERR_WORKSPACE_TOO_SMALL", 5: "DSA_ERR_CUDA", 6: "DSA_ERR_TIMEOUT"}
+
+
+class DSAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = f"{fn} -> {STATUS.get(status, status)}: {_lib().dsa_status_string(status).decode()}"
+        if status == 5:
+            msg += f" (cudaError {_lib().dsa_last_cuda_error()})"
+        super().__init__(msg)
+
+
+class GroupArgs(ctypes.Structure):
+    """Mirror of dsa_group_args in include/dsa.h."""
+    _fields_ = [
+        ("q_idx", _c_p), ("w", _c_p), ("k_idx", _c_p), ("ctx_len", _c_p),
+        ("B", ctypes.c_int32), ("T", ctypes.c_int32), ("S_max", ctypes.c_int32), ("H_I", ctypes.c_int32),
+        ("d_I", ctypes.c_int32), ("topk", ctypes.c_int32), ("pool", ctypes.c_int32),
+        ("group_size", ctypes.c_int32),
+        ("q", ctypes.POINTER(_c_p)), ("kv", ctypes.POINTER(_c_p)), ("v", ctypes.POINTER(_c_p)),
+        ("out", ctypes.POINTER(_c_p)), ("lse", ctypes.POINTER(_c_p)),
+        ("kv_row_stride", _c_i64), ("kv_batch_stride", _c_i64), ("v_row_stride", _c_i64),
+        ("v_batch_stride", _c_i64),
+        ("Hq", ctypes.c_int32), ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32), ("sm_scale", _c_f),
+        ("idx", _c_p),
+    ]
+
+
+_LIB = None
+
+# name -> (restype, argtypes)
+_SIGS = {
+    "dsa_status_string": (ctypes.c_char_p, [_c_int]),
+    "dsa_last_cuda_error": (_c_int, []),
+    "dsa_launch_count": (ctypes.c_uint64, []),
+    "dsa_index_scores": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                  _c_int, _c_int, _c_p, _c_i64, _c_p]),
+    "dsa_topk": (_c_int, [_c_p, _c_i64, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p]),
+    "dsa_sparse_attn_workspace_size": (_c_sz, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "dsa_sparse_attn": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_int, _c_int, _c_int,
+                                 _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_sz, _c_p]),
+    "dsa_index_pool": (_c_int, [_c_p, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p]),
+    "dsa_group_workspace_size": (_c_sz, [ctypes.POINTER(GroupArgs), _c_int]),
+    "dsa_group_forward": (_c_int, [ctypes.POINTER(GroupArgs), _c_p, _c_sz, _c_p]),
+}
+
+
+def _lib() -> ctypes.CDLL:
+    """Load libdsa_b200.so (raises if it has not been built: there is no fallback)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m indexed_sparse_attention_fp8_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype, fn.argtypes = res, args
+        _LIB = lib
+    return _LIB
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise DSAError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device (the library has no CPU path)")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def launch_count() -> int:
+    return int(_lib().dsa_launch_count())
+
+
+# ---------------------------------------------------------------------------------- calls
+
+
+def dsa_index_scores(q_idx: torch.Tensor, w: torch.Tensor, k_idx: torch.Tensor, ctx_len: torch.Tensor,
+                     pool: int = 1, t_begin: int = 0, t_count: Optional[int] = None,
+                     scores: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Indexer scores [B, t_count, ld] fp32 of queries t_begin.. (see dsa_index_scores in dsa.h).
+    q_idx [B,T,H_I,d_I] uint8 (e4m3), w [B,T,H_I] f32, k_idx [B,S,d_I] uint8, ctx_len [B] i32."""
+    B, T, H, D = q_idx.shape
+    S = k_idx.shape[1]
+    tc = T - t_begin if t_count is None else t_count
+    ld = (S + 3) // 4 * 4
+    if scores is None:
+        scores = torch.empty((B, tc, ld), dtype=torch.float32, device=q_idx.device)
+    else:
+        ld = scores.stride(1)
+    _check("dsa_index_scores", _lib().dsa_index_scores(
+        _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(ctx_len), B, T, S, H, D, pool, t_begin, tc, _ptr(scores), ld,
+        _stream(stream)))
+    return scores
+
+
+def dsa_topk(scores: torch.Tensor, ctx_len: torch.Tensor, T: int, S_max: int, k: int, pool: int = 1,
+             t_begin: int = 0, idx: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Top-k token ids [B, T, k*pool] int32 (rows t_begin .. t_begin + scores.shape[1] written)."""
+    B, tc, ld = scores.shape
+    if idx is None:
+        idx = torch.full((B, T, k * pool), -1, dtype=torch.int32, device=scores.device)
+    _check("dsa_topk", _lib().dsa_topk(_ptr(scores), scores.stride(1), _ptr(ctx_len), B, T, S_max, pool, t_begin,
+                                       tc, k, _ptr(idx), _stream(stream)))
+    return idx
+
+
+def dsa_sparse_attn_workspace_size(B: int, T: int, Hq: int, d_v: int, k: int) -> int:
+    return int(_lib().dsa_sparse_attn_workspace_size(B, T, Hq, d_v, k))
+
+
+def dsa_sparse_attn(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, sm_scale: float, d_v: int,
+                    v: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                    lse: Optional[torch.Tensor] = None, want_lse: bool = False,
+                    ws: Optional[torch.Tensor] = None, stream=None):
+    """Sparse attention: q [B,T,Hq,d_qk] bf16, kv [B,S,*] bf16 (K rows; V = kv[..., :d_v] when v is None),
+    idx [B,T,k] int32.  Returns (out [B,T,Hq,d_v] bf16, lse [B,T,Hq] f32 or None)."""
+    B, T, Hq, Dqk = q.shape
+    k = idx.shape[-1]
+    if out is None:
+        out = torch.empty((B, T, Hq, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, T, Hq), dtype=torch.float32, device=q.device)
+    need = dsa_sparse_attn_workspace_size(B, T, Hq, d_v, k)
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wsb = 0 if ws is None else ws.numel() * ws.element_size()
+    v_rs = v.stride(1) if v is not None else 0
+    v_bs = v.stride(0) if v is not None else 0
+    _check("dsa_sparse_attn", _lib().dsa_sparse_attn(
+        _ptr(q), _ptr(kv), _ptr(v), kv.stride(1), kv.stride(0), v_rs, v_bs, _ptr(idx), B, T, Hq, Dqk, d_v, k,
+        float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws), wsb, _stream(stream)))
+    return out, lse
+
+
+def dsa_index_pool(k_idx: torch.Tensor, pool: int = 4, k_pool: Optional[torch.Tensor] = None, stream=None):
+    """IndexPool: [B, S, d_I] e4m3 keys -> [B, S/4, d_I] pooled e4m3 keys."""
+    B, S, D = k_idx.shape
+    if k_pool is None:
+        k_pool = torch.empty((B, S // pool, D), dtype=torch.uint8, device=k_idx.device)
+    _check("dsa_index_pool", _lib().dsa_index_pool(_ptr(k_idx), B, S, D, pool, _ptr(k_pool), _stream(stream)))
+    return k_pool
+
+
+class Group:
+    """Marshalled arguments of one IndexShare group (keeps the pointer arrays alive)."""
+
+    def __init__(self, q_idx, w, k_idx, ctx_len, topk: int, layers: Sequence[dict], sm_scale: float,
+                 d_v: int, pool: int = 1, idx: Optional[torch.Tensor] = None, want_lse: bool = False):
+        B, T, H, D = q_idx.shape
+        S = k_idx.shape[1]
+        L = len(layers)
+        self.layers = list(layers)
+        q0, kv0 = layers[0]["q"], layers[0]["kv"]
+        Hq, Dqk = q0.shape[2], q0.shape[3]
+        for lay in self.layers:
+            if lay.get("out") is None:
+                lay["out"] = torch.empty((B, T, Hq, d_v), dtype=torch.bfloat16, device=q0.device)
+            if want_lse and lay.get("lse") is None:
+                lay["lse"] = torch.empty((B, T, Hq), dtype=torch.float32, device=q0.device)
+        self.idx = idx if idx is not None else torch.empty((B, T, topk * pool), dtype=torch.int32, device=q0.device)
+        arr = lambda xs: (_c_p * L)(*[_ptr(x) for x in xs])  # noqa: E731
+        self._q = arr([l["q"] for l in self.layers])
+        self._kv = arr([l["kv"] for l in self.layers])
+        vs = [l.get("v") for l in self.layers]
+        self._v = arr(vs) if any(v is not None for v in vs) else None
+        self._out = arr([l["out"] for l in self.layers])
+        lses = [l.get("lse") for l in self.layers]
+        self._lse = arr(lses) if any(x is not None for x in lses) else None
+        v_any = next((v for v in vs if v is not None), None)
+        self.args = GroupArgs(
+            q_idx=_ptr(q_idx), w=_ptr(w), k_idx=_ptr(k_idx), ctx_len=_ptr(ctx_len),
+            B=B, T=T, S_max=S, H_I=H, d_I=D, topk=topk, pool=pool, group_size=L,
+            q=self._q, kv=self._kv, v=self._v, out=self._out, lse=self._lse,
+            kv_row_stride=kv0.stride(1), kv_batch_stride=kv0.stride(0),
+            v_row_stride=v_any.stride(1) if v_any is not None else 0,
+            v_batch_stride=v_any.stride(0) if v_any is not None else 0,
+            Hq=Hq, d_qk=Dqk, d_v=d_v, sm_scale=float(sm_scale), idx=_ptr(self.idx))
+        self.device = q0.device
+
+    def workspace_size(self, t_chunk: int) -> int:
+        return int(_lib().dsa_group_workspace_size(ctypes.byref(self.args), int(t_chunk)))
+
+    def forward(self, ws: torch.Tensor, stream=None):
+        _check("dsa_group_forward", _lib().dsa_group_forward(
+            ctypes.byref(self.args), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+        return self.idx, [(l["out"], l.get("lse")) for l in self.layers]
+
+
+def dsa_group_forward(q_idx, w, k_idx, ctx_len, topk: int, layers: Sequence[dict], sm_scale: float, d_v: int,
+                      pool: int = 1, t_chunk: Optional[int] = None, ws: Optional[torch.Tensor] = None,
+                      want_lse: bool = False, stream=None):
+    """One IndexShare group: indexer + top-k once, then attention for each layer dict
+    {"q", "kv", optional "v", "out", "lse"}.  Returns (idx, [(out, lse) per layer])."""
+    g = Group(q_idx, w, k_idx, ctx_len, topk, layers, sm_scale, d_v, pool, want_lse=want_lse)
+    if ws is None:
+        ws = torch.empty(g.workspace_size(t_chunk or q_idx.shape[1]), dtype=torch.uint8, device=g.device)
+    return g.forward(ws, stream)

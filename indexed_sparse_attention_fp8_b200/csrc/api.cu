@@ -1,0 +1,244 @@
+// C ABI of the DSA library: argument validation, workspace sizing and launch sequencing.
+// Every entry point validates everything before its first launch, so a non-zero status
+// (other than DSA_ERR_CUDA) means nothing was enqueued.
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dsa {
+
+static thread_local int g_last_cuda_error = 0;
+static thread_local uint64_t g_launches = 0;
+
+void set_cuda_error(cudaError_t e) { g_last_cuda_error = static_cast<int>(e); }
+void count_launch() { ++g_launches; }
+
+int num_sms() {
+  static int cache[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+namespace {
+
+bool indexer_shape_ok(int H_I, int d_I) { return (H_I == 64 && d_I == 128) || (H_I == 4 && d_I == 64); }
+bool attn_shape_ok(int Hq, int d_qk, int d_v) {
+  return (Hq == 128 && d_qk == 576 && d_v == 512) || (Hq == 16 && d_qk == 128 && d_v == 128);
+}
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int check_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                       const int32_t* ctx_len, int B, int T, int S_max, int H_I, int d_I, int pool,
+                       int t_begin, int t_count, const float* scores, int64_t ld) {
+  if (B < 0 || T < 1 || S_max < 1 || t_begin < 0 || t_count < 0 || t_begin + t_count > T)
+    return DSA_ERR_INVALID_ARG;
+  if (pool != 1 && pool != 4) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (ld < S_max || (ld & 3)) return DSA_ERR_INVALID_ARG;
+  if (B == 0 || t_count == 0) return DSA_OK;
+  if (!q_idx || !w || !k_idx || !ctx_len || !scores) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx) || !aligned16(scores)) return DSA_ERR_MISALIGNED;
+  return DSA_OK;
+}
+
+int check_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, int T, int S_max,
+               int pool, int t_begin, int t_count, int k, const int32_t* idx) {
+  if (B < 0 || T < 1 || S_max < 1 || t_begin < 0 || t_count < 0 || t_begin + t_count > T)
+    return DSA_ERR_INVALID_ARG;
+  if (pool != 1 && pool != 4) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (k < 1 || k > 2048) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (ld < S_max || (ld & 3)) return DSA_ERR_INVALID_ARG;
+  if (B == 0 || t_count == 0) return DSA_OK;
+  if (!scores || !ctx_len || !idx) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(scores)) return DSA_ERR_MISALIGNED;
+  return DSA_OK;
+}
+
+int check_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t kv_rs,
+               int64_t kv_bs, int64_t v_rs, int64_t v_bs, const int32_t* idx, int B, int T, int Hq,
+               int d_qk, int d_v, int k, const uint16_t* out, const void* ws, size_t ws_bytes) {
+  if (B < 0 || T < 0 || k < 1 || k > 8192) return DSA_ERR_INVALID_ARG;
+  if (!attn_shape_ok(Hq, d_qk, d_v)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (Hq == 128 && v != nullptr) return DSA_ERR_UNSUPPORTED_SHAPE;  // MLA: V is part of the K row
+  if (kv_rs < d_qk || kv_bs < 0 || (v && (v_rs < d_v || v_bs < 0))) return DSA_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return DSA_OK;
+  if (!q || !kv || !idx || !out) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || (v && !aligned16(v)))
+    return DSA_ERR_MISALIGNED;
+  if ((kv_rs & 7) || (kv_bs & 7) || (v && ((v_rs & 7) || (v_bs & 7)))) return DSA_ERR_MISALIGNED;
+  const size_t need = attn_workspace_bytes(B, T, Hq, d_v, k);
+  if (ws_bytes < need) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  if (need > 0 && (!ws || !aligned16(ws))) return ws ? DSA_ERR_MISALIGNED : DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+// Workspace pieces of a group call: pooled keys, attention partials, a scores chunk.
+struct GroupWs {
+  size_t pool_bytes, attn_bytes, fixed_bytes;
+  int S_eff;
+  int64_t ld;
+};
+
+GroupWs group_ws(const dsa_group_args* a) {
+  GroupWs g;
+  g.S_eff = a->pool > 1 ? a->S_max / a->pool : a->S_max;
+  g.ld = (int64_t)round_up((size_t)g.S_eff, 4);
+  g.pool_bytes = a->pool > 1 ? round_up((size_t)a->B * g.S_eff * a->d_I, 256) : 0;
+  g.attn_bytes = round_up(attn_workspace_bytes(a->B, a->T, a->Hq, a->d_v, a->topk * a->pool), 256);
+  g.fixed_bytes = g.pool_bytes + g.attn_bytes;
+  return g;
+}
+
+int check_group(const dsa_group_args* a) {
+  if (!a) return DSA_ERR_INVALID_ARG;
+  if (a->group_size < 1 || a->group_size > 16 || !a->q || !a->kv || !a->out || !a->idx)
+    return DSA_ERR_INVALID_ARG;
+  if (a->pool != 1 && a->pool != 4) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (a->pool > 1 && (a->S_max % a->pool)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (a->topk < 1 || a->topk > 2048) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (a->topk * a->pool > 8192) return DSA_ERR_UNSUPPORTED_SHAPE;
+  const int S_eff = a->pool > 1 ? a->S_max / a->pool : a->S_max;
+  const int64_t ld = (int64_t)round_up((size_t)S_eff, 4);
+  int st = check_index_scores(a->q_idx, a->w, a->k_idx, a->ctx_len, a->B, a->T, S_eff, a->H_I,
+                              a->d_I, a->pool, 0, a->T, reinterpret_cast<const float*>(16), ld);
+  if (st != DSA_OK) return st;
+  // the attention workspace is carved from the group workspace: only shapes are checked here
+  for (int l = 0; l < a->group_size; ++l) {
+    const uint16_t* v = a->v ? a->v[l] : nullptr;
+    st = check_attn(a->q[l], a->kv[l], v, a->kv_row_stride, a->kv_batch_stride, a->v_row_stride,
+                    a->v_batch_stride, a->idx, a->B, a->T, a->Hq, a->d_qk, a->d_v,
+                    a->topk * a->pool, a->out[l], reinterpret_cast<const void*>(256), (size_t)-1);
+    if (st != DSA_OK) return st;
+  }
+  return DSA_OK;
+}
+
+}  // namespace
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+const char* dsa_status_string(int status) {
+  switch (status) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case DSA_ERR_MISALIGNED: return "pointer or stride not 16-byte aligned";
+    case DSA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case DSA_ERR_CUDA: return "CUDA launch failed";
+    case DSA_ERR_TIMEOUT: return "bounded device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int dsa_last_cuda_error(void) { return g_last_cuda_error; }
+uint64_t dsa_launch_count(void) { return g_launches; }
+
+int dsa_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                     const int32_t* ctx_len, int B, int T, int S_max, int H_I, int d_I, int pool,
+                     int t_begin, int t_count, float* scores, int64_t ld, void* stream) {
+  const int st = check_index_scores(q_idx, w, k_idx, ctx_len, B, T, S_max, H_I, d_I, pool,
+                                    t_begin, t_count, scores, ld);
+  if (st != DSA_OK || B == 0 || t_count == 0) return st;
+  return launch_index_scores(q_idx, w, k_idx, ctx_len, B, T, S_max, H_I, d_I, pool, t_begin,
+                             t_count, scores, ld, static_cast<cudaStream_t>(stream));
+}
+
+int dsa_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, int T, int S_max,
+             int pool, int t_begin, int t_count, int k, int32_t* idx, void* stream) {
+  const int st = check_topk(scores, ld, ctx_len, B, T, S_max, pool, t_begin, t_count, k, idx);
+  if (st != DSA_OK || B == 0 || t_count == 0) return st;
+  return launch_topk(scores, ld, ctx_len, B, T, S_max, pool, t_begin, t_count, k, idx,
+                     static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_sparse_attn_workspace_size(int B, int T, int Hq, int d_v, int k) {
+  if (B <= 0 || T <= 0 || Hq <= 0 || d_v <= 0 || k <= 0) return 0;
+  return attn_workspace_bytes(B, T, Hq, d_v, k);
+}
+
+int dsa_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t kv_row_stride,
+                    int64_t kv_batch_stride, int64_t v_row_stride, int64_t v_batch_stride,
+                    const int32_t* idx, int B, int T, int Hq, int d_qk, int d_v, int k,
+                    float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                    void* stream) {
+  const int st = check_attn(q, kv, v, kv_row_stride, kv_batch_stride, v_row_stride,
+                            v_batch_stride, idx, B, T, Hq, d_qk, d_v, k, out, ws, ws_bytes);
+  if (st != DSA_OK || B == 0 || T == 0) return st;
+  return launch_sparse_attn(q, kv, v, kv_row_stride, kv_batch_stride, v_row_stride, v_batch_stride,
+                            idx, B, T, Hq, d_qk, d_v, k, sm_scale, out, lse, ws,
+                            static_cast<cudaStream_t>(stream));
+}
+
+int dsa_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool, uint8_t* k_pool,
+                   void* stream) {
+  if (B < 0 || S_max < 0 || d_I <= 0) return DSA_ERR_INVALID_ARG;
+  if (pool != 4 || (S_max % 4) || (d_I % 16)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || S_max == 0) return DSA_OK;
+  if (!k_idx || !k_pool) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(k_idx) || !aligned16(k_pool)) return DSA_ERR_MISALIGNED;
+  return launch_index_pool(k_idx, B, S_max, d_I, k_pool, static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_group_workspace_size(const dsa_group_args* a, int t_chunk) {
+  if (!a || t_chunk < 1) return 0;
+  const GroupWs g = group_ws(a);
+  const int tc = std::min(t_chunk, a->T);
+  return g.fixed_bytes + (size_t)a->B * tc * (size_t)g.ld * sizeof(float);
+}
+
+int dsa_group_forward(const dsa_group_args* a, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_group(a);
+  if (st != DSA_OK) return st;
+  if (a->B == 0) return DSA_OK;
+  const GroupWs g = group_ws(a);
+  const size_t row_bytes = (size_t)a->B * g.ld * sizeof(float);
+  if (ws_bytes < g.fixed_bytes + row_bytes) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  if (!ws) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return DSA_ERR_MISALIGNED;
+  const int t_chunk = (int)std::min<size_t>((size_t)a->T, (ws_bytes - g.fixed_bytes) / row_bytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint8_t* k_pool = base;
+  void* attn_ws = base + g.pool_bytes;
+  float* scores = reinterpret_cast<float*>(base + g.fixed_bytes);
+
+  const uint8_t* keys = a->k_idx;
+  if (a->pool > 1) {
+    st = launch_index_pool(a->k_idx, a->B, a->S_max, a->d_I, k_pool, s);
+    if (st != DSA_OK) return st;
+    keys = k_pool;
+  }
+  // IndexShare: one indexer + one top-k over every query, in chunks that fit the workspace
+  for (int t0 = 0; t0 < a->T; t0 += t_chunk) {
+    const int tc = std::min(t_chunk, a->T - t0);
+    st = launch_index_scores(a->q_idx, a->w, keys, a->ctx_len, a->B, a->T, g.S_eff, a->H_I, a->d_I,
+                             a->pool, t0, tc, scores, g.ld, s);
+    if (st != DSA_OK) return st;
+    st = launch_topk(scores, g.ld, a->ctx_len, a->B, a->T, g.S_eff, a->pool, t0, tc, a->topk,
+                     a->idx, s);
+    if (st != DSA_OK) return st;
+  }
+  // every layer of the group reads the same selection
+  for (int l = 0; l < a->group_size; ++l) {
+    const uint16_t* v = a->v ? a->v[l] : nullptr;
+    float* lse = a->lse ? a->lse[l] : nullptr;
+    st = launch_sparse_attn(a->q[l], a->kv[l], v, a->kv_row_stride, a->kv_batch_stride,
+                            a->v_row_stride, a->v_batch_stride, a->idx, a->B, a->T, a->Hq, a->d_qk,
+                            a->d_v, a->topk * a->pool, a->sm_scale, a->out[l], lse, attn_ws, s);
+    if (st != DSA_OK) return st;
+  }
+  return DSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,28 @@
+// Internal launchers of the DSA library (C++ linkage; the C ABI is in include/dsa.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dsa {
+
+int launch_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                        const int32_t* ctx_len, int B, int T, int S_max, int H_I, int d_I, int pool,
+                        int t_begin, int t_count, float* scores, int64_t ld, cudaStream_t stream);
+
+int launch_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, int T, int S_max,
+                int pool, int t_begin, int t_count, int k, int32_t* idx, cudaStream_t stream);
+
+// Split count the attention uses for a problem (1 = no split, no workspace).
+int attn_num_splits(int B, int T, int Hq, int k);
+size_t attn_workspace_bytes(int B, int T, int Hq, int d_v, int k);
+int launch_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v,
+                       int64_t kv_row_stride, int64_t kv_batch_stride, int64_t v_row_stride,
+                       int64_t v_batch_stride, const int32_t* idx, int B, int T, int Hq, int d_qk,
+                       int d_v, int k, float sm_scale, uint16_t* out, float* lse, void* ws,
+                       cudaStream_t stream);
+
+int launch_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, uint8_t* k_pool,
+                      cudaStream_t stream);
+
+}  // namespace dsa

@@ -1,0 +1,134 @@
+"""The C ABI without a GPU: the library builds, loads, exports every function include/dsa.h
+declares, and rejects bad arguments before any CUDA call (fake pointers are never touched:
+every call here fails validation, which happens before the first launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import indexed_sparse_attention_fp8_b200 as dsa
+from indexed_sparse_attention_fp8_b200 import build as dsa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, WS_SMALL = 0, 1, 2, 3, 4
+A = 0x10000  # a 16-byte aligned fake address; never dereferenced by the calls below
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dsa_build.build()
+    return dsa._lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+char\s*\*|int|size_t|uint64_t)\s+(dsa_\w+)\s*\(", src, re.M)))
+
+
+def test_header_declares_the_four_calls_and_helpers():
+    names = declared_functions()
+    for n in ["dsa_index_scores", "dsa_topk", "dsa_sparse_attn", "dsa_group_forward", "dsa_index_pool",
+              "dsa_group_workspace_size", "dsa_sparse_attn_workspace_size", "dsa_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_library_is_the_in_tree_native_build(lib):
+    assert os.path.dirname(dsa.LIB_PATH) == os.path.dirname(dsa.__file__)
+    assert lib._name == dsa.LIB_PATH
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.dsa_status_string(code)
+    assert lib.dsa_status_string(99) == b"unknown status"
+
+
+def test_index_scores_validation(lib):
+    f = lib.dsa_index_scores
+    good = dict(q=A, w=A, k=A, c=A, B=1, T=8, S=8, H=64, D=128, pool=1, tb=0, tc=8, sc=A, ld=8)
+
+    def call(**kw):
+        a = {**good, **kw}
+        return f(a["q"], a["w"], a["k"], a["c"], a["B"], a["T"], a["S"], a["H"], a["D"], a["pool"], a["tb"], a["tc"],
+                 a["sc"], a["ld"], None)
+    assert call(H=8) == UNSUPPORTED
+    assert call(H=64, D=64) == UNSUPPORTED
+    assert call(pool=2) == UNSUPPORTED
+    assert call(tb=4, tc=5) == INVALID
+    assert call(ld=6) == INVALID            # ld not a multiple of 4
+    assert call(ld=4) == INVALID            # ld < S_max
+    assert call(q=None) == INVALID
+    assert call(k=A + 8) == MISALIGNED
+    assert call(tc=0) == OK                 # empty chunk: nothing to launch
+
+
+def test_topk_validation(lib):
+    f = lib.dsa_topk
+    assert f(A, 8, A, 1, 8, 8, 1, 0, 8, 0, A, None) == UNSUPPORTED      # k = 0
+    assert f(A, 8, A, 1, 8, 8, 1, 0, 8, 4096, A, None) == UNSUPPORTED   # k > 2048
+    assert f(A, 8, A, 1, 8, 8, 3, 0, 8, 4, A, None) == UNSUPPORTED      # pool 3
+    assert f(A + 4, 8, A, 1, 8, 8, 1, 0, 8, 4, A, None) == MISALIGNED
+    assert f(A, 8, None, 1, 8, 8, 1, 0, 8, 4, A, None) == INVALID
+    assert f(A, 8, A, 0, 8, 8, 1, 0, 8, 4, A, None) == OK               # B = 0
+
+
+def test_sparse_attn_validation(lib):
+    f = lib.dsa_sparse_attn
+
+    def call(Hq=128, dqk=576, dv=512, v=None, kv_rs=576, k=2048, B=1, T=4, ws=None, wsb=0, q=A):
+        return f(q, A, v, kv_rs, 576 * 64, 0, 0, A, B, T, Hq, dqk, dv, k, 0.04, A, None, ws, wsb, None)
+    assert call(Hq=64) == UNSUPPORTED
+    assert call(dqk=512) == UNSUPPORTED
+    assert call(v=A) == UNSUPPORTED         # MLA shapes read V from the latent row
+    assert call(kv_rs=500) == INVALID
+    assert call(kv_rs=580) == MISALIGNED    # row stride not a multiple of 16 bytes
+    assert call(q=A + 2) == MISALIGNED
+    assert call(k=0) == INVALID
+    # decode-shaped problems split the keys and need a workspace
+    need = lib.dsa_sparse_attn_workspace_size(32, 1, 128, 512, 2048)
+    assert need > 0
+    assert call(B=32, T=1, ws=A, wsb=need - 1) == WS_SMALL
+    # long prefill needs none
+    assert lib.dsa_sparse_attn_workspace_size(1, 32768, 128, 512, 2048) == 0
+
+
+def test_index_pool_validation(lib):
+    f = lib.dsa_index_pool
+    assert f(A, 1, 10, 128, 4, A, None) == UNSUPPORTED    # S not a multiple of 4
+    assert f(A, 1, 16, 128, 2, A, None) == UNSUPPORTED
+    assert f(A, 1, 16, 24, 4, A, None) == UNSUPPORTED     # d_I not a multiple of 16
+    assert f(A + 1, 1, 16, 128, 4, A, None) == MISALIGNED
+    assert f(A, 0, 16, 128, 4, A, None) == OK
+
+
+def _group_args(pool=1, topk=2048, S=32768, T=32768, B=1, group=4, d_I=128, H_I=64):
+    P = ctypes.c_void_p
+    arr = (P * group)(*([A] * group))
+    return dsa.GroupArgs(q_idx=A, w=A, k_idx=A, ctx_len=A, B=B, T=T, S_max=S, H_I=H_I, d_I=d_I, topk=topk,
+                         pool=pool, group_size=group, q=arr, kv=arr, v=None, out=arr, lse=None,
+                         kv_row_stride=576, kv_batch_stride=576 * S, v_row_stride=0, v_batch_stride=0,
+                         Hq=128, d_qk=576, d_v=512, sm_scale=0.04, idx=A), arr
+
+
+def test_group_workspace_and_validation(lib):
+    args, keep = _group_args()
+    one = lib.dsa_group_workspace_size(ctypes.byref(args), 1)
+    big = lib.dsa_group_workspace_size(ctypes.byref(args), 1024)
+    assert one == 32768 * 4 and big == 1024 * 32768 * 4     # a chunk of fp32 score rows
+    # too small a workspace is refused before any launch
+    assert lib.dsa_group_forward(ctypes.byref(args), A, one - 16, None) == WS_SMALL
+    bad, keep2 = _group_args(topk=4096)
+    assert lib.dsa_group_forward(ctypes.byref(bad), A, 1 << 40, None) == UNSUPPORTED
+    pool_args, keep3 = _group_args(pool=4, topk=512, S=1048576, T=8192)
+    need = lib.dsa_group_workspace_size(ctypes.byref(pool_args), 1)
+    assert need == (1048576 // 4) * 128 + (1048576 // 4) * 4   # pooled keys + one score row
+    odd, keep4 = _group_args(pool=4, topk=512, S=1048574, T=8192)
+    assert lib.dsa_group_forward(ctypes.byref(odd), A, 1 << 40, None) == UNSUPPORTED
