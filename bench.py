@@ -1,0 +1,518 @@
+"""Benchmark of the DSA layer group on B200: query tokens/s per 4-layer IndexShare group.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill128k] [--impl ours|reference]
+
+A step is one IndexShare group over the whole workload: the FP8 indexer and the top-k over
+every query (in workspace-sized query chunks), then sparse attention for each of the 4
+layers, all inside one dsa_group_forward call (the C ABI).  Inputs are synthetic and seeded
+(indexed_sparse_attention_fp8_b200.workloads), already resident in HBM for `value`; `e2e`
+repeats the step from pinned host buffers with the host<->device copies inside the timed
+region.  Inputs are larger than L2, so no flush is needed between steps.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own replica of the workload
+(the path shards by sequence / query block with no exchange), value = all ranks' queries /
+max-over-ranks time, scaling "weak".
+
+The JSON line also carries: the decode line (32 x 256K), the per-layer-indexer comparator
+at 128K with the IndexShare speedup, a per-kernel breakdown from CUDA events, the roofline
+of the dominant kernel, SM clocks sampled during the timed region, and the CPU oracle's
+throughput on a bounded sample (cpu_baseline).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from indexed_sparse_attention_fp8_b200 import workloads as W  # noqa: E402
+
+METRIC = "query tok/s per 4-layer IndexShare group (prefill 128K, decode 256K); % roofline"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"], "bf16_sus": d["bf16_tflops_sustained"],
+                "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sus": 1400.0, "src": "fallback"}
+
+
+# ------------------------------------------------------------------------------ work counts
+
+def causal_pairs(wl: W.Workload) -> int:
+    """Visible (query, key-row) pairs of the indexer (pooled rows when pool > 1)."""
+    tot = 0
+    for t in range(wl.T):
+        pos = wl.ctx - wl.T + t
+        tot += min(wl.S // wl.pool, pos // wl.pool + 1)
+    return tot * wl.B
+
+
+def selected_pairs(wl: W.Workload) -> int:
+    """Sum over queries of the number of selected tokens (k_eff, expanded for IndexPool)."""
+    tot = 0
+    for t in range(wl.T):
+        pos = wl.ctx - wl.T + t
+        if wl.pool == 1:
+            tot += min(wl.topk, pos + 1)
+        else:
+            nb = min(wl.topk, pos // wl.pool + 1)
+            tot += min(nb * wl.pool, pos + 1)
+    return tot * wl.B
+
+
+def indexer_flops(wl):
+    return 2 * wl.H_I * wl.d_I * causal_pairs(wl)
+
+
+def attn_flops(wl):
+    return wl.Hq * 2 * (wl.d_qk + wl.d_v) * selected_pairs(wl)
+
+
+def attn_bytes(wl):
+    """Gathered KV rows (bf16) + q + out + idx per layer."""
+    row = wl.d_qk * 2 if wl.kv_latent else (wl.d_qk + wl.d_v) * 2
+    return selected_pairs(wl) * row + wl.B * wl.T * wl.Hq * (wl.d_qk + wl.d_v) * 2 + wl.B * wl.T * wl.topk * wl.pool * 4
+
+
+# ------------------------------------------------------------------------------ clocks
+
+def gpu_id(dev) -> str:
+    """nvidia-smi identifier of a torch device (UUID, so CUDA_VISIBLE_DEVICES cannot mislead it)."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:  # pragma: no cover
+        return str(torch.cuda.current_device())
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: str):
+        self.gpu = gpu
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ our arm
+
+def make_group(wl, dev, dsa, layers=None, indexer_layer=0, share_q=False):
+    ind = W.make_indexer_inputs(wl, device=dev, layer=indexer_layer)
+    n = wl.group if layers is None else layers
+    lays = []
+    for l in range(n):
+        a = W.make_attn_inputs(wl, l, device=dev) if (l == 0 or not share_q) else \
+            {"q": lays[0]["q"], "kv": W.make_attn_inputs(wl, l, device=dev)["kv"], "v": None}
+        lays.append({"q": a["q"], "kv": a["kv"], "v": a["v"]})
+    return ind, lays
+
+
+def time_region(fn, steps, stream):
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record(stream)
+    for _ in range(steps):
+        fn()
+    e.record(stream)
+    torch.cuda.synchronize()
+    return s.elapsed_time(e)
+
+
+def run_ours(args, rank, world, dev):
+    import indexed_sparse_attention_fp8_b200 as dsa
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+    wl = W.WORKLOADS[args.workload]
+    # q/out aliasing across layers would change no work; memory allows distinct tensors except at 128K
+    ind, lays = make_group(wl, dev, dsa)
+    g = dsa.Group(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk, lays, wl.sm_scale, wl.d_v,
+                  pool=wl.pool)
+    t_chunk = args.t_chunk or max(1, min(wl.T, (args.score_ws_gb << 30) // (wl.B * ((wl.S // wl.pool + 3) // 4 * 4) * 4)))
+    ws = torch.empty(g.workspace_size(t_chunk), dtype=torch.uint8, device=dev)
+    step = lambda: g.forward(ws, stream)  # noqa: E731
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    l0 = dsa.launch_count()
+    with ClockSampler(gpu_id(dev)) as clk:
+        ms = time_region(step, args.steps, stream)
+    launches = dsa.launch_count() - l0
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    q_per_step = wl.B * wl.T
+    value = q_per_step * world / (ms_step / 1e3)
+
+    # ---- per-kernel breakdown: the same step as separate C-ABI calls with events between them
+    brk = breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, args.steps if args.steps <= 3 else 3)
+
+    res = {
+        "metric": METRIC, "value": value, "unit": "query tok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8-e4m3 indexer / bf16 attention (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "ctx": wl.ctx, "H_I": wl.H_I, "d_I": wl.d_I,
+                   "topk": wl.topk, "pool": wl.pool, "Hq": wl.Hq, "d_qk": wl.d_qk, "d_v": wl.d_v,
+                   "group": wl.group, "t_chunk": t_chunk, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (126 MB); no flush"},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "breakdown_ms": brk,
+    }
+    res["roofline"] = roofline(wl, brk, pk)
+    del g, ws
+    torch.cuda.empty_cache()
+    return res, wl, ind, lays
+
+
+def breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, reps):
+    """Average device time of each kernel family over `reps` steps, CUDA events on `stream`."""
+    S_eff = wl.S // wl.pool
+    ld = (S_eff + 3) // 4 * 4
+    scores = torch.empty((wl.B, t_chunk, ld), dtype=torch.float32, device=ind["q_idx"].device)
+    keys = ind["k_idx"]
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    tot = {"pool": 0.0, "indexer": 0.0, "topk": 0.0, "attn": 0.0}
+    n = {"indexer": 0, "topk": 0, "attn": 0, "pool": 0}
+    attn_ws = torch.empty(max(1, dsa.dsa_sparse_attn_workspace_size(wl.B, wl.T, wl.Hq, wl.d_v, wl.topk * wl.pool)),
+                          dtype=torch.uint8, device=scores.device)
+    for _ in range(reps):
+        marks = []
+        if wl.pool > 1:
+            a, b = ev(), ev()
+            a.record(stream)
+            keys = dsa.dsa_index_pool(ind["k_idx"], stream=stream)
+            b.record(stream)
+            marks.append(("pool", a, b))
+        for t0 in range(0, wl.T, t_chunk):
+            tc = min(t_chunk, wl.T - t0)
+            a, b, c = ev(), ev(), ev()
+            a.record(stream)
+            dsa.dsa_index_scores(ind["q_idx"], ind["w"], keys, ind["ctx_len"], pool=wl.pool, t_begin=t0, t_count=tc,
+                                 scores=scores[:, :tc], stream=stream)
+            b.record(stream)
+            dsa.dsa_topk(scores[:, :tc], ind["ctx_len"], wl.T, S_eff, wl.topk, pool=wl.pool, t_begin=t0, idx=g.idx,
+                         stream=stream)
+            c.record(stream)
+            marks += [("indexer", a, b), ("topk", b, c)]
+        for L in lays:
+            a, b = ev(), ev()
+            a.record(stream)
+            dsa.dsa_sparse_attn(L["q"], L["kv"], g.idx, wl.sm_scale, wl.d_v, v=L["v"], out=L["out"], ws=attn_ws,
+                                stream=stream)
+            b.record(stream)
+            marks.append(("attn", a, b))
+        torch.cuda.synchronize()
+        for name, a, b in marks:
+            tot[name] += a.elapsed_time(b)
+            n[name] += 1
+    out = {k: tot[k] / reps for k in tot if n[k]}
+    out["per_launch"] = {"indexer_chunk": tot["indexer"] / max(1, n["indexer"]),
+                         "topk_chunk": tot["topk"] / max(1, n["topk"]), "attn_layer": tot["attn"] / max(1, n["attn"])}
+    return out
+
+
+def roofline(wl, brk, pk):
+    """Roofline of the kernel with the largest share of the step."""
+    fp8_peak = 2.0 * pk["bf16_sus"]   # nominal fp8:bf16 ratio 2 on the measured bf16 figure
+    ent = {
+        "indexer": {"bound": "tensor", "achieved": indexer_flops(wl) / (brk["indexer"] * 1e-3) / 1e12,
+                    "peak": fp8_peak, "unit": "TFLOP/s", "dtype": "fp8", "traffic": None,
+                    "peak_src": f"2 x {pk['src']} bf16 sustained"},
+        "attn": {"bound": "tensor", "achieved": attn_flops(wl) / (brk["per_launch"]["attn_layer"] * 1e-3) / 1e12,
+                 "peak": pk["bf16_sus"], "unit": "TFLOP/s", "dtype": "bf16", "traffic": None,
+                 "peak_src": f"{pk['src']} bf16 sustained"},
+    }
+    if wl.B * wl.T <= 64:   # decode: the attention reads every gathered row once; HBM-bound
+        ent["attn"] = {"bound": "hbm", "achieved": attn_bytes(wl) / (brk["per_launch"]["attn_layer"] * 1e-3) / 1e9,
+                       "peak": pk["hbm_gbs"], "unit": "GB/s", "traffic": None, "peak_src": f"{pk['src']} copy"}
+        ent["indexer"] = {"bound": "hbm",
+                          "achieved": (wl.B * wl.S * wl.d_I + wl.B * wl.T * wl.H_I * (wl.d_I + 4))
+                          / (brk["indexer"] * 1e-3) / 1e9,
+                          "peak": pk["hbm_gbs"], "unit": "GB/s", "traffic": None, "peak_src": f"{pk['src']} copy"}
+    top = max(("indexer", "attn"), key=lambda k: brk[k])
+    r = dict(ent[top])
+    r["kernel"] = top
+    r["frac"] = r["achieved"] / r["peak"]
+    r["others"] = {k: {kk: vv for kk, vv in v.items()} | {"frac": v["achieved"] / v["peak"]}
+                   for k, v in ent.items() if k != top}
+    return r
+
+
+def run_e2e(args, wl, ind, lays, dev, stream):
+    """Same step from pinned host memory: H2D of every input, the group call, D2H of every output."""
+    import indexed_sparse_attention_fp8_b200 as dsa
+    host = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in ind.items()}
+    for k in host:
+        host[k].copy_(ind[k])
+    hq = torch.empty_like(lays[0]["q"], device="cpu").pin_memory()
+    hkv = torch.empty_like(lays[0]["kv"], device="cpu").pin_memory()
+    hq.copy_(lays[0]["q"])
+    hkv.copy_(lays[0]["kv"])
+    g = dsa.Group(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk, lays, wl.sm_scale, wl.d_v, pool=wl.pool)
+    hout = torch.empty_like(g.layers[0]["out"], device="cpu").pin_memory()
+    t_chunk = args.t_chunk or max(1, min(wl.T, (args.score_ws_gb << 30) // (wl.B * ((wl.S // wl.pool + 3) // 4 * 4) * 4)))
+    ws = torch.empty(g.workspace_size(t_chunk), dtype=torch.uint8, device=dev)
+    h2d = sum(v.numel() * v.element_size() for v in host.values()) + len(lays) * (
+        hq.numel() * hq.element_size() + hkv.numel() * hkv.element_size())
+    d2h = len(lays) * hout.numel() * hout.element_size() + g.idx.numel() * 4
+    hidx = torch.empty_like(g.idx, device="cpu").pin_memory()
+
+    def step():
+        for k in host:
+            ind[k].copy_(host[k], non_blocking=True)
+        for L in g.layers:
+            L["q"].copy_(hq, non_blocking=True)
+            L["kv"].copy_(hkv, non_blocking=True)
+        g.forward(ws, stream)
+        for L in g.layers:
+            hout.copy_(L["out"], non_blocking=True)
+        hidx.copy_(g.idx, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, args.e2e_steps))
+    ms = time_region(step, steps, stream) / steps
+    del ws, g
+    return {"value": wl.B * wl.T / (ms / 1e3), "unit": "query tok/s", "ms_per_step": ms, "steps": steps,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def run_secondary(args, name, dev, steps=3, per_layer=False):
+    """Another workload (decode) or the per-layer-indexer comparator, timed the same way."""
+    import indexed_sparse_attention_fp8_b200 as dsa
+    stream = torch.cuda.current_stream()
+    wl = W.WORKLOADS[name]
+    if not per_layer:
+        ind, lays = make_group(wl, dev, dsa)
+        g = dsa.Group(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk, lays, wl.sm_scale, wl.d_v,
+                      pool=wl.pool)
+        t_chunk = max(1, min(wl.T, (args.score_ws_gb << 30) // (wl.B * ((wl.S // wl.pool + 3) // 4 * 4) * 4)))
+        ws = torch.empty(g.workspace_size(t_chunk), dtype=torch.uint8, device=dev)
+        fn = lambda: g.forward(ws, stream)  # noqa: E731
+        for _ in range(max(3, args.warmup)):
+            fn()
+        ms = time_region(fn, steps, stream) / steps
+        brk = breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, 3)
+        r = {"workload": name, "value": wl.B * wl.T / (ms / 1e3), "unit": "query tok/s", "ms_per_step": ms,
+             "steps": steps, "breakdown_ms": brk, "roofline": roofline(wl, brk, peaks())}
+        del g, ws, ind, lays
+        torch.cuda.empty_cache()
+        return r
+    # per-layer indexer: each layer runs its own indexer + top-k (group_size 1, own indexer inputs)
+    inds = [W.make_indexer_inputs(wl, device=dev, layer=l) for l in range(wl.group)]
+    q0 = W.make_attn_inputs(wl, 0, device=dev)["q"]   # q shared across layers to fit memory (same work)
+    lays = [{"q": q0, "kv": W.make_attn_inputs(wl, l, device=dev)["kv"], "v": None} for l in range(wl.group)]
+    outbuf = torch.empty((wl.B, wl.T, wl.Hq, wl.d_v), dtype=torch.bfloat16, device=dev)
+    gs = [dsa.Group(inds[l]["q_idx"], inds[l]["w"], inds[l]["k_idx"], inds[l]["ctx_len"], wl.topk,
+                    [dict(lays[l], out=outbuf)], wl.sm_scale, wl.d_v) for l in range(wl.group)]
+    t_chunk = max(1, min(wl.T, (args.score_ws_gb << 30) // (wl.B * ((wl.S + 3) // 4 * 4) * 4)))
+    ws = torch.empty(gs[0].workspace_size(t_chunk), dtype=torch.uint8, device=dev)
+    fn = lambda: [g.forward(ws, stream) for g in gs]  # noqa: E731
+    fn()
+    ms = time_region(fn, steps, stream) / steps
+    r = {"workload": name + " per-layer indexer", "value": wl.B * wl.T / (ms / 1e3), "unit": "query tok/s",
+         "ms_per_step": ms, "steps": steps}
+    del gs, ws, inds, lays, outbuf
+    torch.cuda.empty_cache()
+    return r
+
+
+# ------------------------------------------------------------------------------ oracle arm
+
+_ORACLE_CACHE = {}
+
+
+def _oracle_inputs(wl):
+    """CPU inputs for timing the oracle: one sequence's full key caches (decoded once, input
+    conversion outside the timed region) and 64 query rows, from the same seeded generators."""
+    import oracle as O
+    if wl.name in _ORACLE_CACHE:
+        return _ORACLE_CACHE[wl.name]
+    small = wl.replace(B=1, T=min(wl.T, 64))
+    ind = W.make_indexer_inputs(small, device="cpu")
+    kdec = O.e4m3_to_f64(ind["k_idx"][0].numpy())
+    kp = O.e4m3_to_f64(O.index_pool(ind["k_idx"][0].numpy())) if wl.pool > 1 else None
+    layers = []
+    for l in range(wl.group):
+        a = W.make_attn_inputs(small.replace(T=1), l, device="cpu")
+        K = O.bf16_to_f64(a["kv"][0].view(torch.int16).numpy().view(np.uint16))
+        V = K[:, : wl.d_v] if wl.kv_latent else O.bf16_to_f64(a["v"][0].view(torch.int16).numpy().view(np.uint16))
+        q = O.bf16_to_f64(a["q"][0, 0].view(torch.int16).numpy().view(np.uint16))
+        layers.append({"q": q, "K": K, "V": V})
+    qrows = [O.e4m3_to_f64(ind["q_idx"][0, i].numpy()) for i in range(small.T)]
+    wrows = [ind["w"][0, i].numpy() for i in range(small.T)]
+    _ORACLE_CACHE[wl.name] = (kdec, kp, layers, qrows, wrows)
+    return _ORACLE_CACHE[wl.name]
+
+
+def oracle_sample(wl, seconds: float, seed: int = 0):
+    """Time the CPU oracle, as it stands, on query rows drawn uniformly from the workload's
+    positions: per row the indexer over every visible key, the top-k, and the attention of
+    every layer of the group.  Returns (rows/s, rows, threads, seconds spent)."""
+    import oracle as O
+    kdec, kp, layers, qrows, wrows = _oracle_inputs(wl)
+    rng = np.random.default_rng(seed)
+    rows, spent = 0, 0.0
+    while spent < seconds:
+        t = int(rng.integers(0, wl.T))
+        pos = wl.ctx - wl.T + t
+        s0 = time.perf_counter()
+        O.group_forward_row(qrows[t % len(qrows)], wrows[t % len(wrows)], kdec, pos, wl.topk, layers, wl.sm_scale,
+                            wl.pool, kp)
+        spent += time.perf_counter() - s0
+        rows += 1
+    return rows / spent, rows, torch.get_num_threads(), spent
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    wl = W.WORKLOADS[args.workload]
+    per_step = max(1.0, args.ref_seconds / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(wl, per_step * 0.2)
+    vals, rows_tot, spent_tot = [], 0, 0.0
+    for s in range(args.steps):
+        v, rows, cores, spent = oracle_sample(wl, per_step, seed=s)
+        vals.append(v)
+        rows_tot += rows
+        spent_tot += spent
+    value = rows_tot / spent_tot
+    note = (f"{rows_tot} query rows sampled uniformly from {wl.name}; each row = indexer over all visible keys, "
+            f"top-{wl.topk}, sparse attention for {wl.group} layers, fp64 numpy; key caches decoded once outside timing")
+    return {"metric": METRIC, "value": value, "unit": "query tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "ctx": wl.ctx, "topk": wl.topk, "group": wl.group},
+            "cpu_baseline": {"value": value, "unit": "query tok/s", "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": note},
+            "e2e": {"value": value, "unit": "query tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill128k", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--t-chunk", type=int, default=0)
+    ap.add_argument("--score-ws-gb", type=int, default=8, help="GiB of workspace for indexer score chunks")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--ref-seconds", type=float, default=60.0)
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl" if args.impl == "ours" else "gloo",
+                                             timeout=datetime.timedelta(seconds=600))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    res, wl, ind, lays = run_ours(args, rank, world, dev)
+    if not args.no_e2e:
+        try:
+            res["e2e"] = run_e2e(args, wl, ind, lays, dev, torch.cuda.current_stream())
+        except (RuntimeError, torch.cuda.OutOfMemoryError) as e:  # pinned host memory can run out
+            res["e2e"] = {"error": str(e)[:300]}
+    del ind, lays
+    torch.cuda.empty_cache()
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0 and not args.no_secondary and args.workload == "prefill128k":
+        try:
+            pl = run_secondary(args, "prefill128k", dev, steps=2, per_layer=True)
+            pl["indexshare_speedup"] = pl["ms_per_step"] / res["ms_per_step"]
+            res["per_layer_indexer"] = pl
+        except torch.cuda.OutOfMemoryError as e:  # pragma: no cover
+            res["per_layer_indexer"] = {"error": str(e)[:200]}
+        res["decode256k"] = run_secondary(args, "decode256k", dev, steps=10)
+    if rank == 0 and world == 1:
+        v, rows, cores, spent = oracle_sample(W.WORKLOADS[args.workload], args.cpu_seconds)
+        res["cpu_baseline"] = {"value": v, "unit": "query tok/s", "cores": cores, "kind": "oracle",
+                               "sample": f"{rows} query rows of {args.workload} in {spent:.1f}s (indexer row + "
+                                         f"top-k + {W.WORKLOADS[args.workload].group} attention layers, fp64)"}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -64,6 +64,19 @@ int dsa_last_cuda_error(void);
  * (a running counter, for accounting in benchmarks). */
 uint64_t dsa_launch_count(void);
 
+/* Synchronises `stream`, then reads and clears the device status words of the library's
+ * kernels on the current device.  Returns DSA_OK, or DSA_ERR_TIMEOUT when a kernel gave up
+ * one of its bounded waits since the last call (that launch exited early and its outputs
+ * are incomplete), or DSA_ERR_CUDA if the synchronisation failed.  Every wait inside the
+ * tensor-core kernels has a time limit, so no launch can hang. */
+int dsa_device_status(void* stream);
+
+/* Test hook for the failure path: enqueues one thread that waits, through the kernels' own
+ * bounded wait, on a barrier that nothing ever completes, so the wait gives up after
+ * limit_ns (1 ns .. 1 s) and sets the device status word; the next dsa_device_status() then
+ * returns DSA_ERR_TIMEOUT.  Faults nothing; the CUDA context stays usable. */
+int dsa_debug_wait_timeout(uint64_t limit_ns, void* stream);
+
 /* ------------------------------------------------------------------------------------
  * dsa_index_scores - the lightning indexer (Stage 1, coarse scoring; FP8 per the
  * IndexShare post).  For every query t in [t_begin, t_begin + t_count) of every sequence:

@@ -55,6 +55,8 @@ _SIGS = {
     "dsa_status_string": (ctypes.c_char_p, [_c_int]),
     "dsa_last_cuda_error": (_c_int, []),
     "dsa_launch_count": (ctypes.c_uint64, []),
+    "dsa_device_status": (_c_int, [_c_p]),
+    "dsa_debug_wait_timeout": (_c_int, [ctypes.c_uint64, _c_p]),
     "dsa_index_scores": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                   _c_int, _c_int, _c_p, _c_i64, _c_p]),
     "dsa_topk": (_c_int, [_c_p, _c_i64, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p]),
@@ -102,6 +104,17 @@ def _stream(stream) -> Optional[int]:
 
 def launch_count() -> int:
     return int(_lib().dsa_launch_count())
+
+
+def dsa_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the kernels' device status: 0, or 6
+    (DSA_ERR_TIMEOUT) when a bounded device wait gave up."""
+    return int(_lib().dsa_device_status(_stream(stream)))
+
+
+def dsa_debug_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Enqueue the bounded-wait probe: its wait runs out after limit_ns and sets the status."""
+    _check("dsa_debug_wait_timeout", _lib().dsa_debug_wait_timeout(int(limit_ns), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------------- calls

@@ -142,7 +142,21 @@ const char* dsa_status_string(int status) {
 }
 
 int dsa_last_cuda_error(void) { return g_last_cuda_error; }
+
+int dsa_device_status(void* stream) {
+  const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return DSA_ERR_CUDA;
+  }
+  return indexer_take_status() ? DSA_ERR_TIMEOUT : DSA_OK;
+}
 uint64_t dsa_launch_count(void) { return g_launches; }
+
+int dsa_debug_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return DSA_ERR_INVALID_ARG;
+  return launch_wait_timeout_probe(limit_ns, static_cast<cudaStream_t>(stream));
+}
 
 int dsa_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                      const int32_t* ctx_len, int B, int T, int S_max, int H_I, int d_I, int pool,

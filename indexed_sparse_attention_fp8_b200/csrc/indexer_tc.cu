@@ -1,0 +1,378 @@
+// Lightning indexer on the 5th-generation tensor cores (Stage 1 of "DeepSeek Sparse
+// Attention", "GLM 5.2: How Four Co-Designed Mechanisms Beat Raw Scale"; FP8 per the
+// twiscan.com IndexShare post):
+//
+//     I[t,s] = sum_j w[t,j] * max(0, q_idx[t,j,:] . k_idx[s,:])
+//
+// GEMM view: A = 128 keys x d_I (e4m3, K-major rows of the key cache), B = QB queries x H_I
+// heads = N rows x d_I (e4m3, the q_idx rows of QB consecutive queries), D = A B^T in TMEM
+// (128 lanes = keys, N fp32 columns = (query, head)).  Each TMEM lane holds every head of
+// every query of the block for one key, so the weighted ReLU reduction over heads runs in
+// one thread, and the per-head logits never leave the SM.
+//
+// Persistent kernel, one CTA per SM, warp-specialised:
+//   warp 0      TMA producer: key tiles (ring of NA stages), query blocks + head weights
+//               (2 stages), all through mbarrier transaction counts
+//   warp 1      TMEM owner and MMA issuer: d_I/32 tcgen05.mma (kind::f8f6f4, M=128, N) per
+//               key tile into one of two TMEM accumulators
+//   warps 2..9  epilogue: tcgen05.ld the accumulator, w * relu, sum over heads, causal mask,
+//               coalesced fp32 stores of the score rows
+// Work items are (sequence, block of QB queries, chunk of KC key tiles); key tiles past the
+// causal frontier of the block's last query are never loaded or multiplied.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace dsa {
+namespace {
+
+using namespace tc;
+
+constexpr int KTILE = 128;        // keys per tile (MMA M)
+constexpr int KC = 32;            // key tiles per work item
+constexpr int NA = 6;             // key-tile stages
+constexpr int NUM_THREADS = 320;  // 10 warps
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no legal wait comes close
+
+template <int H, int D, int QB>
+struct IdxCfg {
+  static constexpr int N = QB * H;                 // MMA N: (query, head) columns
+  static constexpr int A_BYTES = KTILE * D;        // one key tile
+  static constexpr int B_BYTES = N * D;            // one query block
+  static constexpr int W_BYTES = QB * H * 4;       // head weights of the block
+  static constexpr int HALVES = N >= 128 ? 2 : 1;  // epilogue column halves
+  static constexpr int COLS = N / HALVES;          // columns per epilogue warp
+  static constexpr int CHUNKS = COLS / 32;
+  static constexpr int QPH = COLS / H > 0 ? COLS / H : 1;  // queries per epilogue warp
+  static constexpr uint32_t TMEM_COLS = 2 * N <= 32 ? 32 : (2 * N <= 64 ? 64 : (2 * N <= 128 ? 128 : (2 * N <= 256 ? 256 : 512)));
+  static constexpr uint32_t SBO = 8 * D;           // 8-row group stride of a swizzled tile
+  static constexpr uint32_t LAYOUT = D == 128 ? kLayoutSw128 : kLayoutSw64;
+  static constexpr uint32_t IDESC = instr_desc(128, N, 0);
+  // shared memory map (offsets from a 1024-aligned base)
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + NA * A_BYTES;
+  static constexpr int OFF_W = OFF_B + 2 * B_BYTES;
+  static constexpr int OFF_BAR = OFF_W + 2 * W_BYTES;
+  static constexpr int NBAR = 2 * NA + 8;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
+  static_assert(D == 128 || D == 64, "row = one swizzle atom");
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
+  static_assert(COLS % 32 == 0 && (COLS % H == 0 || H % COLS == 0), "epilogue split");
+  static_assert(H <= COLS, "a query's heads stay in one warp");
+  static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "tile alignment");
+};
+
+struct ItemGeom {
+  int b, t0, nq, kt0, kt1;
+};
+
+// Decodes work item `it` and returns false when it holds no visible key tile.
+__device__ __forceinline__ bool item_geom(int it, int QB, int nqb, int nkc, int T, int t_begin, int t_count,
+                                          int S_max, int pool, const int32_t* __restrict__ ctx_len, ItemGeom& g) {
+  const int kc = it % nkc;
+  const int r = it / nkc;
+  const int qb = r % nqb;
+  g.b = r / nqb;
+  g.t0 = t_begin + qb * QB;
+  g.nq = min(QB, t_begin + t_count - g.t0);
+  const int pos_last = __ldg(ctx_len + g.b) - T + g.t0 + g.nq - 1;
+  if (pos_last < 0) return false;
+  const int n_valid = min(S_max, pos_last / pool + 1);
+  const int ntiles = (n_valid + KTILE - 1) / KTILE;
+  g.kt0 = kc * KC;
+  g.kt1 = min(g.kt0 + KC, ntiles);
+  return g.kt0 < g.kt1;
+}
+
+template <int H, int D, int QB>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
+                       const float* __restrict__ w, const int32_t* __restrict__ ctx_len, int B, int T, int S_max,
+                       int pool, int t_begin, int t_count, float* __restrict__ scores, int64_t ld) {
+  using C = IdxCfg<H, D, QB>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sbase = (sraw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - sraw);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  auto a_full = [&](int s) { return bar0 + 8u * s; };
+  auto a_empty = [&](int s) { return bar0 + 8u * (NA + s); };
+  auto b_full = [&](int s) { return bar0 + 8u * (2 * NA + s); };
+  auto b_empty = [&](int s) { return bar0 + 8u * (2 * NA + 2 + s); };
+  auto acc_full = [&](int s) { return bar0 + 8u * (2 * NA + 4 + s); };
+  auto acc_empty = [&](int s) { return bar0 + 8u * (2 * NA + 6 + s); };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + C::OFF_MISC);
+  volatile int* abort = reinterpret_cast<volatile int*>(sgen + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqb = (t_count + QB - 1) / QB;
+  const int nkc = ((S_max + KTILE - 1) / KTILE + KC - 1) / KC;
+  const int items = B * nqb * nkc;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NA; ++i) {
+      mbar_init(a_full(i), 1);
+      mbar_init(a_empty(i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(b_full(i), 1);
+      mbar_init(b_empty(i), 1 + 4 * C::HALVES);  // MMA commit + every epilogue warp
+      mbar_init(acc_full(i), 1);
+      mbar_init(acc_empty(i), 4 * C::HALVES);
+    }
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_q);
+    }
+    uint32_t a_cnt = 0, b_cnt = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
+      ItemGeom g;
+      if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g)) continue;
+      const int bs = b_cnt & 1;
+      if (!(ok = mbar_wait(b_empty(bs), ((b_cnt >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
+      if (lane == 0) {
+        const uint32_t wbytes = (uint32_t)(g.nq * H * 4);
+        mbar_arrive_expect_tx(b_full(bs), C::B_BYTES + wbytes);
+        tma_load_2d(sbase + C::OFF_B + bs * C::B_BYTES, &tmap_q, b_full(bs), 0, (g.b * T + g.t0) * H);
+        bulk_load(sbase + C::OFF_W + bs * C::W_BYTES, w + ((int64_t)g.b * T + g.t0) * H, wbytes, b_full(bs));
+      }
+      ++b_cnt;
+      for (int kt = g.kt0; kt < g.kt1; ++kt) {
+        const int as = a_cnt % NA;
+        if (!(ok = mbar_wait(a_empty(as), ((a_cnt / NA) & 1) ^ 1, abort, kWaitLimitNs))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(a_full(as), C::A_BYTES);
+          tma_load_2d(sbase + C::OFF_A + as * C::A_BYTES, &tmap_k, a_full(as), 0, g.b * S_max + kt * KTILE);
+        }
+        ++a_cnt;
+      }
+      __syncwarp();
+    }
+    if (!ok) {  // drain the copies this warp issued before giving up (bounded waits)
+      for (uint32_t i = (a_cnt > NA ? a_cnt - NA : 0); i < a_cnt; ++i)
+        mbar_wait_bounded(a_full(i % NA), (i / NA) & 1, 100000000ull);
+      for (uint32_t i = (b_cnt > 2 ? b_cnt - 2 : 0); i < b_cnt; ++i)
+        mbar_wait_bounded(b_full(i & 1), (i >> 1) & 1, 100000000ull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    uint32_t a_cnt = 0, b_cnt = 0, acc_cnt = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
+      ItemGeom g;
+      if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g)) continue;
+      const int bs = b_cnt & 1;
+      if (!(ok = mbar_wait(b_full(bs), (b_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
+      const uint32_t b_addr = sbase + C::OFF_B + bs * C::B_BYTES;
+      for (int kt = g.kt0; kt < g.kt1; ++kt) {
+        const int as = a_cnt % NA;
+        const int ab = acc_cnt & 1;
+        if (!(ok = mbar_wait(a_full(as), (a_cnt / NA) & 1, abort, kWaitLimitNs))) break;
+        if (!(ok = mbar_wait(acc_empty(ab), ((acc_cnt >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a_addr = sbase + C::OFF_A + as * C::A_BYTES;
+          const uint32_t d_tmem = tmem_base + (uint32_t)(ab * C::N);
+#pragma unroll
+          for (int k = 0; k < D / 32; ++k) {
+            mma_f8(d_tmem, smem_desc(a_addr + 32 * k, C::SBO, C::LAYOUT), smem_desc(b_addr + 32 * k, C::SBO, C::LAYOUT),
+                   C::IDESC, k > 0 ? 1u : 0u);
+          }
+          mma_commit(a_empty(as));
+          mma_commit(acc_full(ab));
+        }
+        __syncwarp();
+        ++a_cnt;
+        ++acc_cnt;
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(b_empty(bs));
+      __syncwarp();
+      ++b_cnt;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (8 warps)
+    const int quad = warp & 3;          // TMEM lanes 32*quad .. +31
+    const int half = (warp - 2) >> 2;   // column half
+    const int row = quad * 32 + lane;   // key within the tile
+    uint32_t b_cnt = 0, acc_cnt = 0;
+    bool ok = true;
+    // warps beyond the accumulator's column halves take no part (the barriers count only
+    // the active ones)
+    for (int it = blockIdx.x; half < C::HALVES && it < items && ok; it += gridDim.x) {
+      ItemGeom g;
+      if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g)) continue;
+      const int bs = b_cnt & 1;
+      if (!(ok = mbar_wait(b_full(bs), (b_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
+      const float* wsm = reinterpret_cast<const float*>(sgen + C::OFF_W + bs * C::W_BYTES) + half * C::COLS;
+      const int ctx_b = __ldg(ctx_len + g.b);
+      for (int kt = g.kt0; kt < g.kt1; ++kt) {
+        const int ab = acc_cnt & 1;
+        if (!(ok = mbar_wait(acc_full(ab), (acc_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
+        tc_fence_after();
+        {
+          float acc[C::QPH];
+#pragma unroll
+          for (int q = 0; q < C::QPH; ++q) acc[q] = 0.f;
+          const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(ab * C::N + half * C::COLS);
+#pragma unroll
+          for (int c = 0; c < C::CHUNKS; ++c) {
+            float v[32];
+            tmem_ld32(taddr + 32 * c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 wv = *reinterpret_cast<const float4*>(wsm + 32 * c + i);
+              const int ql = (32 * c + i) / H;   // compile-time after unrolling
+              acc[ql] = fmaf(wv.x, fmaxf(v[i + 0], 0.f), acc[ql]);
+              acc[ql] = fmaf(wv.y, fmaxf(v[i + 1], 0.f), acc[ql]);
+              acc[ql] = fmaf(wv.z, fmaxf(v[i + 2], 0.f), acc[ql]);
+              acc[ql] = fmaf(wv.w, fmaxf(v[i + 3], 0.f), acc[ql]);
+            }
+          }
+          const int s = kt * KTILE + row;
+#pragma unroll
+          for (int q = 0; q < C::QPH; ++q) {
+            const int qq = half * C::QPH + q;
+            if (qq < g.nq && s < S_max) {
+              const int t = g.t0 + qq;
+              const int pos = ctx_b - T + t;
+              const float val = (s * pool <= pos) ? acc[q] : -INFINITY;
+              scores[((int64_t)g.b * t_count + (t - t_begin)) * ld + s] = val;
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty(ab));
+        ++acc_cnt;
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_empty(bs));
+      ++b_cnt;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D uint8 tensor map: `rows` rows of `row_bytes`, boxes of box_rows x row_bytes.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t row_bytes, uint32_t box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {row_bytes, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int H, int D, int QB>
+int launch_tc(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* ctx_len, int B, int T,
+              int S_max, int pool, int t_begin, int t_count, float* scores, int64_t ld, cudaStream_t stream) {
+  using C = IdxCfg<H, D, QB>;
+  CUtensorMap mk, mq;
+  if (!make_map(&mk, k_idx, (uint64_t)B * S_max, D, KTILE)) return DSA_ERR_CUDA;
+  if (!make_map(&mq, q_idx, (uint64_t)B * T * H, D, C::N)) return DSA_ERR_CUDA;
+  auto kern = index_scores_tc_kernel<H, D, QB>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  const int nqb = (t_count + QB - 1) / QB;
+  const int nkc = ((S_max + KTILE - 1) / KTILE + KC - 1) / KC;
+  const int64_t items = (int64_t)B * nqb * nkc;
+  const int grid = (int)std::min<int64_t>(items, num_sms());
+  kern<<<grid, NUM_THREADS, C::SMEM, stream>>>(mk, mq, w, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld);
+  return check_launch();
+}
+
+}  // namespace
+
+int launch_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* ctx_len, int B,
+                        int T, int S_max, int H_I, int d_I, int pool, int t_begin, int t_count, float* scores,
+                        int64_t ld, cudaStream_t stream) {
+  if (B == 0 || t_count == 0 || S_max == 0) return DSA_OK;
+  if (H_I == 64 && d_I == 128) {
+    if (t_count < 4)  // decode-like: one query per block keeps the MMA N at the head count
+      return launch_tc<64, 128, 1>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, stream);
+    return launch_tc<64, 128, 4>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, stream);
+  }
+  if (H_I == 4 && d_I == 64)
+    return launch_tc<4, 64, 64>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, stream);
+  return DSA_ERR_UNSUPPORTED_SHAPE;
+}
+
+namespace {
+// Test hook: one thread waits on an mbarrier that nothing ever arrives at, through the same
+// bounded wait the tensor-core kernels use, so the time limit runs out and the device
+// status word is set.  The kernel then returns normally; the context stays usable.
+__global__ void wait_timeout_probe_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = smem_u32(&bar);
+  abort_flag = 0;
+  mbar_init(b, 1);
+  fence_barrier_init();
+  mbar_wait(b, 0, &abort_flag, limit_ns);
+}
+}  // namespace
+
+int launch_wait_timeout_probe(uint64_t limit_ns, cudaStream_t stream) {
+  wait_timeout_probe_kernel<<<1, 1, 0, stream>>>(limit_ns);
+  return check_launch();
+}
+
+// Reads and clears the indexer's device status word (bit 0: a bounded wait gave up).
+unsigned int indexer_take_status() {
+  unsigned int v = 0, zero = 0;
+  cudaMemcpyFromSymbol(&v, g_status, sizeof(v));
+  if (v) cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
+  return v;
+}
+
+}  // namespace dsa

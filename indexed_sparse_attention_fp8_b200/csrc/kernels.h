@@ -22,6 +22,11 @@ int launch_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v,
                        int d_v, int k, float sm_scale, uint16_t* out, float* lse, void* ws,
                        cudaStream_t stream);
 
+// Reads and clears the device status word of the tensor-core indexer.
+unsigned int indexer_take_status();
+// Launches the bounded-wait probe (see dsa_debug_wait_timeout).
+int launch_wait_timeout_probe(uint64_t limit_ns, cudaStream_t stream);
+
 int launch_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, uint8_t* k_pool,
                       cudaStream_t stream);
 

@@ -16,6 +16,12 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
+@pytest.fixture(autouse=True)
+def _no_device_timeouts():
+    yield
+    assert dsa.dsa_device_status() == 0, "a kernel gave up a bounded wait"
+
+
 def _inputs(wl, layers=4):
     ind = W.make_indexer_inputs(wl, device=DEV)
     lays = [W.make_attn_inputs(wl, l, device=DEV) for l in range(layers)]
