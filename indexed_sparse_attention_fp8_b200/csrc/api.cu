@@ -149,7 +149,9 @@ int dsa_device_status(void* stream) {
     set_cuda_error(e);
     return DSA_ERR_CUDA;
   }
-  return indexer_take_status() ? DSA_ERR_TIMEOUT : DSA_OK;
+  const unsigned int a = indexer_take_status();
+  const unsigned int b = attn_tc_take_status();
+  return (a | b) ? DSA_ERR_TIMEOUT : DSA_OK;
 }
 uint64_t dsa_launch_count(void) { return g_launches; }
 

@@ -311,6 +311,17 @@ attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ 
   if (lse != nullptr && threadIdx.x == 0) lse[row] = wsum > 0.f ? mx + __logf(wsum) : -INFINITY;
 }
 
+}  // namespace
+
+int launch_attn_combine(const float* part_o, const float* part_lse, int splits, int64_t rows, int d_v,
+                        uint16_t* out, float* lse, cudaStream_t stream) {
+  attn_combine_kernel<<<(unsigned)rows, 128, 0, stream>>>(part_o, part_lse, splits, rows, d_v,
+                                                         reinterpret_cast<__nv_bfloat16*>(out), lse);
+  return check_launch();
+}
+
+namespace {
+
 template <int D_QK, int D_V, int HG, bool LATENT>
 int launch_cfg(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t kv_rs, int64_t kv_bs,
                int64_t v_rs, int64_t v_bs, const int32_t* idx, int B, int T, int Hq, int k,
@@ -342,9 +353,7 @@ int launch_cfg(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t
       scale_log2, reinterpret_cast<__nv_bfloat16*>(out), lse, part_o, part_lse);
   int st = check_launch();
   if (st != DSA_OK || splits == 1) return st;
-  attn_combine_kernel<<<(unsigned)rows, 128, 0, stream>>>(part_o, part_lse, splits, rows, D_V,
-                                                         reinterpret_cast<__nv_bfloat16*>(out), lse);
-  return check_launch();
+  return launch_attn_combine(part_o, part_lse, splits, rows, D_V, out, lse, stream);
 }
 
 }  // namespace
@@ -369,10 +378,9 @@ int launch_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v,
                        void* ws, cudaStream_t stream) {
   if (B == 0 || T == 0) return DSA_OK;
   if (Hq == 128 && d_qk == 576 && d_v == 512) {
-    // MLA latent form only: V must be the first d_v columns of the K row
+    // MLA latent form only: V must be the first d_v columns of the K row (tensor-core kernel)
     if (v != nullptr) return DSA_ERR_UNSUPPORTED_SHAPE;
-    return launch_cfg<576, 512, 64, true>(q, kv, v, kv_rs, kv_bs, v_rs, v_bs, idx, B, T, Hq, k,
-                                          sm_scale, out, lse, ws, stream);
+    return launch_sparse_mla_tc(q, kv, kv_rs, kv_bs, idx, B, T, k, sm_scale, out, lse, ws, stream);
   }
   if (Hq == 16 && d_qk == 128 && d_v == 128) {
     if (v == nullptr)

@@ -27,6 +27,15 @@ unsigned int indexer_take_status();
 // Launches the bounded-wait probe (see dsa_debug_wait_timeout).
 int launch_wait_timeout_probe(uint64_t limit_ns, cudaStream_t stream);
 
+// Tensor-core sparse MLA attention (128 heads, latent 576 / V 512); same split rule.
+int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, int64_t kv_bs, const int32_t* idx,
+                         int B, int T, int k, float sm_scale, uint16_t* out, float* lse, void* ws,
+                         cudaStream_t stream);
+unsigned int attn_tc_take_status();
+// Merges split-key attention partials (normalised fp32 O and log-sum-exp per split).
+int launch_attn_combine(const float* part_o, const float* part_lse, int splits, int64_t rows, int d_v,
+                        uint16_t* out, float* lse, cudaStream_t stream);
+
 int launch_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, uint8_t* k_pool,
                       cudaStream_t stream);
 
