@@ -178,7 +178,8 @@ def run_ours(args, rank, world, dev):
     stream = torch.cuda.current_stream()
     pk = peaks()
     wl = W.WORKLOADS[args.workload]
-    # q/out aliasing across layers would change no work; memory allows distinct tensors except at 128K
+    if args.T:
+        wl = wl.replace(T=args.T)
     ind, lays = make_group(wl, dev, dsa)
     g = dsa.Group(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk, lays, wl.sm_scale, wl.d_v,
                   pool=wl.pool)
@@ -459,6 +460,7 @@ def main():
     ap.add_argument("--workload", default="prefill128k", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--t-chunk", type=int, default=0)
+    ap.add_argument("--T", type=int, default=0, help="override the number of new queries (small profiling cases)")
     ap.add_argument("--score-ws-gb", type=int, default=8, help="GiB of workspace for indexer score chunks")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
@@ -502,7 +504,7 @@ def main():
         except torch.cuda.OutOfMemoryError as e:  # pragma: no cover
             res["per_layer_indexer"] = {"error": str(e)[:200]}
         res["decode256k"] = run_secondary(args, "decode256k", dev, steps=10)
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
         v, rows, cores, spent = oracle_sample(W.WORKLOADS[args.workload], args.cpu_seconds)
         res["cpu_baseline"] = {"value": v, "unit": "query tok/s", "cores": cores, "kind": "oracle",
                                "sample": f"{rows} query rows of {args.workload} in {spent:.1f}s (indexer row + "

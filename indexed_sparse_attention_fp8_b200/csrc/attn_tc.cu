@@ -39,8 +39,9 @@ constexpr int KV_STAGE = KB * K_BLK;                // 36864
 constexpr int OFF_P = OFF_KV + 2 * KV_STAGE;        // 221184
 constexpr int P_BYTES = HQ * NK * 2;                // 8192 (rows of 64 B, 64-byte swizzle)
 constexpr int OFF_BAR = OFF_P + P_BYTES;            // 229376
-constexpr int NBARS = 10;
-constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+constexpr int NBARS = 12;
+constexpr int OFF_IDS = OFF_BAR + NBARS * 8;          // two stages of NK selected ids
+constexpr int OFF_MISC = OFF_IDS + 2 * NK * 4;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;    // + alignment slack
 constexpr int THREADS = 288;
 constexpr int GATHER_THREADS = 128;
@@ -95,6 +96,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   auto s_empty = [&](int s) { return bar0 + 8u * (6 + s); };
   const uint32_t p_full = bar0 + 8u * 8;
   const uint32_t pv_done = bar0 + 8u * 9;
+  auto ids_ready = [&](int s) { return bar0 + 8u * (10 + s); };
+  volatile int* ids_s = reinterpret_cast<volatile int*>(sgen + OFF_IDS);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(sgen + OFF_MISC + 4);
 
@@ -117,6 +120,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     }
     mbar_init(p_full, 4);
     mbar_init(pv_done, 1);
+    mbar_init(ids_ready(0), 1);
+    mbar_init(ids_ready(1), 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -131,26 +136,50 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ gather (cp.async)
-    const int gt = threadIdx.x - 128;
+    // Warp gw copies rows gw, gw+4, ..: lane l moves 16-byte chunks l, l+32, l+64 of a row,
+    // so each row is read with coalesced requests.  A tile's 32 ids come from one coalesced
+    // load per warp, issued a tile ahead, and reach the rows through shuffles.
+    const int gw = warp - 4;
     const __nv_bfloat16* qrow = q + (int64_t)bt * HQ * DQK;
-    for (int i = gt; i < HQ * ROWCH; i += GATHER_THREADS) {
-      const int r = i / ROWCH, c = i % ROWCH;
-      const uint32_t dst = sbase + OFF_Q + (c >> 3) * Q_BLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-      cp_async16(dst, qrow + (int64_t)r * DQK + c * 8, 16);
+    for (int r = gw; r < HQ; r += 4) {
+      const __nv_bfloat16* src = qrow + (int64_t)r * DQK;
+      for (int c = lane; c < ROWCH; c += 32) {
+        const uint32_t dst = sbase + OFF_Q + (c >> 3) * Q_BLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+        cp_async16(dst, src + c * 8, 16);
+      }
     }
     const __nv_bfloat16* kvb = kv + (int64_t)b * kv_bs;
+    auto load_id = [&](int j) -> int {
+      const int p = kbeg + j * NK + lane;
+      return (j < ntiles && p < kend) ? __ldg(irow + p) : -1;
+    };
+    int id_next = load_id(0);
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int st = j & 1;
+      const int id_cur = id_next;
+      id_next = load_id(j + 1);
       if (!(ok = mbar_wait(kv_empty(st), ((j >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
+      if (gw == 0) {   // publish the tile's ids for the softmax warps
+        ids_s[st * NK + lane] = id_cur;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ids_ready(st));
+      }
       const uint32_t stage = sbase + OFF_KV + st * KV_STAGE;
-      const int p0 = kbeg + j * NK;
-      for (int i = gt; i < NK * ROWCH; i += GATHER_THREADS) {
-        const int r = i / ROWCH, c = i % ROWCH;
-        const int p = p0 + r;
-        const int key = p < kend ? __ldg(irow + p) : -1;
-        const uint32_t dst = stage + (c >> 3) * K_BLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-        cp_async16(dst, kvb + (int64_t)(key < 0 ? 0 : key) * kv_rs + c * 8, key < 0 ? 0 : 16);
+#pragma unroll
+      for (int i = 0; i < NK / 4; ++i) {
+        const int r = gw + 4 * i;
+        const int key = __shfl_sync(0xffffffffu, id_cur, r);
+        const __nv_bfloat16* src = kvb + (int64_t)(key < 0 ? 0 : key) * kv_rs;
+        const int nbytes = key < 0 ? 0 : 16;
+#pragma unroll
+        for (int cc = 0; cc < 3; ++cc) {
+          const int c = lane + 32 * cc;
+          if (c < ROWCH) {
+            const uint32_t dst = stage + (c >> 3) * K_BLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+            cp_async16(dst, src + c * 8, nbytes);
+          }
+        }
       }
       // one arrival per gather thread, triggered when all its copies so far (q too) have landed
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(kv_full(st)) : "memory");
@@ -203,7 +232,6 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     const int row = warp * 32 + lane;  // head
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     float m_use = -INFINITY, l_run = 0.f;
-    const bool vec_ids = (k & 3) == 0;   // 16-byte id loads need rows that start 16-byte aligned
     bool ok = true;
     const uint32_t prow = sbase + OFF_P + row * 64;
     for (int j = 0; j < ntiles; ++j) {
@@ -217,24 +245,12 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       __syncwarp();
       if (lane == 0) mbar_arrive(s_empty(st));
       // mask skipped ids (negative entries and the ragged end), scale to the log2 domain
-      const int p0 = kbeg + j * NK;
+      if (!(ok = mbar_wait(ids_ready(st), (j >> 1) & 1, abort, kWaitLimitNs))) break;
       float mt = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        int4 id4;
-        if (vec_ids && p0 + i + 3 < kend) {
-          id4 = __ldg(reinterpret_cast<const int4*>(irow + p0 + i));
-        } else {
-          id4.x = p0 + i + 0 < kend ? __ldg(irow + p0 + i + 0) : -1;
-          id4.y = p0 + i + 1 < kend ? __ldg(irow + p0 + i + 1) : -1;
-          id4.z = p0 + i + 2 < kend ? __ldg(irow + p0 + i + 2) : -1;
-          id4.w = p0 + i + 3 < kend ? __ldg(irow + p0 + i + 3) : -1;
-        }
-        s[i + 0] = id4.x >= 0 ? s[i + 0] * scale_log2 : -INFINITY;
-        s[i + 1] = id4.y >= 0 ? s[i + 1] * scale_log2 : -INFINITY;
-        s[i + 2] = id4.z >= 0 ? s[i + 2] * scale_log2 : -INFINITY;
-        s[i + 3] = id4.w >= 0 ? s[i + 3] * scale_log2 : -INFINITY;
-        mt = fmaxf(mt, fmaxf(fmaxf(s[i], s[i + 1]), fmaxf(s[i + 2], s[i + 3])));
+      for (int i = 0; i < 32; ++i) {
+        s[i] = ids_s[st * NK + i] >= 0 ? s[i] * scale_log2 : -INFINITY;
+        mt = fmaxf(mt, s[i]);
       }
       // P of the previous tile must have been consumed (and O be stable) before writing P
       if (j >= 1 && !(ok = mbar_wait(pv_done, (j - 1) & 1, abort, kWaitLimitNs))) break;

@@ -229,35 +229,57 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
         if (!(ok = mbar_wait(acc_full(ab), (acc_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
         tc_fence_after();
         {
-          float acc[C::QPH];
-#pragma unroll
-          for (int q = 0; q < C::QPH; ++q) acc[q] = 0.f;
           const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(ab * C::N + half * C::COLS);
-#pragma unroll
-          for (int c = 0; c < C::CHUNKS; ++c) {
-            float v[32];
-            tmem_ld32(taddr + 32 * c, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const float4 wv = *reinterpret_cast<const float4*>(wsm + 32 * c + i);
-              const int ql = (32 * c + i) / H;   // compile-time after unrolling
-              acc[ql] = fmaf(wv.x, fmaxf(v[i + 0], 0.f), acc[ql]);
-              acc[ql] = fmaf(wv.y, fmaxf(v[i + 1], 0.f), acc[ql]);
-              acc[ql] = fmaf(wv.z, fmaxf(v[i + 2], 0.f), acc[ql]);
-              acc[ql] = fmaf(wv.w, fmaxf(v[i + 3], 0.f), acc[ql]);
-            }
-          }
           const int s = kt * KTILE + row;
-#pragma unroll
-          for (int q = 0; q < C::QPH; ++q) {
-            const int qq = half * C::QPH + q;
+          // finished sum of query ql (local to this warp) -> masked store
+          auto store = [&](int ql, float val) {
+            const int qq = half * C::QPH + ql;
             if (qq < g.nq && s < S_max) {
               const int t = g.t0 + qq;
               const int pos = ctx_b - T + t;
-              const float val = (s * pool <= pos) ? acc[q] : -INFINITY;
-              scores[((int64_t)g.b * t_count + (t - t_begin)) * ld + s] = val;
+              scores[((int64_t)g.b * t_count + (t - t_begin)) * ld + s] = (s * pool <= pos) ? val : -INFINITY;
             }
+          };
+          // w * relu(x) over 4 columns into two packed accumulators
+          auto quad4 = [&](const float* v, int col, uint64_t& a0, uint64_t& a1) {
+            const float4 wv = *reinterpret_cast<const float4*>(wsm + col);
+            a0 = ffma2(pack2(wv.x, wv.y), pack2(fmaxf(v[0], 0.f), fmaxf(v[1], 0.f)), a0);
+            a1 = ffma2(pack2(wv.z, wv.w), pack2(fmaxf(v[2], 0.f), fmaxf(v[3], 0.f)), a1);
+          };
+          float v[2][32];
+          tmem_ld32(taddr, v[0]);
+          tmem_ld_wait();
+          uint64_t a2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+          for (int c = 0; c < C::CHUNKS; ++c) {
+            if (c + 1 < C::CHUNKS) tmem_ld32(taddr + 32 * (c + 1), v[(c + 1) & 1]);   // in flight during c
+            const float* vc = v[c & 1];
+            if constexpr (H >= 32) {
+              // a query spans H/32 chunks: 4 packed partial sums, chains of H/16 FMAs
+#pragma unroll
+              for (int i = 0; i < 32; i += 8) {
+                quad4(vc + i, 32 * c + i, a2[0], a2[1]);
+                quad4(vc + i + 4, 32 * c + i + 4, a2[2], a2[3]);
+              }
+              if ((c + 1) % (H / 32) == 0) {
+                float x0, x1, x2, x3, x4, x5, x6, x7;
+                unpack2(a2[0], x0, x1); unpack2(a2[1], x2, x3); unpack2(a2[2], x4, x5); unpack2(a2[3], x6, x7);
+                store(c / (H / 32), ((x0 + x1) + (x2 + x3)) + ((x4 + x5) + (x6 + x7)));
+                a2[0] = a2[1] = a2[2] = a2[3] = 0ull;
+              }
+            } else {
+              // 32/H whole queries per chunk
+#pragma unroll
+              for (int qc = 0; qc < 32 / H; ++qc) {
+                uint64_t b0 = 0ull, b1 = 0ull;
+#pragma unroll
+                for (int i = 0; i < H; i += 4) quad4(vc + qc * H + i, 32 * c + qc * H + i, b0, b1);
+                float x0, x1, x2, x3;
+                unpack2(b0, x0, x1); unpack2(b1, x2, x3);
+                store(c * (32 / H) + qc, (x0 + x1) + (x2 + x3));
+              }
+            }
+            if (c + 1 < C::CHUNKS) tmem_ld_wait();
           }
         }
         tc_fence_before();
