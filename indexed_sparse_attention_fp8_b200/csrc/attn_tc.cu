@@ -3,21 +3,28 @@
 // the selected tokens only).  All 128 query heads of a token share one latent row per key:
 // K = the 576-wide row, V = its first 512 columns.
 //
-// TMEM holds 128 lanes x 512 fp32 columns, exactly the size of O = 128 heads x 512 dv, so one
-// CTA cannot keep O and the scores together.  Each query is therefore served by a pair of
-// CTAs: both compute the full score tile S = q K^T (M = 128 heads), and CTA h accumulates
-// O[:, 256h .. 256h+255].  Per CTA, TMEM = 2 x 32 score columns + 256 output columns.
+// TMEM holds 128 lanes x 512 fp32 columns, exactly the size of O = 128 heads x 512 dv, so a
+// query is served by a cluster of two CTAs.  CTA c (c = 0, 1):
+//   * holds q[:, 288c .. 288c+287] in TMEM (the MMA's A operand, so no shared-memory
+//     bandwidth goes to re-reading q) and computes the partial scores over those 288 columns
+//     (18 x tcgen05.mma M128 N32 K16 per tile of 32 keys), then swaps its partial with the
+//     partner through distributed shared memory; both add the two partials in the same
+//     order, so both hold the same scores, softmax and P;
+//   * accumulates O[:, 256c .. 256c+255] = P V in TMEM (2 x M128 N256 K16 per tile, V read
+//     MN-major straight from the gathered rows);
+//   * gathers only the row columns it needs: c = 0 columns 0..287, c = 1 columns 256..575.
+// Per CTA: an 8-stage ring of 20 KB key tiles; TMEM 2 x 32 score + 144 q + 256 output columns.
 //
-//   warps 0-3  softmax: thread = head.  Loads its S row from TMEM, masks skipped ids, keeps a
-//              running max that is only moved when a tile exceeds it by more than 2^8 (then O
-//              is rescaled in TMEM), writes P = exp2(S - m) as bf16 to shared memory, and at
-//              the end normalises O and writes the output (or a split partial).
-//   warps 4-7  gather: 16-byte cp.async of the selected latent rows into a 2-stage ring laid
-//              out as the tensor core's 128-byte-swizzled K-major tile (which is also V's
-//              MN-major tile), plus q once.
-//   warp 8     TMEM owner and MMA issuer: S_j = q K_j^T (36 x M128 N32 K16), then
-//              O += P_{j-1} V_{j-1} (2 x M128 N256 K16, V read MN-major from the same rows).
-// All waits are bounded (see tc_common.cuh).
+//   warps 0-3  softmax: thread = head.  Partial scores from TMEM -> partner; partner's partial
+//              + own -> masked scores; running max moved only when a tile exceeds it by more
+//              than 2^8 (then O is rescaled in TMEM); P = exp2(S - m) as bf16 in shared
+//              memory; at the end O / l is written out (or a split partial with its lse).
+//              First, each thread stores its head's q columns into TMEM.
+//   warps 4-7  gather: 16-byte cp.async of the selected rows into the 128-byte-swizzled
+//              K-major layout the tensor core reads (also V's MN-major layout).
+//   warp 8     TMEM owner and MMA issuer.
+// Every wait is bounded (tc_common.cuh); the two CTAs meet at cluster barriers only at start
+// and end.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -28,42 +35,42 @@ namespace {
 using namespace tc;
 
 constexpr int HQ = 128, DQK = 576, DV = 512, DVH = 256;
-constexpr int NK = 32;                  // keys per tile (MMA N of the score product)
-constexpr int KB = DQK / 64;            // 64-column blocks of a row (9)
-constexpr int ROWCH = DQK / 8;          // 16-byte chunks per row (72)
-constexpr int Q_BLK = HQ * 128;         // one 64-column block of q: 128 rows x 128 B
-constexpr int K_BLK = NK * 128;         // one 64-column block of a key tile: 32 rows x 128 B
-constexpr int OFF_Q = 0;
-constexpr int OFF_KV = OFF_Q + KB * Q_BLK;          // 147456
-constexpr int KV_STAGE = KB * K_BLK;                // 36864
-constexpr int OFF_P = OFF_KV + 2 * KV_STAGE;        // 221184
-constexpr int P_BYTES = HQ * NK * 2;                // 8192 (rows of 64 B, 64-byte swizzle)
-constexpr int OFF_BAR = OFF_P + P_BYTES;            // 229376
-constexpr int NBARS = 12;
-constexpr int OFF_IDS = OFF_BAR + NBARS * 8;          // two stages of NK selected ids
-constexpr int OFF_MISC = OFF_IDS + 2 * NK * 4;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;    // + alignment slack
+constexpr int NK = 32;                  // keys per tile
+constexpr int NS = 8;                   // key-tile stages
+constexpr int BLKS = 5;                 // 64-column blocks of a key row held per CTA
+constexpr int K_BLK = NK * 128;         // 32 rows x 128 B
+constexpr int KSTEPS = 18;              // 288 score columns / 16 per MMA
+constexpr int KV_STAGE = BLKS * K_BLK;                 // 20480
+constexpr int OFF_KV = 0;
+constexpr int OFF_P = OFF_KV + NS * KV_STAGE;          // 163840
+constexpr int P_BYTES = HQ * NK * 2;                   // 8192: rows of 64 B, 64-byte swizzle
+constexpr int OFF_X = OFF_P + P_BYTES;                 // partner's partial scores, 2 buffers
+constexpr int X_BYTES = HQ * NK * 4;                   // 16384
+constexpr int OFF_IDS = OFF_X + 2 * X_BYTES;
+constexpr int OFF_BAR = OFF_IDS + NS * NK * 4;
+constexpr int NBARS = 4 * NS + 11;
+constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;       // + alignment slack
 constexpr int THREADS = 288;
 constexpr int GATHER_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_S = 0;      // two score buffers of NK columns
+constexpr uint32_t COL_S = 0;      // two partial-score buffers of NK columns
+constexpr uint32_t COL_Q = 64;     // this CTA's 288 q columns as packed bf16 pairs: 144 columns
 constexpr uint32_t COL_O = 256;    // DVH output columns
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr float kRescaleLog2 = 8.0f;   // move the running max only when it grows by > 2^8
+constexpr float kRescaleLog2 = 8.0f;
 
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert((OFF_P % 1024) == 0 && (OFF_KV % 1024) == 0, "operand tiles must be swizzle-atom aligned");
 
 constexpr uint32_t IDESC_S = instr_desc(128, NK, 1);                   // bf16, K-major A and B
 constexpr uint32_t IDESC_PV = instr_desc(128, DVH, 1) | (1u << 16);    // B (V) MN-major
 
-// Descriptor with an explicit leading byte offset (MN-major operands).
 __device__ __forceinline__ uint64_t smem_desc_lbo(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1u << 46) | ((uint64_t)layout << 61);
 }
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -73,14 +80,87 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]),
       "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31]));
 }
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31]));
+}
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]));
+}
+// D[tmem] (+)= A[tmem] x B[smem desc]^T, bf16 inputs, fp32 accumulation (A read from TMEM:
+// row m in lane m, element k of the row at column k/2, even k in the low half).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
-
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+// ---- cluster (distributed shared memory) helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait on a local barrier that the partner CTA completes (cluster-scope acquire).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 31u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        atomicOr(&g_status, 1u);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
+__global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(THREADS, 1)
 sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv, int64_t kv_rs,
                      int64_t kv_bs, const int32_t* __restrict__ idx, int T, int k, int keys_per_split,
                      float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
@@ -91,37 +171,48 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   uint8_t* sgen = smem_raw + (sbase - sraw);
   const uint32_t bar0 = sbase + OFF_BAR;
   auto kv_full = [&](int s) { return bar0 + 8u * s; };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (2 + s); };
-  auto s_full = [&](int s) { return bar0 + 8u * (4 + s); };
-  auto s_empty = [&](int s) { return bar0 + 8u * (6 + s); };
-  const uint32_t p_full = bar0 + 8u * 8;
-  const uint32_t pv_done = bar0 + 8u * 9;
-  auto ids_ready = [&](int s) { return bar0 + 8u * (10 + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (NS + s); };
+  auto ids_ready = [&](int s) { return bar0 + 8u * (2 * NS + s); };
+  auto s_full = [&](int s) { return bar0 + 8u * (3 * NS + s); };
+  auto s_empty = [&](int s) { return bar0 + 8u * (3 * NS + 2 + s); };
+  auto x_full = [&](int s) { return bar0 + 8u * (3 * NS + 4 + s); };   // partner's partial landed here
+  auto x_free = [&](int s) { return bar0 + 8u * (3 * NS + 6 + s); };   // partner read what we sent it
+  const uint32_t p_full = bar0 + 8u * (3 * NS + 8);
+  const uint32_t pv_done = bar0 + 8u * (3 * NS + 9);
+  const uint32_t q_ready = bar0 + 8u * (3 * NS + 10);
   volatile int* ids_s = reinterpret_cast<volatile int*>(sgen + OFF_IDS);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(sgen + OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = (int)cluster_rank();       // 0 or 1: score columns 288*half.., output columns 256*half..
+  const uint32_t partner = (uint32_t)(half ^ 1);
   const int bt = blockIdx.x;
-  const int half = blockIdx.y;
   const int sp = blockIdx.z;
   const int b = bt / T;
   const int kbeg = sp * keys_per_split;
   const int kend = min(k, kbeg + keys_per_split);
   const int ntiles = kend > kbeg ? (kend - kbeg + NK - 1) / NK : 0;
   const int32_t* irow = idx + (int64_t)bt * k;
+  const int blk0 = half == 0 ? 0 : 4;             // first 64-column block held by this CTA
+  const int ch_lo = half == 0 ? 0 : 32;           // gathered 16-byte chunks [ch_lo, ch_hi) of a row
+  const int ch_hi = half == 0 ? 36 : 72;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(kv_full(s), GATHER_THREADS);
       mbar_init(kv_empty(s), 1);
+      mbar_init(ids_ready(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(s_full(s), 1);
       mbar_init(s_empty(s), 4);
+      mbar_init(x_full(s), 4);   // the partner's 4 softmax warps
+      mbar_init(x_free(s), 4);
     }
     mbar_init(p_full, 4);
     mbar_init(pv_done, 1);
-    mbar_init(ids_ready(0), 1);
-    mbar_init(ids_ready(1), 1);
+    mbar_init(q_ready, 4);
     *abort = 0;
     fence_barrier_init();
   }
@@ -130,24 +221,13 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // both CTAs' barriers exist before either signals the other
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ gather (cp.async)
-    // Warp gw copies rows gw, gw+4, ..: lane l moves 16-byte chunks l, l+32, l+64 of a row,
-    // so each row is read with coalesced requests.  A tile's 32 ids come from one coalesced
-    // load per warp, issued a tile ahead, and reach the rows through shuffles.
     const int gw = warp - 4;
-    const __nv_bfloat16* qrow = q + (int64_t)bt * HQ * DQK;
-    for (int r = gw; r < HQ; r += 4) {
-      const __nv_bfloat16* src = qrow + (int64_t)r * DQK;
-      for (int c = lane; c < ROWCH; c += 32) {
-        const uint32_t dst = sbase + OFF_Q + (c >> 3) * Q_BLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-        cp_async16(dst, src + c * 8, 16);
-      }
-    }
     const __nv_bfloat16* kvb = kv + (int64_t)b * kv_bs;
     auto load_id = [&](int j) -> int {
       const int p = kbeg + j * NK + lane;
@@ -156,11 +236,11 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     int id_next = load_id(0);
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      const int st = j & 1;
+      const int st = j % NS;
       const int id_cur = id_next;
       id_next = load_id(j + 1);
-      if (!(ok = mbar_wait(kv_empty(st), ((j >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
-      if (gw == 0) {   // publish the tile's ids for the softmax warps
+      if (!(ok = mbar_wait(kv_empty(st), ((j / NS) & 1) ^ 1, abort, kWaitLimitNs))) break;
+      if (gw == 0) {
         ids_s[st * NK + lane] = id_cur;
         __syncwarp();
         if (lane == 0) mbar_arrive(ids_ready(st));
@@ -173,15 +253,14 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         const __nv_bfloat16* src = kvb + (int64_t)(key < 0 ? 0 : key) * kv_rs;
         const int nbytes = key < 0 ? 0 : 16;
 #pragma unroll
-        for (int cc = 0; cc < 3; ++cc) {
-          const int c = lane + 32 * cc;
-          if (c < ROWCH) {
-            const uint32_t dst = stage + (c >> 3) * K_BLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = ch_lo + lane + 32 * cc;
+          if (c < ch_hi) {
+            const uint32_t dst = stage + ((c >> 3) - blk0) * K_BLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
             cp_async16(dst, src + c * 8, nbytes);
           }
         }
       }
-      // one arrival per gather thread, triggered when all its copies so far (q too) have landed
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(kv_full(st)) : "memory");
     }
     cp_async_wait<0>();
@@ -192,36 +271,39 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       if (!mbar_wait(p_full, jj & 1, abort, kWaitLimitNs)) return false;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t stage = sbase + OFF_KV + (jj & 1) * KV_STAGE;
+        const uint32_t stage = sbase + OFF_KV + (jj % NS) * KV_STAGE;
 #pragma unroll
         for (int kk = 0; kk < NK / 16; ++kk) {
           const uint64_t ad = smem_desc(sbase + OFF_P + kk * 32, 512, kLayoutSw64);
-          // V = this half's 256 columns: blocks 4*half .. 4*half+3 of the rows, keys 16kk..16kk+15
-          const uint64_t bd = smem_desc_lbo(stage + (4 * half) * K_BLK + kk * 2048, K_BLK, 1024, kLayoutSw128);
+          // V columns 256*half .. +255 are the stage's blocks 0..3 for both CTAs
+          const uint64_t bd = smem_desc_lbo(stage + kk * 2048, K_BLK, 1024, kLayoutSw128);
           mma_bf16(tmem + COL_O, ad, bd, IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(kv_empty(jj & 1));
+        mma_commit(kv_empty(jj % NS));
         mma_commit(pv_done);
       }
       __syncwarp();
       return true;
     };
+    const int ks0 = half * KSTEPS;
+    if (ntiles > 0) ok = mbar_wait(q_ready, 0, abort, kWaitLimitNs);
     for (int j = 0; j < ntiles && ok; ++j) {
-      const int st = j & 1;
-      if (!(ok = mbar_wait(kv_full(st), (j >> 1) & 1, abort, kWaitLimitNs))) break;
-      if (!(ok = mbar_wait(s_empty(st), ((j >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
+      const int st = j % NS, sb = j & 1;
+      if (!(ok = mbar_wait(kv_full(st), (j / NS) & 1, abort, kWaitLimitNs))) break;
+      if (!(ok = mbar_wait(s_empty(sb), ((j >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
       tc_fence_after();
       fence_proxy_async();
       if (lane == 0) {
         const uint32_t stage = sbase + OFF_KV + st * KV_STAGE;
-#pragma unroll 4
-        for (int ks = 0; ks < DQK / 16; ++ks) {
-          const uint32_t off = (ks & 3) * 32;   // 16 columns = 32 bytes inside the swizzle atom
-          const uint64_t ad = smem_desc(sbase + OFF_Q + (ks >> 2) * Q_BLK + off, 1024, kLayoutSw128);
-          const uint64_t bd = smem_desc(stage + (ks >> 2) * K_BLK + off, 1024, kLayoutSw128);
-          mma_bf16(tmem + COL_S + st * NK, ad, bd, IDESC_S, ks > 0 ? 1u : 0u);
+#pragma unroll 2
+        for (int i = 0; i < KSTEPS; ++i) {
+          const int ks = ks0 + i;                      // global 16-column step 0..35
+          const uint32_t blk = (uint32_t)((ks >> 2) - blk0);
+          const uint32_t off = (uint32_t)(ks & 3) * 32u;   // 16 columns = 32 bytes inside the atom
+          const uint64_t bd = smem_desc(stage + blk * K_BLK + off, 1024, kLayoutSw128);
+          mma_bf16_ts(tmem + COL_S + sb * NK, tmem + COL_Q + 8u * i, bd, IDESC_S, i > 0 ? 1u : 0u);
         }
-        mma_commit(s_full(st));
+        mma_commit(s_full(sb));
       }
       __syncwarp();
       if (j >= 1) ok = issue_pv(j - 1);
@@ -234,22 +316,69 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     float m_use = -INFINITY, l_run = 0.f;
     bool ok = true;
     const uint32_t prow = sbase + OFF_P + row * 64;
+    {
+      // q[head, 288*half .. +287] -> TMEM lane `head`, bf16 pairs packed per 32-bit column
+      const uint4* qsrc = reinterpret_cast<const uint4*>(q + ((int64_t)bt * HQ + row) * DQK + 288 * half);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t w[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 v = __ldg(qsrc + 8 * c + i);
+          w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+        }
+        tmem_st32u(tmem + lane_off + COL_Q + 32 * c, w);
+      }
+      uint32_t w16[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = __ldg(qsrc + 32 + i);
+        w16[4 * i] = v.x; w16[4 * i + 1] = v.y; w16[4 * i + 2] = v.z; w16[4 * i + 3] = v.w;
+      }
+      tmem_st16u(tmem + lane_off + COL_Q + 128, w16);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
     for (int j = 0; j < ntiles; ++j) {
-      const int st = j & 1;
-      if (!(ok = mbar_wait(s_full(st), (j >> 1) & 1, abort, kWaitLimitNs))) break;
+      const int sb = j & 1;
+      if (!(ok = mbar_wait(s_full(sb), (j >> 1) & 1, abort, kWaitLimitNs))) break;
       tc_fence_after();
       float s[32];
-      tmem_ld32(tmem + lane_off + COL_S + st * NK, s);
+      tmem_ld32(tmem + lane_off + COL_S + sb * NK, s);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_empty(st));
-      // mask skipped ids (negative entries and the ragged end), scale to the log2 domain
-      if (!(ok = mbar_wait(ids_ready(st), (j >> 1) & 1, abort, kWaitLimitNs))) break;
+      if (lane == 0) mbar_arrive(s_empty(sb));
+      // ---- swap partial scores with the partner (row r: 8 swizzled 16-byte chunks)
+      if (!(ok = mbar_wait_cluster(x_free(sb), ((j >> 1) & 1) ^ 1, abort))) break;
+      const uint32_t xrow_local = sbase + OFF_X + sb * X_BYTES + row * 128;
+      const uint32_t xrow_remote = map_to_cta(xrow_local, partner);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_cluster_v4(xrow_remote + ((c ^ (row & 7)) << 4), s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_cta(x_full(sb), partner));
+      if (!(ok = mbar_wait_cluster(x_full(sb), (j >> 1) & 1, abort))) break;
+      float o4[32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float4 v;
+        asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                     : "r"(xrow_local + ((c ^ (row & 7)) << 4)));
+        o4[4 * c] = v.x; o4[4 * c + 1] = v.y; o4[4 * c + 2] = v.z; o4[4 * c + 3] = v.w;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_cta(x_free(sb), partner));
+      // both CTAs add the partials in column order (cols 0..287 first), so both get the same scores
+      if (!(ok = mbar_wait(ids_ready(j % NS), (j / NS) & 1, abort, kWaitLimitNs))) break;
       float mt = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        s[i] = ids_s[st * NK + i] >= 0 ? s[i] * scale_log2 : -INFINITY;
+        const float full = half == 0 ? s[i] + o4[i] : o4[i] + s[i];
+        s[i] = ids_s[(j % NS) * NK + i] >= 0 ? full * scale_log2 : -INFINITY;
         mt = fmaxf(mt, s[i]);
       }
       // P of the previous tile must have been consumed (and O be stable) before writing P
@@ -272,7 +401,6 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         l_run *= alpha;
         m_use = mt;
       }
-      // P = exp2(s - m_use) -> bf16, 64-byte-swizzled rows of 32 keys
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
@@ -349,6 +477,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+  cluster_sync();   // neither CTA leaves while the partner may still touch its shared memory
 }
 
 }  // namespace
