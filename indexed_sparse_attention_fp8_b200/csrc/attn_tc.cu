@@ -7,18 +7,20 @@
 // query is served by a cluster of two CTAs.  CTA c (c = 0, 1):
 //   * holds q[:, 288c .. 288c+287] in TMEM (the MMA's A operand, so no shared-memory
 //     bandwidth goes to re-reading q) and computes the partial scores over those 288 columns
-//     (18 x tcgen05.mma M128 N32 K16 per tile of 32 keys), then swaps its partial with the
+//     (18 x tcgen05.mma M128 N64 K16 per tile of 64 keys), then swaps its partial with the
 //     partner through distributed shared memory; both add the two partials in the same
 //     order, so both hold the same scores, softmax and P;
 //   * accumulates O[:, 256c .. 256c+255] = P V in TMEM (2 x M128 N256 K16 per tile, V read
 //     MN-major straight from the gathered rows);
+//     (P.V: 4 x M128 N256 K16 per tile)
 //   * gathers only the row columns it needs: c = 0 columns 0..287, c = 1 columns 256..575.
-// Per CTA: an 8-stage ring of 20 KB key tiles; TMEM 2 x 32 score + 144 q + 256 output columns.
+// Per CTA: a 3-stage ring of 40 KB key tiles; TMEM 64 score + 144 q + 256 output columns.
 //
-//   warps 0-3  softmax: thread = head.  Partial scores from TMEM -> partner; partner's partial
+//   warps 0-3  softmax: thread = head.  Partial scores from TMEM -> partner (asynchronous
+//              remote stores that complete the partner's barrier); partner's partial
 //              + own -> masked scores; running max moved only when a tile exceeds it by more
-//              than 2^8 (then O is rescaled in TMEM); P = exp2(S - m) as bf16 in shared
-//              memory; at the end O / l is written out (or a split partial with its lse).
+//              than 2^8 (then O is rescaled in TMEM); P = exp2(S - m) as bf16 in one of two
+//              shared-memory buffers, so a tile's softmax overlaps the previous tile's P.V; at the end O / l is written out (or a split partial with its lse).
 //              First, each thread stores its head's q columns into TMEM.
 //   warps 4-7  gather: 16-byte cp.async of the selected rows into the 128-byte-swizzled
 //              K-major layout the tensor core reads (also V's MN-major layout).
@@ -35,33 +37,34 @@ namespace {
 using namespace tc;
 
 constexpr int HQ = 128, DQK = 576, DV = 512, DVH = 256;
-constexpr int NK = 32;                  // keys per tile
-constexpr int NS = 8;                   // key-tile stages
+constexpr int NK = 64;                  // keys per tile
+constexpr int NS = 3;                   // key-tile stages
 constexpr int BLKS = 5;                 // 64-column blocks of a key row held per CTA
-constexpr int K_BLK = NK * 128;         // 32 rows x 128 B
+constexpr int K_BLK = NK * 128;         // 64 rows x 128 B
 constexpr int KSTEPS = 18;              // 288 score columns / 16 per MMA
-constexpr int KV_STAGE = BLKS * K_BLK;                 // 20480
+constexpr int KV_STAGE = BLKS * K_BLK;                 // 40960
 constexpr int OFF_KV = 0;
-constexpr int OFF_P = OFF_KV + NS * KV_STAGE;          // 163840
-constexpr int P_BYTES = HQ * NK * 2;                   // 8192: rows of 64 B, 64-byte swizzle
-constexpr int OFF_X = OFF_P + P_BYTES;                 // partner's partial scores, 2 buffers
-constexpr int X_BYTES = HQ * NK * 4;                   // 16384
+constexpr int OFF_P = OFF_KV + NS * KV_STAGE;          // 2 P buffers: rows of 128 B (64 keys bf16)
+constexpr int P_BYTES = HQ * NK * 2;                   // 16384
+constexpr int OFF_X = OFF_P + 2 * P_BYTES;             // partner's partial scores, 2 buffers
+constexpr int X_BYTES = HQ * NK * 4;                   // 32768
 constexpr int OFF_IDS = OFF_X + 2 * X_BYTES;
 constexpr int OFF_BAR = OFF_IDS + NS * NK * 4;
-constexpr int NBARS = 4 * NS + 11;
+constexpr int NBARS = 3 * NS + 12;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;       // + alignment slack
 constexpr int THREADS = 288;
 constexpr int GATHER_THREADS = 128;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_S = 0;      // two partial-score buffers of NK columns
+constexpr uint32_t COL_S = 0;      // partial scores, NK columns
 constexpr uint32_t COL_Q = 64;     // this CTA's 288 q columns as packed bf16 pairs: 144 columns
 constexpr uint32_t COL_O = 256;    // DVH output columns
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
 
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert((OFF_P % 1024) == 0 && (OFF_KV % 1024) == 0, "operand tiles must be swizzle-atom aligned");
+static_assert((OFF_P % 1024) == 0 && (OFF_KV % 1024) == 0 && (OFF_X % 16) == 0, "alignment");
+static_assert(COL_Q + 144 <= COL_O && COL_S + NK <= COL_Q, "TMEM map");
 
 constexpr uint32_t IDESC_S = instr_desc(128, NK, 1);                   // bf16, K-major A and B
 constexpr uint32_t IDESC_PV = instr_desc(128, DVH, 1) | (1u << 16);    // B (V) MN-major
@@ -156,6 +159,18 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
     }
   }
 }
+// 16-byte asynchronous store into a cluster peer's shared memory; completes `bytes` of the
+// peer barrier's transaction count when it lands (no fence on the issuing side).
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];\n"
+               ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+               : "memory");
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
@@ -173,12 +188,12 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   auto kv_full = [&](int s) { return bar0 + 8u * s; };
   auto kv_empty = [&](int s) { return bar0 + 8u * (NS + s); };
   auto ids_ready = [&](int s) { return bar0 + 8u * (2 * NS + s); };
-  auto s_full = [&](int s) { return bar0 + 8u * (3 * NS + s); };
-  auto s_empty = [&](int s) { return bar0 + 8u * (3 * NS + 2 + s); };
-  auto x_full = [&](int s) { return bar0 + 8u * (3 * NS + 4 + s); };   // partner's partial landed here
-  auto x_free = [&](int s) { return bar0 + 8u * (3 * NS + 6 + s); };   // partner read what we sent it
-  const uint32_t p_full = bar0 + 8u * (3 * NS + 8);
-  const uint32_t pv_done = bar0 + 8u * (3 * NS + 9);
+  const uint32_t s_full = bar0 + 8u * (3 * NS);
+  const uint32_t s_empty = bar0 + 8u * (3 * NS + 1);
+  auto x_full = [&](int s) { return bar0 + 8u * (3 * NS + 2 + s); };   // partner's partial landed here
+  auto x_free = [&](int s) { return bar0 + 8u * (3 * NS + 4 + s); };   // partner read what we sent it
+  auto p_full = [&](int s) { return bar0 + 8u * (3 * NS + 6 + s); };
+  auto pv_done = [&](int s) { return bar0 + 8u * (3 * NS + 8 + s); };
   const uint32_t q_ready = bar0 + 8u * (3 * NS + 10);
   volatile int* ids_s = reinterpret_cast<volatile int*>(sgen + OFF_IDS);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + OFF_MISC);
@@ -204,14 +219,14 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       mbar_init(kv_empty(s), 1);
       mbar_init(ids_ready(s), 1);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, 4);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(s_full(s), 1);
-      mbar_init(s_empty(s), 4);
-      mbar_init(x_full(s), 4);   // the partner's 4 softmax warps
-      mbar_init(x_free(s), 4);
+      mbar_init(x_full(s), 4);   // one expect-tx arrival per softmax warp, plus the partner's bytes
+      mbar_init(x_free(s), 4);   // the partner's 4 softmax warps
+      mbar_init(p_full(s), 4);
+      mbar_init(pv_done(s), 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
     mbar_init(q_ready, 4);
     *abort = 0;
     fence_barrier_init();
@@ -221,27 +236,37 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     tmem_relinquish();
   }
   tc_fence_before();
-  cluster_sync();   // both CTAs' barriers exist before either signals the other
+  __syncthreads();
+  if (warp < 4 && lane == 0) {   // arm the first use of both exchange buffers (a quarter each)
+    mbar_arrive_expect_tx(x_full(0), X_BYTES / 4);
+    mbar_arrive_expect_tx(x_full(1), X_BYTES / 4);
+  }
+  cluster_sync();   // both CTAs' barriers exist (and are armed) before either signals the other
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ gather (cp.async)
+    // Warp gw copies rows gw, gw+4, ..: lane l moves 16-byte chunks l, l+32 of its column
+    // range, so each row is read with coalesced requests.  A tile's ids come from one
+    // coalesced load per warp, issued a tile ahead, and reach the rows through shuffles.
     const int gw = warp - 4;
     const __nv_bfloat16* kvb = kv + (int64_t)b * kv_bs;
-    auto load_id = [&](int j) -> int {
-      const int p = kbeg + j * NK + lane;
+    auto load_id = [&](int j, int r) -> int {
+      const int p = kbeg + j * NK + r;
       return (j < ntiles && p < kend) ? __ldg(irow + p) : -1;
     };
-    int id_next = load_id(0);
+    int id_next0 = load_id(0, lane), id_next1 = load_id(0, lane + 32);
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int st = j % NS;
-      const int id_cur = id_next;
-      id_next = load_id(j + 1);
+      const int id0 = id_next0, id1 = id_next1;
+      id_next0 = load_id(j + 1, lane);
+      id_next1 = load_id(j + 1, lane + 32);
       if (!(ok = mbar_wait(kv_empty(st), ((j / NS) & 1) ^ 1, abort, kWaitLimitNs))) break;
       if (gw == 0) {
-        ids_s[st * NK + lane] = id_cur;
+        ids_s[st * NK + lane] = id0;
+        ids_s[st * NK + 32 + lane] = id1;
         __syncwarp();
         if (lane == 0) mbar_arrive(ids_ready(st));
       }
@@ -249,7 +274,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
 #pragma unroll
       for (int i = 0; i < NK / 4; ++i) {
         const int r = gw + 4 * i;
-        const int key = __shfl_sync(0xffffffffu, id_cur, r);
+        const int key = __shfl_sync(0xffffffffu, r < 32 ? id0 : id1, r & 31);
         const __nv_bfloat16* src = kvb + (int64_t)(key < 0 ? 0 : key) * kv_rs;
         const int nbytes = key < 0 ? 0 : 16;
 #pragma unroll
@@ -268,19 +293,20 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     // ------------------------------------------------------------ MMA issuer
     bool ok = true;
     auto issue_pv = [&](int jj) -> bool {
-      if (!mbar_wait(p_full, jj & 1, abort, kWaitLimitNs)) return false;
+      const int pb = jj & 1;
+      if (!mbar_wait(p_full(pb), (jj >> 1) & 1, abort, kWaitLimitNs)) return false;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t stage = sbase + OFF_KV + (jj % NS) * KV_STAGE;
 #pragma unroll
         for (int kk = 0; kk < NK / 16; ++kk) {
-          const uint64_t ad = smem_desc(sbase + OFF_P + kk * 32, 512, kLayoutSw64);
-          // V columns 256*half .. +255 are the stage's blocks 0..3 for both CTAs
+          const uint64_t ad = smem_desc(sbase + OFF_P + pb * P_BYTES + kk * 32, 1024, kLayoutSw128);
+          // V columns 256*half .. +255 are the stage's blocks 0..3 for both CTAs; keys 16kk..
           const uint64_t bd = smem_desc_lbo(stage + kk * 2048, K_BLK, 1024, kLayoutSw128);
           mma_bf16(tmem + COL_O, ad, bd, IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(kv_empty(jj % NS));
-        mma_commit(pv_done);
+        mma_commit(pv_done(pb));
       }
       __syncwarp();
       return true;
@@ -288,9 +314,9 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     const int ks0 = half * KSTEPS;
     if (ntiles > 0) ok = mbar_wait(q_ready, 0, abort, kWaitLimitNs);
     for (int j = 0; j < ntiles && ok; ++j) {
-      const int st = j % NS, sb = j & 1;
+      const int st = j % NS;
       if (!(ok = mbar_wait(kv_full(st), (j / NS) & 1, abort, kWaitLimitNs))) break;
-      if (!(ok = mbar_wait(s_empty(sb), ((j >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
+      if (!(ok = mbar_wait(s_empty, (j & 1) ^ 1, abort, kWaitLimitNs))) break;
       tc_fence_after();
       fence_proxy_async();
       if (lane == 0) {
@@ -301,9 +327,9 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
           const uint32_t blk = (uint32_t)((ks >> 2) - blk0);
           const uint32_t off = (uint32_t)(ks & 3) * 32u;   // 16 columns = 32 bytes inside the atom
           const uint64_t bd = smem_desc(stage + blk * K_BLK + off, 1024, kLayoutSw128);
-          mma_bf16_ts(tmem + COL_S + sb * NK, tmem + COL_Q + 8u * i, bd, IDESC_S, i > 0 ? 1u : 0u);
+          mma_bf16_ts(tmem + COL_S, tmem + COL_Q + 8u * i, bd, IDESC_S, i > 0 ? 1u : 0u);
         }
-        mma_commit(s_full(sb));
+        mma_commit(s_full);
       }
       __syncwarp();
       if (j >= 1) ok = issue_pv(j - 1);
@@ -315,7 +341,6 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     float m_use = -INFINITY, l_run = 0.f;
     bool ok = true;
-    const uint32_t prow = sbase + OFF_P + row * 64;
     {
       // q[head, 288*half .. +287] -> TMEM lane `head`, bf16 pairs packed per 32-bit column
       const uint4* qsrc = reinterpret_cast<const uint4*>(q + ((int64_t)bt * HQ + row) * DQK + 288 * half);
@@ -341,52 +366,73 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
     }
+    const uint32_t sw = (uint32_t)(row & 7);
     for (int j = 0; j < ntiles; ++j) {
-      const int sb = j & 1;
-      if (!(ok = mbar_wait(s_full(sb), (j >> 1) & 1, abort, kWaitLimitNs))) break;
+      const int xb = j & 1, pb = j & 1, st = j % NS;
+      if (!(ok = mbar_wait(s_full, j & 1, abort, kWaitLimitNs))) break;
       tc_fence_after();
-      float s[32];
-      tmem_ld32(tmem + lane_off + COL_S + sb * NK, s);
+      float s[NK];
+      tmem_ld32(tmem + lane_off + COL_S, *reinterpret_cast<float(*)[32]>(s));
+      tmem_ld32(tmem + lane_off + COL_S + 32, *reinterpret_cast<float(*)[32]>(s + 32));
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(s_empty(sb));
-      // ---- swap partial scores with the partner (row r: 8 swizzled 16-byte chunks)
-      if (!(ok = mbar_wait_cluster(x_free(sb), ((j >> 1) & 1) ^ 1, abort))) break;
-      const uint32_t xrow_local = sbase + OFF_X + sb * X_BYTES + row * 128;
-      const uint32_t xrow_remote = map_to_cta(xrow_local, partner);
+      if (lane == 0) mbar_arrive(s_empty);
+      // ---- send the partial to the partner (row r of its buffer xb; 16 swizzled chunks)
+      if (!(ok = mbar_wait_cluster(x_free(xb), ((j >> 1) & 1) ^ 1, abort))) break;
+      {
+        const uint32_t xrow_remote = map_to_cta(sbase + OFF_X + xb * X_BYTES + row * 256, partner);
+        const uint32_t xbar_remote = map_to_cta(x_full(xb), partner);
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        st_cluster_v4(xrow_remote + ((c ^ (row & 7)) << 4), s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(map_to_cta(x_full(sb), partner));
-      if (!(ok = mbar_wait_cluster(x_full(sb), (j >> 1) & 1, abort))) break;
-      float o4[32];
+        for (int c = 0; c < 16; ++c)
+          st_async_v4(xrow_remote + ((c ^ sw) << 4), s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3], xbar_remote);
+      }
+      // ---- receive the partner's partial
+      if (!(ok = mbar_wait_cluster(x_full(xb), (j >> 1) & 1, abort))) break;
+      float o4[NK];
+      {
+        const uint32_t xrow = sbase + OFF_X + xb * X_BYTES + row * 256;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float4 v;
-        asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
-                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                     : "r"(xrow_local + ((c ^ (row & 7)) << 4)));
-        o4[4 * c] = v.x; o4[4 * c + 1] = v.y; o4[4 * c + 2] = v.z; o4[4 * c + 3] = v.w;
+        for (int c = 0; c < 16; ++c) {
+          float4 v;
+          asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+                       : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                       : "r"(xrow + ((c ^ sw) << 4)));
+          o4[4 * c] = v.x; o4[4 * c + 1] = v.y; o4[4 * c + 2] = v.z; o4[4 * c + 3] = v.w;
+        }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(map_to_cta(x_free(sb), partner));
-      // both CTAs add the partials in column order (cols 0..287 first), so both get the same scores
-      if (!(ok = mbar_wait(ids_ready(j % NS), (j / NS) & 1, abort, kWaitLimitNs))) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(x_full(xb), X_BYTES / 4);               // arm the buffer's next use
+        mbar_arrive_cluster(map_to_cta(x_free(xb), partner));         // the partner may refill it
+      }
+      // ---- masked full scores: both CTAs add the partials in column order (0..287 first)
+      if (!(ok = mbar_wait(ids_ready(st), (j / NS) & 1, abort, kWaitLimitNs))) break;
       float mt = -INFINITY;
+      {
+        const uint32_t ids_addr = sbase + OFF_IDS + st * NK * 4;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float full = half == 0 ? s[i] + o4[i] : o4[i] + s[i];
-        s[i] = ids_s[(j % NS) * NK + i] >= 0 ? full * scale_log2 : -INFINITY;
-        mt = fmaxf(mt, s[i]);
+        for (int c = 0; c < NK / 4; ++c) {
+          int4 id4;
+          asm volatile("ld.shared.v4.s32 {%0,%1,%2,%3}, [%4];\n"
+                       : "=r"(id4.x), "=r"(id4.y), "=r"(id4.z), "=r"(id4.w) : "r"(ids_addr + 16 * c));
+          const int idv[4] = {id4.x, id4.y, id4.z, id4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * c + e;
+            const float full = half == 0 ? s[i] + o4[i] : o4[i] + s[i];
+            s[i] = idv[e] >= 0 ? full * scale_log2 : -INFINITY;
+            mt = fmaxf(mt, s[i]);
+          }
+        }
       }
-      // P of the previous tile must have been consumed (and O be stable) before writing P
-      if (j >= 1 && !(ok = mbar_wait(pv_done, (j - 1) & 1, abort, kWaitLimitNs))) break;
-      tc_fence_after();
+      // ---- P buffer pb was last read by P.V of tile j-2
+      if (j >= 2 && !(ok = mbar_wait(pv_done(pb), ((j >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
       if (mt > m_use + kRescaleLog2 || (m_use == -INFINITY && mt > -INFINITY)) {
-        const float alpha = (m_use == -INFINITY) ? 0.f : exp2f(m_use - mt);
+        const float alpha = (m_use == -INFINITY) ? 0.f : ex2(m_use - mt);
         if (j >= 1 && m_use != -INFINITY) {   // O already holds earlier tiles: rescale it
+          if (!(ok = mbar_wait(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort, kWaitLimitNs))) break;
+          tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < DVH; c += 32) {
             float o[32];
@@ -401,27 +447,31 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         l_run *= alpha;
         m_use = mt;
       }
-      uint32_t pk[16];
+      // ---- P = exp2(s - m_use) as bf16, one 128-byte swizzled row per head
+      {
+        const uint32_t prow = sbase + OFF_P + pb * P_BYTES + row * 128;
+        const bool live = m_use != -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float p0v = m_use == -INFINITY ? 0.f : exp2f(s[i] - m_use);
-        const float p1v = m_use == -INFINITY ? 0.f : exp2f(s[i + 1] - m_use);
-        l_run += p0v + p1v;
-        pk[i >> 1] = pack2_bf16(p0v, p1v);
-      }
+        for (int c = 0; c < 8; ++c) {
+          uint32_t pk[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint32_t dst = prow + ((c ^ ((row >> 1) & 3)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(dst), "r"(pk[4 * c]), "r"(pk[4 * c + 1]),
-                     "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3]));
+          for (int e = 0; e < 4; ++e) {
+            const float p0v = live ? ex2(s[8 * c + 2 * e] - m_use) : 0.f;
+            const float p1v = live ? ex2(s[8 * c + 2 * e + 1] - m_use) : 0.f;
+            l_run += p0v + p1v;
+            pk[e] = pack2_bf16(p0v, p1v);
+          }
+          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(prow + ((c ^ sw) << 4)), "r"(pk[0]),
+                       "r"(pk[1]), "r"(pk[2]), "r"(pk[3]));
+        }
       }
       fence_proxy_async();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(p_full(pb));
     }
     // ---- epilogue: wait for the last P.V, normalise, write
-    if (ok && ntiles > 0) ok = mbar_wait(pv_done, (ntiles - 1) & 1, abort, kWaitLimitNs);
+    if (ok && ntiles > 0) ok = mbar_wait(pv_done((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1, abort, kWaitLimitNs);
     tc_fence_after();
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
     const float lse_r = l_run > 0.f ? (m_use + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
