@@ -16,8 +16,8 @@
 //   * gathers only the row columns it needs: c = 0 columns 0..287, c = 1 columns 256..575.
 // Per CTA: a 3-stage ring of 40 KB key tiles; TMEM 64 score + 144 q + 256 output columns.
 //
-//   warps 0-3  softmax: thread = head.  Partial scores from TMEM -> partner (asynchronous
-//              remote stores that complete the partner's barrier); partner's partial
+//   warps 0-3  softmax: thread = head.  Partial scores from TMEM -> a local stage -> one bulk
+//              copy into the partner (completing the partner's barrier); partner's partial
 //              + own -> masked scores; running max moved only when a tile exceeds it by more
 //              than 2^8 (then O is rescaled in TMEM); P = exp2(S - m) as bf16 in one of two
 //              shared-memory buffers, so a tile's softmax overlaps the previous tile's P.V; at the end O / l is written out (or a split partial with its lse).
@@ -46,11 +46,12 @@ constexpr int KV_STAGE = BLKS * K_BLK;                 // 40960
 constexpr int OFF_KV = 0;
 constexpr int OFF_P = OFF_KV + NS * KV_STAGE;          // 2 P buffers: rows of 128 B (64 keys bf16)
 constexpr int P_BYTES = HQ * NK * 2;                   // 16384
-constexpr int OFF_X = OFF_P + 2 * P_BYTES;             // partner's partial scores, 2 buffers
-constexpr int X_BYTES = HQ * NK * 4;                   // 32768
-constexpr int OFF_IDS = OFF_X + 2 * X_BYTES;
+constexpr int X_BYTES = HQ * NK * 4;                   // 32768: one tile of fp32 partial scores
+constexpr int OFF_XS = OFF_P + 2 * P_BYTES;            // own partial, staged for the bulk copy out
+constexpr int OFF_X = OFF_XS + X_BYTES;                // partner's partial, copied in
+constexpr int OFF_IDS = OFF_X + X_BYTES;
 constexpr int OFF_BAR = OFF_IDS + NS * NK * 4;
-constexpr int NBARS = 3 * NS + 12;
+constexpr int NBARS = 3 * NS + 14;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;       // + alignment slack
 constexpr int THREADS = 288;
@@ -63,7 +64,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
 
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert((OFF_P % 1024) == 0 && (OFF_KV % 1024) == 0 && (OFF_X % 16) == 0, "alignment");
+static_assert((OFF_P % 1024) == 0 && (OFF_KV % 1024) == 0 && (OFF_X % 128) == 0 && (OFF_XS % 128) == 0, "alignment");
 static_assert(COL_Q + 144 <= COL_O && COL_S + NK <= COL_Q, "TMEM map");
 
 constexpr uint32_t IDESC_S = instr_desc(128, NK, 1);                   // bf16, K-major A and B
@@ -190,11 +191,13 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   auto ids_ready = [&](int s) { return bar0 + 8u * (2 * NS + s); };
   const uint32_t s_full = bar0 + 8u * (3 * NS);
   const uint32_t s_empty = bar0 + 8u * (3 * NS + 1);
-  auto x_full = [&](int s) { return bar0 + 8u * (3 * NS + 2 + s); };   // partner's partial landed here
-  auto x_free = [&](int s) { return bar0 + 8u * (3 * NS + 4 + s); };   // partner read what we sent it
+  const uint32_t x_full = bar0 + 8u * (3 * NS + 2);   // partner's partial landed in OFF_X
+  const uint32_t x_free = bar0 + 8u * (3 * NS + 3);   // partner has read what we copied into it
   auto p_full = [&](int s) { return bar0 + 8u * (3 * NS + 6 + s); };
   auto pv_done = [&](int s) { return bar0 + 8u * (3 * NS + 8 + s); };
   const uint32_t q_ready = bar0 + 8u * (3 * NS + 10);
+  const uint32_t xs_free = bar0 + 8u * (3 * NS + 11);   // the stage of the outgoing partial may be written
+  const uint32_t xs_full = bar0 + 8u * (3 * NS + 12);   // all 128 rows of the outgoing partial are staged
   volatile int* ids_s = reinterpret_cast<volatile int*>(sgen + OFF_IDS);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(sgen + OFF_MISC + 4);
@@ -221,13 +224,15 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     }
     mbar_init(s_full, 1);
     mbar_init(s_empty, 4);
+    mbar_init(x_full, 1);   // one expect-tx arrival per use, plus the partner's bytes
+    mbar_init(x_free, 4);   // the partner's 4 softmax warps, once each has read its rows
     for (int s = 0; s < 2; ++s) {
-      mbar_init(x_full(s), 4);   // one expect-tx arrival per softmax warp, plus the partner's bytes
-      mbar_init(x_free(s), 4);   // the partner's 4 softmax warps
       mbar_init(p_full(s), 4);
       mbar_init(pv_done(s), 1);
     }
     mbar_init(q_ready, 4);
+    mbar_init(xs_free, 1);
+    mbar_init(xs_full, 128);
     *abort = 0;
     fence_barrier_init();
   }
@@ -237,10 +242,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   }
   tc_fence_before();
   __syncthreads();
-  if (warp < 4 && lane == 0) {   // arm the first use of both exchange buffers (a quarter each)
-    mbar_arrive_expect_tx(x_full(0), X_BYTES / 4);
-    mbar_arrive_expect_tx(x_full(1), X_BYTES / 4);
-  }
+  if (threadIdx.x == 0) mbar_arrive_expect_tx(x_full, X_BYTES);   // arm the first exchange
   cluster_sync();   // both CTAs' barriers exist (and are armed) before either signals the other
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -378,20 +380,39 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_empty);
-      // ---- send the partial to the partner (row r of its buffer xb; 16 swizzled chunks)
-      if (!(ok = mbar_wait_cluster(x_free(xb), ((j >> 1) & 1) ^ 1, abort))) break;
+      // ---- send the partial to the partner: rows staged locally, one bulk copy of the tile
       {
-        const uint32_t xrow_remote = map_to_cta(sbase + OFF_X + xb * X_BYTES + row * 256, partner);
-        const uint32_t xbar_remote = map_to_cta(x_full(xb), partner);
+        if (threadIdx.x == 0) {   // the previous copy out has finished reading the stage
+          if (j >= 1) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+          mbar_arrive(xs_free);
+        }
+        if (!(ok = mbar_wait(xs_free, j & 1, abort, kWaitLimitNs))) break;
+        const uint32_t xs_row = sbase + OFF_XS + row * 256;
 #pragma unroll
         for (int c = 0; c < 16; ++c)
-          st_async_v4(xrow_remote + ((c ^ sw) << 4), s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3], xbar_remote);
+          asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};\n" ::"r"(xs_row + ((c ^ sw) << 4)), "f"(s[4 * c]),
+                       "f"(s[4 * c + 1]), "f"(s[4 * c + 2]), "f"(s[4 * c + 3]));
+        fence_proxy_async();
+        mbar_arrive(xs_full);
+        if (threadIdx.x == 0) {
+          // every row is staged, and the partner has read our previous copy out of its buffer
+          ok = mbar_wait(xs_full, j & 1, abort, kWaitLimitNs) && mbar_wait_cluster(x_free, (j & 1) ^ 1, abort);
+          if (ok) {
+            asm volatile(
+                "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+                "cp.async.bulk.commit_group;\n"
+                ::"r"(map_to_cta(sbase + OFF_X, partner)), "r"(sbase + OFF_XS), "r"((uint32_t)X_BYTES),
+                  "r"(map_to_cta(x_full, partner))
+                : "memory");
+          }
+          if (!ok) break;
+        }
       }
       // ---- receive the partner's partial
-      if (!(ok = mbar_wait_cluster(x_full(xb), (j >> 1) & 1, abort))) break;
+      if (!(ok = mbar_wait_cluster(x_full, j & 1, abort))) break;
       float o4[NK];
       {
-        const uint32_t xrow = sbase + OFF_X + xb * X_BYTES + row * 256;
+        const uint32_t xrow = sbase + OFF_X + row * 256;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           float4 v;
@@ -403,8 +424,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       }
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_expect_tx(x_full(xb), X_BYTES / 4);               // arm the buffer's next use
-        mbar_arrive_cluster(map_to_cta(x_free(xb), partner));         // the partner may refill it
+        if (warp == 0) mbar_arrive_expect_tx(x_full, X_BYTES);   // arm the next exchange
+        mbar_arrive_cluster(map_to_cta(x_free, partner));        // the partner may copy in again
       }
       // ---- masked full scores: both CTAs add the partials in column order (0..287 first)
       if (!(ok = mbar_wait(ids_ready(st), (j / NS) & 1, abort, kWaitLimitNs))) break;
@@ -521,6 +542,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     }
   }
 
+  if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
   tc_fence_before();
   __syncthreads();
   if (warp == 8) {
