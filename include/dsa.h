@@ -143,6 +143,30 @@ int dsa_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v,
                     size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * dsa_sparse_attn_noalloc - dsa_sparse_attn for callers that can neither allocate device
+ * memory nor pass a workspace (for example an operator inside a runtime that owns all device
+ * memory and offers its operators no scratch, or a serving loop that must not call cudaMalloc
+ * once it runs).  The method described in the sources has no counterpart to this call: it is
+ * a deployment variant.  Same arguments, layouts and results as dsa_sparse_attn minus `ws`;
+ * the split-key partials go to a fixed scratch array inside the library instead.
+ *   - The scratch is dsa_noalloc_scratch_bytes() (16 MiB) per GPU that loads the library,
+ *     held until the process exits.  Problems whose partials need more (see
+ *     dsa_sparse_attn_workspace_size) return DSA_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
+ *   - The first call on a device looks up the scratch's device address (with that device
+ *     current) and caches it; make that first call before any stream capture.
+ *   - All calls on a device share the scratch: calls whose kernels may overlap on the GPU
+ *     (other streams, other host threads) race on it and must be serialised by the caller.
+ *     Nothing in the scratch needs to start at zero; a call ignores what the last one left.
+ *   - Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ * ------------------------------------------------------------------------------------ */
+size_t dsa_noalloc_scratch_bytes(void);
+int dsa_sparse_attn_noalloc(const uint16_t* q, const uint16_t* kv, const uint16_t* v,
+                            int64_t kv_row_stride, int64_t kv_batch_stride, int64_t v_row_stride,
+                            int64_t v_batch_stride, const int32_t* idx, int B, int T, int Hq,
+                            int d_qk, int d_v, int k, float sm_scale, uint16_t* out, float* lse,
+                            void* stream);
+
+/* ------------------------------------------------------------------------------------
  * dsa_index_pool - IndexPool ("What changed": four indexer keys pooled into one):
  *     k_pool[b, g, :] = e4m3(((k[4g] + k[4g+1]) + (k[4g+2] + k[4g+3])) * 0.25)
  * with the sum in fp32 on the decoded keys and the requantisation round-to-nearest-even,

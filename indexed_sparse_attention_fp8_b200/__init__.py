@@ -64,6 +64,9 @@ _SIGS = {
     "dsa_sparse_attn": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_int, _c_int, _c_int,
                                  _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_sz, _c_p]),
     "dsa_index_pool": (_c_int, [_c_p, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p]),
+    "dsa_noalloc_scratch_bytes": (_c_sz, []),
+    "dsa_sparse_attn_noalloc": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_int, _c_int,
+                                         _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p]),
     "dsa_group_workspace_size": (_c_sz, [ctypes.POINTER(GroupArgs), _c_int]),
     "dsa_group_forward": (_c_int, [ctypes.POINTER(GroupArgs), _c_p, _c_sz, _c_p]),
 }
@@ -175,6 +178,26 @@ def dsa_sparse_attn(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, sm_sca
     _check("dsa_sparse_attn", _lib().dsa_sparse_attn(
         _ptr(q), _ptr(kv), _ptr(v), kv.stride(1), kv.stride(0), v_rs, v_bs, _ptr(idx), B, T, Hq, Dqk, d_v, k,
         float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws), wsb, _stream(stream)))
+    return out, lse
+
+
+def dsa_sparse_attn_noalloc(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, sm_scale: float, d_v: int,
+                            v: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                            lse: Optional[torch.Tensor] = None, want_lse: bool = False, stream=None):
+    """dsa_sparse_attn without a workspace: split partials use the library's fixed scratch
+    (dsa_noalloc_scratch_bytes() per GPU).  For callers that cannot allocate device memory;
+    calls that may overlap on one GPU share that scratch and must be serialised."""
+    B, T, Hq, Dqk = q.shape
+    k = idx.shape[-1]
+    if out is None:
+        out = torch.empty((B, T, Hq, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, T, Hq), dtype=torch.float32, device=q.device)
+    v_rs = v.stride(1) if v is not None else 0
+    v_bs = v.stride(0) if v is not None else 0
+    _check("dsa_sparse_attn_noalloc", _lib().dsa_sparse_attn_noalloc(
+        _ptr(q), _ptr(kv), _ptr(v), kv.stride(1), kv.stride(0), v_rs, v_bs, _ptr(idx), B, T, Hq, Dqk, d_v, k,
+        float(sm_scale), _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
 
 

@@ -1,0 +1,78 @@
+// Sparse attention without a caller workspace: the split-key partials live in a fixed scratch
+// array that this file owns, so the call allocates no device memory at any point.
+//
+// Who needs it: code that can neither allocate device memory nor hand the library a workspace
+// buffer -- for instance an operator plugged into a runtime that owns all device memory and
+// gives its operators no scratch, or a serving loop that must not call cudaMalloc once it is
+// running (an allocation there can synchronise the device, or fail once the memory pool has
+// claimed the GPU).  Such callers still pass their own inputs and outputs.
+//
+// Costs and limits, in plain terms:
+//   * every GPU that loads the library keeps kScratchBytes (16 MiB) reserved until the process
+//     exits, whether or not this entry point is ever called;
+//   * all calls on a device share the one array, so two calls whose kernels overlap on that
+//     device (different streams, or a second host thread) race on it: serialise them;
+//   * problems whose split partials need more than kScratchBytes are rejected up front.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace dsa {
+namespace {
+
+// 16 MiB, enough for the split partials of up to ~60 decode queries at 128 heads x 512 dv.
+constexpr size_t kScratchBytes = size_t(16) << 20;
+
+// The scratch itself.  Host code must not use this name as a pointer: on the host it is only a
+// stand-in for the symbol, so its device address is fetched with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up on the first call for
+// that device (with the device current) and cached; nullptr on failure (error recorded).
+void* scratch_on_current_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    set_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidDevice);
+    return nullptr;
+  }
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      set_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+      return nullptr;
+    }
+    g_scratch_ptr[dev] = p;
+  }
+  return g_scratch_ptr[dev];
+}
+
+}  // namespace
+}  // namespace dsa
+
+extern "C" {
+
+size_t dsa_noalloc_scratch_bytes(void) { return dsa::kScratchBytes; }
+
+int dsa_sparse_attn_noalloc(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t kv_row_stride,
+                            int64_t kv_batch_stride, int64_t v_row_stride, int64_t v_batch_stride,
+                            const int32_t* idx, int B, int T, int Hq, int d_qk, int d_v, int k, float sm_scale,
+                            uint16_t* out, float* lse, void* stream) {
+  // Every partial the split kernels write is written before it is read, so nothing in the
+  // shared scratch has to start at zero and the previous call's contents are harmless.
+  const size_t need = dsa_sparse_attn_workspace_size(B, T, Hq, d_v, k);
+  if (need > dsa::kScratchBytes) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  if (need > 0) {
+    scratch = dsa::scratch_on_current_device();
+    if (scratch == nullptr) return DSA_ERR_CUDA;
+  }
+  return dsa_sparse_attn(q, kv, v, kv_row_stride, kv_batch_stride, v_row_stride, v_batch_stride, idx, B, T, Hq,
+                         d_qk, d_v, k, sm_scale, out, lse, scratch, need > 0 ? dsa::kScratchBytes : 0, stream);
+}
+
+}  // extern "C"
