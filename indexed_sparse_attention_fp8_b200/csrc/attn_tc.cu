@@ -16,8 +16,9 @@
 //   * gathers only the row columns it needs: c = 0 columns 0..287, c = 1 columns 256..575.
 // Per CTA: a 3-stage ring of 40 KB key tiles; TMEM 64 score + 144 q + 256 output columns.
 //
-//   warps 0-3  softmax: thread = head.  Partial scores from TMEM -> a local stage -> one bulk
-//              copy into the partner (completing the partner's barrier); partner's partial
+//   warps 0-3  softmax: thread = head.  Partial scores from TMEM -> a local stage -> per warp,
+//              one 8 KB bulk copy into the partner (completing that warp's barrier there);
+//              partner's partial
 //              + own -> masked scores; running max moved only when a tile exceeds it by more
 //              than 2^8 (then O is rescaled in TMEM); P = exp2(S - m) as bf16 in one of two
 //              shared-memory buffers, so a tile's softmax overlaps the previous tile's P.V; at the end O / l is written out (or a split partial with its lse).
@@ -51,7 +52,7 @@ constexpr int OFF_XS = OFF_P + 2 * P_BYTES;            // own partial, staged fo
 constexpr int OFF_X = OFF_XS + X_BYTES;                // partner's partial, copied in
 constexpr int OFF_IDS = OFF_X + X_BYTES;
 constexpr int OFF_BAR = OFF_IDS + NS * NK * 4;
-constexpr int NBARS = 3 * NS + 14;
+constexpr int NBARS = 3 * NS + 22;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;       // + alignment slack
 constexpr int THREADS = 288;
@@ -191,13 +192,12 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   auto ids_ready = [&](int s) { return bar0 + 8u * (2 * NS + s); };
   const uint32_t s_full = bar0 + 8u * (3 * NS);
   const uint32_t s_empty = bar0 + 8u * (3 * NS + 1);
-  const uint32_t x_full = bar0 + 8u * (3 * NS + 2);   // partner's partial landed in OFF_X
-  const uint32_t x_free = bar0 + 8u * (3 * NS + 3);   // partner has read what we copied into it
+  // per softmax warp w (rows 32w..32w+31): the partner's rows landed / the partner read ours
+  auto x_full = [&](int w) { return bar0 + 8u * (3 * NS + 13 + w); };
+  auto x_free = [&](int w) { return bar0 + 8u * (3 * NS + 17 + w); };
   auto p_full = [&](int s) { return bar0 + 8u * (3 * NS + 6 + s); };
   auto pv_done = [&](int s) { return bar0 + 8u * (3 * NS + 8 + s); };
   const uint32_t q_ready = bar0 + 8u * (3 * NS + 10);
-  const uint32_t xs_free = bar0 + 8u * (3 * NS + 11);   // the stage of the outgoing partial may be written
-  const uint32_t xs_full = bar0 + 8u * (3 * NS + 12);   // all 128 rows of the outgoing partial are staged
   volatile int* ids_s = reinterpret_cast<volatile int*>(sgen + OFF_IDS);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(sgen + OFF_MISC + 4);
@@ -224,15 +224,15 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     }
     mbar_init(s_full, 1);
     mbar_init(s_empty, 4);
-    mbar_init(x_full, 1);   // one expect-tx arrival per use, plus the partner's bytes
-    mbar_init(x_free, 4);   // the partner's 4 softmax warps, once each has read its rows
+    for (int w = 0; w < 4; ++w) {
+      mbar_init(x_full(w), 1);   // one expect-tx arrival per use, plus the partner's 8 KB
+      mbar_init(x_free(w), 1);   // the partner's warp w, once it has read our rows
+    }
     for (int s = 0; s < 2; ++s) {
       mbar_init(p_full(s), 4);
       mbar_init(pv_done(s), 1);
     }
     mbar_init(q_ready, 4);
-    mbar_init(xs_free, 1);
-    mbar_init(xs_full, 128);
     *abort = 0;
     fence_barrier_init();
   }
@@ -242,7 +242,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   }
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) mbar_arrive_expect_tx(x_full, X_BYTES);   // arm the first exchange
+  if (warp < 4 && lane == 0) mbar_arrive_expect_tx(x_full(warp), X_BYTES / 4);   // arm the first exchange
   cluster_sync();   // both CTAs' barriers exist (and are armed) before either signals the other
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -380,36 +380,36 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_empty);
-      // ---- send the partial to the partner: rows staged locally, one bulk copy of the tile
+      // ---- send this warp's 32 partial rows to the partner's warp: stage locally, one 8 KB
+      //      bulk copy that completes the partner's per-warp barrier (no CTA-wide sync)
       {
-        if (threadIdx.x == 0) {   // the previous copy out has finished reading the stage
-          if (j >= 1) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
-          mbar_arrive(xs_free);
-        }
-        if (!(ok = mbar_wait(xs_free, j & 1, abort, kWaitLimitNs))) break;
+        if (lane == 0 && j >= 1) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+        __syncwarp();
         const uint32_t xs_row = sbase + OFF_XS + row * 256;
 #pragma unroll
         for (int c = 0; c < 16; ++c)
           asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};\n" ::"r"(xs_row + ((c ^ sw) << 4)), "f"(s[4 * c]),
                        "f"(s[4 * c + 1]), "f"(s[4 * c + 2]), "f"(s[4 * c + 3]));
         fence_proxy_async();
-        mbar_arrive(xs_full);
-        if (threadIdx.x == 0) {
-          // every row is staged, and the partner has read our previous copy out of its buffer
-          ok = mbar_wait(xs_full, j & 1, abort, kWaitLimitNs) && mbar_wait_cluster(x_free, (j & 1) ^ 1, abort);
+        __syncwarp();
+        if (lane == 0) {
+          // the partner's warp has read our previous rows out of its buffer
+          ok = mbar_wait_cluster(x_free(warp), (j & 1) ^ 1, abort);
           if (ok) {
+            const uint32_t off = (uint32_t)(warp * 32 * 256);
             asm volatile(
                 "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
                 "cp.async.bulk.commit_group;\n"
-                ::"r"(map_to_cta(sbase + OFF_X, partner)), "r"(sbase + OFF_XS), "r"((uint32_t)X_BYTES),
-                  "r"(map_to_cta(x_full, partner))
+                ::"r"(map_to_cta(sbase + OFF_X + off, partner)), "r"(sbase + OFF_XS + off), "r"((uint32_t)(X_BYTES / 4)),
+                  "r"(map_to_cta(x_full(warp), partner))
                 : "memory");
           }
-          if (!ok) break;
         }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
       }
-      // ---- receive the partner's partial
-      if (!(ok = mbar_wait_cluster(x_full, j & 1, abort))) break;
+      // ---- receive the partner's rows for this warp
+      if (!(ok = mbar_wait_cluster(x_full(warp), j & 1, abort))) break;
       float o4[NK];
       {
         const uint32_t xrow = sbase + OFF_X + row * 256;
@@ -424,8 +424,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       }
       __syncwarp();
       if (lane == 0) {
-        if (warp == 0) mbar_arrive_expect_tx(x_full, X_BYTES);   // arm the next exchange
-        mbar_arrive_cluster(map_to_cta(x_free, partner));        // the partner may copy in again
+        mbar_arrive_expect_tx(x_full(warp), X_BYTES / 4);        // arm this warp's next exchange
+        mbar_arrive_cluster(map_to_cta(x_free(warp), partner));  // the partner's warp may copy in again
       }
       // ---- masked full scores: both CTAs add the partials in column order (0..287 first)
       if (!(ok = mbar_wait(ids_ready(st), (j / NS) & 1, abort, kWaitLimitNs))) break;
@@ -542,7 +542,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     }
   }
 
-  if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
+  if (warp < 4 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");   // own copies landed
   tc_fence_before();
   __syncthreads();
   if (warp == 8) {
