@@ -51,7 +51,7 @@ constexpr int X_BYTES = HQ * NK * 4;                   // 32768: one tile of fp3
 constexpr int OFF_XS = OFF_P + 2 * P_BYTES;            // own partial, staged for the bulk copy out
 constexpr int OFF_X = OFF_XS + X_BYTES;                // partner's partial, copied in
 constexpr int OFF_IDS = OFF_X + X_BYTES;
-constexpr int OFF_BAR = OFF_IDS + NS * NK * 4;
+constexpr int OFF_BAR = OFF_IDS + NS * NK * 4 + 16 * NS;   // ids + an all-valid flag per stage
 constexpr int NBARS = 3 * NS + 22;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;       // + alignment slack
@@ -269,6 +269,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       if (gw == 0) {
         ids_s[st * NK + lane] = id0;
         ids_s[st * NK + 32 + lane] = id1;
+        const unsigned all_valid = __all_sync(0xffffffffu, id0 >= 0 && id1 >= 0);
+        if (lane == 0) ids_s[NS * NK + 4 * st] = (int)all_valid;   // tile needs no masking
         __syncwarp();
         if (lane == 0) mbar_arrive(ids_ready(st));
       }
@@ -346,23 +348,30 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     {
       // q[head, 288*half .. +287] -> TMEM lane `head`, bf16 pairs packed per 32-bit column
       const uint4* qsrc = reinterpret_cast<const uint4*>(q + ((int64_t)bt * HQ + row) * DQK + 288 * half);
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      uint4 qa[16], qb[20];   // all 36 loads in flight together
+#pragma unroll
+      for (int i = 0; i < 16; ++i) qa[i] = __ldg(qsrc + i);
+#pragma unroll
+      for (int i = 0; i < 20; ++i) qb[i] = __ldg(qsrc + 16 + i);
+      {
         uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 v = __ldg(qsrc + 8 * c + i);
-          w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-        }
-        tmem_st32u(tmem + lane_off + COL_Q + 32 * c, w);
-      }
-      uint32_t w16[16];
+        for (int i = 0; i < 8; ++i) { w[4 * i] = qa[i].x; w[4 * i + 1] = qa[i].y; w[4 * i + 2] = qa[i].z; w[4 * i + 3] = qa[i].w; }
+        tmem_st32u(tmem + lane_off + COL_Q, w);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 v = __ldg(qsrc + 32 + i);
-        w16[4 * i] = v.x; w16[4 * i + 1] = v.y; w16[4 * i + 2] = v.z; w16[4 * i + 3] = v.w;
+        for (int i = 0; i < 8; ++i) { w[4 * i] = qa[8 + i].x; w[4 * i + 1] = qa[8 + i].y; w[4 * i + 2] = qa[8 + i].z; w[4 * i + 3] = qa[8 + i].w; }
+        tmem_st32u(tmem + lane_off + COL_Q + 32, w);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { w[4 * i] = qb[i].x; w[4 * i + 1] = qb[i].y; w[4 * i + 2] = qb[i].z; w[4 * i + 3] = qb[i].w; }
+        tmem_st32u(tmem + lane_off + COL_Q + 64, w);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { w[4 * i] = qb[8 + i].x; w[4 * i + 1] = qb[8 + i].y; w[4 * i + 2] = qb[8 + i].z; w[4 * i + 3] = qb[8 + i].w; }
+        tmem_st32u(tmem + lane_off + COL_Q + 96, w);
+        uint32_t w16[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { w16[4 * i] = qb[16 + i].x; w16[4 * i + 1] = qb[16 + i].y; w16[4 * i + 2] = qb[16 + i].z; w16[4 * i + 3] = qb[16 + i].w; }
+        tmem_st16u(tmem + lane_off + COL_Q + 128, w16);
       }
-      tmem_st16u(tmem + lane_off + COL_Q + 128, w16);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -429,23 +438,30 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       }
       // ---- masked full scores: both CTAs add the partials in column order (0..287 first)
       if (!(ok = mbar_wait(ids_ready(st), (j / NS) & 1, abort, kWaitLimitNs))) break;
-      float mt = -INFINITY;
+      float mt = -INFINITY;   // in the log2 domain (scaled)
       {
-        const uint32_t ids_addr = sbase + OFF_IDS + st * NK * 4;
+        const bool all_valid = ids_s[NS * NK + 4 * st] != 0;
 #pragma unroll
-        for (int c = 0; c < NK / 4; ++c) {
-          int4 id4;
-          asm volatile("ld.shared.v4.s32 {%0,%1,%2,%3}, [%4];\n"
-                       : "=r"(id4.x), "=r"(id4.y), "=r"(id4.z), "=r"(id4.w) : "r"(ids_addr + 16 * c));
-          const int idv[4] = {id4.x, id4.y, id4.z, id4.w};
+        for (int i = 0; i < NK; ++i) s[i] = half == 0 ? s[i] + o4[i] : o4[i] + s[i];   // same order in both CTAs
+        if (!all_valid) {
+          const uint32_t ids_addr = sbase + OFF_IDS + st * NK * 4;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = 4 * c + e;
-            const float full = half == 0 ? s[i] + o4[i] : o4[i] + s[i];
-            s[i] = idv[e] >= 0 ? full * scale_log2 : -INFINITY;
-            mt = fmaxf(mt, s[i]);
+          for (int c = 0; c < NK / 4; ++c) {
+            int4 id4;
+            asm volatile("ld.shared.v4.s32 {%0,%1,%2,%3}, [%4];\n"
+                         : "=r"(id4.x), "=r"(id4.y), "=r"(id4.z), "=r"(id4.w) : "r"(ids_addr + 16 * c));
+            if (id4.x < 0) s[4 * c] = -INFINITY;
+            if (id4.y < 0) s[4 * c + 1] = -INFINITY;
+            if (id4.z < 0) s[4 * c + 2] = -INFINITY;
+            if (id4.w < 0) s[4 * c + 3] = -INFINITY;
           }
         }
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < NK; i += 4) {
+          m0 = fmaxf(m0, s[i]); m1 = fmaxf(m1, s[i + 1]); m2 = fmaxf(m2, s[i + 2]); m3 = fmaxf(m3, s[i + 3]);
+        }
+        mt = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * scale_log2;   // scale > 0 commutes with max
       }
       // ---- P buffer pb was last read by P.V of tile j-2
       if (j >= 2 && !(ok = mbar_wait(pv_done(pb), ((j >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
@@ -477,8 +493,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
           uint32_t pk[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p0v = live ? ex2(s[8 * c + 2 * e] - m_use) : 0.f;
-            const float p1v = live ? ex2(s[8 * c + 2 * e + 1] - m_use) : 0.f;
+            const float p0v = live ? ex2(fmaf(s[8 * c + 2 * e], scale_log2, -m_use)) : 0.f;
+            const float p1v = live ? ex2(fmaf(s[8 * c + 2 * e + 1], scale_log2, -m_use)) : 0.f;
             l_run += p0v + p1v;
             pk[e] = pack2_bf16(p0v, p1v);
           }
