@@ -23,9 +23,9 @@
 //              than 2^8 (then O is rescaled in TMEM); P = exp2(S - m) as bf16 in one of two
 //              shared-memory buffers, so a tile's softmax overlaps the previous tile's P.V; at the end O / l is written out (or a split partial with its lse).
 //              First, each thread stores its head's q columns into TMEM.
-//   warps 4-7  gather: 16-byte cp.async of the selected rows into the 128-byte-swizzled
+//   warps 4-6  gather: 16-byte cp.async of the selected rows into the 128-byte-swizzled
 //              K-major layout the tensor core reads (also V's MN-major layout).
-//   warp 8     TMEM owner and MMA issuer.
+//   warp 7     TMEM owner and MMA issuer.
 // Every wait is bounded (tc_common.cuh); the two CTAs meet at cluster barriers only at start
 // and end.
 #include "common.cuh"
@@ -55,8 +55,9 @@ constexpr int OFF_BAR = OFF_IDS + NS * NK * 4 + 16 * NS;   // ids + an all-valid
 constexpr int NBARS = 3 * NS + 22;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;       // + alignment slack
-constexpr int THREADS = 288;
-constexpr int GATHER_THREADS = 128;
+constexpr int THREADS = 256;            // 8 warps: 2 per SM sub-partition, so up to 255 registers
+constexpr int GATHER_THREADS = 96;
+constexpr int MMA_WARP = 7;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S = 0;      // partial scores, NK columns
 constexpr uint32_t COL_Q = 64;     // this CTA's 288 q columns as packed bf16 pairs: 144 columns
@@ -236,7 +237,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     *abort = 0;
     fence_barrier_init();
   }
-  if (warp == 8) {
+  if (warp == MMA_WARP) {
     tmem_alloc(sbase + OFF_MISC, TMEM_COLS);
     tmem_relinquish();
   }
@@ -247,9 +248,9 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= 4 && warp < 8) {
+  if (warp >= 4 && warp < MMA_WARP) {
     // ------------------------------------------------------------ gather (cp.async)
-    // Warp gw copies rows gw, gw+4, ..: lane l moves 16-byte chunks l, l+32 of its column
+    // Warp gw copies rows gw, gw+3, ..: lane l moves 16-byte chunks l, l+32 of its column
     // range, so each row is read with coalesced requests.  A tile's ids come from one
     // coalesced load per warp, issued a tile ahead, and reach the rows through shuffles.
     const int gw = warp - 4;
@@ -275,9 +276,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         if (lane == 0) mbar_arrive(ids_ready(st));
       }
       const uint32_t stage = sbase + OFF_KV + st * KV_STAGE;
-#pragma unroll
-      for (int i = 0; i < NK / 4; ++i) {
-        const int r = gw + 4 * i;
+#pragma unroll 4
+      for (int r = gw; r < NK; r += 3) {
         const int key = __shfl_sync(0xffffffffu, r < 32 ? id0 : id1, r & 31);
         const __nv_bfloat16* src = kvb + (int64_t)(key < 0 ? 0 : key) * kv_rs;
         const int nbytes = key < 0 ? 0 : 16;
@@ -293,7 +293,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(kv_full(st)) : "memory");
     }
     cp_async_wait<0>();
-  } else if (warp == 8) {
+  } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     bool ok = true;
     auto issue_pv = [&](int jj) -> bool {
@@ -561,7 +561,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   if (warp < 4 && lane == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");   // own copies landed
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
