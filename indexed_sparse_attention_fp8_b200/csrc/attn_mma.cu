@@ -359,6 +359,15 @@ int launch_cfg(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t
 }  // namespace
 
 int attn_num_splits(int B, int T, int Hq, int k) {
+  if (Hq == 128) {
+    // tensor-core MLA kernel: one CTA pair per (query, split), one CTA per SM.  Aim for a
+    // single wave of pairs and keep at least 8 key tiles per split, so the fixed per-CTA work
+    // (q into TMEM, the output write) stays small next to the gathers.
+    const int64_t pairs = (int64_t)B * T;
+    int splits = 1;
+    while (pairs * splits * 2 * 2 <= 148 && k / (splits * 2) >= 512 && splits < 16) splits *= 2;
+    return splits;
+  }
   const int64_t base = (int64_t)B * T * (Hq >= 64 ? Hq / 64 : 1);
   int splits = 1;
   while (base * splits < kTargetCtas && k / (splits * 2) >= 128 && splits < 16) splits *= 2;
