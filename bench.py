@@ -161,6 +161,21 @@ def make_group(wl, dev, dsa, layers=None, indexer_layer=0, share_q=False):
     return ind, lays
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value (every rank takes part; world 1 returns x)."""
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step: int, world: int, ms_per_step: float) -> float:
+    """Whole-job units/s: every rank processes its own units each step (weak scaling), and the
+    step takes as long as the slowest rank."""
+    return units_per_rank_step * world / (ms_per_step / 1e3)
+
+
 def time_region(fn, steps, stream):
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
@@ -196,13 +211,9 @@ def run_ours(args, rank, world, dev):
     with ClockSampler(gpu_id(dev)) as clk:
         ms = time_region(step, args.steps, stream)
     launches = dsa.launch_count() - l0
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
     ms_step = ms / args.steps
-    q_per_step = wl.B * wl.T
-    value = q_per_step * world / (ms_step / 1e3)
+    value = job_throughput(wl.B * wl.T, world, ms_step)
 
     # ---- per-kernel breakdown: the same step as separate C-ABI calls with events between them
     brk = breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, args.steps if args.steps <= 3 else 3)
@@ -334,7 +345,7 @@ def run_e2e(args, wl, ind, lays, dev, stream):
     steps = max(1, min(args.steps, args.e2e_steps))
     ms = time_region(step, steps, stream) / steps
     del ws, g
-    return {"value": wl.B * wl.T / (ms / 1e3), "unit": "query tok/s", "ms_per_step": ms, "steps": steps,
+    return {"value": job_throughput(wl.B * wl.T, 1, ms), "unit": "query tok/s", "ms_per_step": ms, "steps": steps,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
@@ -489,9 +500,17 @@ def main():
     res, wl, ind, lays = run_ours(args, rank, world, dev)
     if not args.no_e2e:
         try:
-            res["e2e"] = run_e2e(args, wl, ind, lays, dev, torch.cuda.current_stream())
+            e2e = run_e2e(args, wl, ind, lays, dev, torch.cuda.current_stream())
         except (RuntimeError, torch.cuda.OutOfMemoryError) as e:  # pinned host memory can run out
-            res["e2e"] = {"error": str(e)[:300]}
+            e2e = {"error": str(e)[:300]}
+        # every rank joins the reduction, a failed one with an infinite time
+        ms = max_over_ranks(e2e.get("ms_per_step", math.inf), world, dev)
+        if "error" not in e2e:
+            if math.isfinite(ms):
+                e2e.update(value=job_throughput(wl.B * wl.T, world, ms), ms_per_step=ms)
+            else:
+                e2e = {"error": "the end-to-end step failed on another rank"}
+        res["e2e"] = e2e
     del ind, lays
     torch.cuda.empty_cache()
     if world > 1:

@@ -224,22 +224,126 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       if (!(ok = mbar_wait(b_full(bs), (b_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
       const float* wsm = reinterpret_cast<const float*>(sgen + C::OFF_W + bs * C::W_BYTES) + half * C::COLS;
       const int ctx_b = __ldg(ctx_len + g.b);
+      // H == 64: the 16x256b TMEM shape gives each thread 2 keys x 2 heads per 8-column group,
+      // always the same two heads (columns 2(lane%4), +1 of every group), so this thread's head
+      // weights live in registers for the whole work item: 8 packed pairs per query.
+      uint64_t wr[H == 64 ? C::QPH : 1][8];
+      if constexpr (H == 64) {
+#pragma unroll
+        for (int ql = 0; ql < C::QPH; ++ql)
+#pragma unroll
+          for (int gg = 0; gg < 8; ++gg)
+            wr[ql][gg] = *reinterpret_cast<const uint64_t*>(wsm + ql * H + 8 * gg + 2 * (lane & 3));
+      }
+      if constexpr (H == 64) {
+        // Each tile's accumulator slice comes to registers in STEPS loads, (query ql of this
+        // warp, row half rh of its 32 TMEM lanes) each, double-buffered in one flat pipeline
+        // across the tiles of the item: the next tile's first load is in flight while this
+        // tile's last step is summed and its sums are reduced across the quad and stored.
+        constexpr int STEPS = 2 * C::QPH;
+        static_assert(STEPS % 2 == 0, "buffer parity follows the step");
+        float v[2][32];
+        auto issue = [&](int ab, int st, float (&dst)[32]) {
+          tmem_ld_16x256b_x8(tmem_base + (uint32_t)(ab * C::N + half * C::COLS) +
+                                 ((uint32_t)(quad * 32 + (st & 1) * 16) << 16) + (uint32_t)((st >> 1) * H),
+                             dst);
+        };
+        auto store = [&](int ql, int s, float val) {
+          const int qq = half * C::QPH + ql;
+          if (qq < g.nq && s < S_max) {
+            const int t = g.t0 + qq;
+            const int pos = ctx_b - T + t;
+            scores[((int64_t)g.b * t_count + (t - t_begin)) * ld + s] = (s * pool <= pos) ? val : -INFINITY;
+          }
+        };
+        if (g.kt0 < g.kt1) {
+          if (!(ok = mbar_wait(acc_full(acc_cnt & 1), (acc_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
+          tc_fence_after();
+          issue(acc_cnt & 1, 0, v[0]);
+          tmem_ld_wait();
+          launder(v[0]);
+        }
+        for (int kt = g.kt0; kt < g.kt1; ++kt) {
+          const int ab = acc_cnt & 1;
+          const bool more = kt + 1 < g.kt1;
+          float red[2 * STEPS];  // per step: partial sums of key A (lane base + lane/4) and key B (+8)
+#pragma unroll
+          for (int st = 0; st < STEPS; ++st) {
+            if (st + 1 < STEPS) {
+              issue(ab, st + 1, v[(st + 1) & 1]);
+            } else {
+              // every load of this tile has completed: hand the accumulator back to the MMA
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(acc_empty(ab));
+              if (more) {
+                if (!(ok = mbar_wait(acc_full(ab ^ 1), ((acc_cnt + 1) >> 1) & 1, abort, kWaitLimitNs))) break;
+                tc_fence_after();
+                issue(ab ^ 1, 0, v[0]);
+              }
+            }
+            const float* vc = v[st & 1];
+            const int ql = st >> 1;
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};  // key A even/odd groups, key B even/odd
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+              const float* x = vc + 4 * r;
+              acc[r & 1] = ffma2(wr[ql][r], pack2(fmaxf(x[0], 0.f), fmaxf(x[1], 0.f)), acc[r & 1]);
+              acc[2 + (r & 1)] = ffma2(wr[ql][r], pack2(fmaxf(x[2], 0.f), fmaxf(x[3], 0.f)), acc[2 + (r & 1)]);
+            }
+            float xa0, xa1, xb0, xb1;
+            unpack2(fadd2(acc[0], acc[1]), xa0, xa1);
+            unpack2(fadd2(acc[2], acc[3]), xb0, xb1);
+            red[2 * st] = xa0 + xa1;
+            red[2 * st + 1] = xb0 + xb1;
+            if (st + 1 < STEPS) {
+              tmem_ld_wait();
+              launder(v[(st + 1) & 1]);
+            }
+          }
+          if (!ok) break;
+          ++acc_cnt;
+          // Sum over the 4 threads of a quad (each holds 16 of a query's 64 heads) as a
+          // transposing reduction: after the xor-1 round a thread keeps the values of its key
+          // (A on even lanes, B on odd), after the xor-2 round those of its row half.
+          const int odd = lane & 1, bit1 = (lane >> 1) & 1;
+          float k1[STEPS];
+#pragma unroll
+          for (int m = 0; m < STEPS; ++m) {
+            const float mine = odd ? red[2 * m + 1] : red[2 * m];
+            const float other = odd ? red[2 * m] : red[2 * m + 1];
+            k1[m] = mine + __shfl_xor_sync(0xffffffffu, other, 1);
+          }
+#pragma unroll
+          for (int n = 0; n < C::QPH; ++n) {
+            const float mine = bit1 ? k1[2 * n + 1] : k1[2 * n];
+            const float other = bit1 ? k1[2 * n] : k1[2 * n + 1];
+            store(n, kt * KTILE + quad * 32 + bit1 * 16 + (lane >> 2) + 8 * odd,
+                  mine + __shfl_xor_sync(0xffffffffu, other, 2));
+          }
+          if (more) {
+            tmem_ld_wait();
+            launder(v[0]);
+          }
+        }
+      } else {
       for (int kt = g.kt0; kt < g.kt1; ++kt) {
         const int ab = acc_cnt & 1;
         if (!(ok = mbar_wait(acc_full(ab), (acc_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
         tc_fence_after();
+        // finished sum of query ql (local to this warp) for key s -> masked store
+        auto store = [&](int ql, int s, float val) {
+          const int qq = half * C::QPH + ql;
+          if (qq < g.nq && s < S_max) {
+            const int t = g.t0 + qq;
+            const int pos = ctx_b - T + t;
+            scores[((int64_t)g.b * t_count + (t - t_begin)) * ld + s] = (s * pool <= pos) ? val : -INFINITY;
+          }
+        };
+        const uint32_t tcol = tmem_base + (uint32_t)(ab * C::N + half * C::COLS);
         {
-          const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(ab * C::N + half * C::COLS);
+          const uint32_t taddr = tcol + ((uint32_t)(quad * 32) << 16);
           const int s = kt * KTILE + row;
-          // finished sum of query ql (local to this warp) -> masked store
-          auto store = [&](int ql, float val) {
-            const int qq = half * C::QPH + ql;
-            if (qq < g.nq && s < S_max) {
-              const int t = g.t0 + qq;
-              const int pos = ctx_b - T + t;
-              scores[((int64_t)g.b * t_count + (t - t_begin)) * ld + s] = (s * pool <= pos) ? val : -INFINITY;
-            }
-          };
           // w * relu(x) over 4 columns into two packed accumulators
           auto quad4 = [&](const float* v, int col, uint64_t& a0, uint64_t& a1) {
             const float4 wv = *reinterpret_cast<const float4*>(wsm + col);
@@ -264,7 +368,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
               if ((c + 1) % (H / 32) == 0) {
                 float x0, x1, x2, x3, x4, x5, x6, x7;
                 unpack2(a2[0], x0, x1); unpack2(a2[1], x2, x3); unpack2(a2[2], x4, x5); unpack2(a2[3], x6, x7);
-                store(c / (H / 32), ((x0 + x1) + (x2 + x3)) + ((x4 + x5) + (x6 + x7)));
+                store(c / (H / 32), s, ((x0 + x1) + (x2 + x3)) + ((x4 + x5) + (x6 + x7)));
                 a2[0] = a2[1] = a2[2] = a2[3] = 0ull;
               }
             } else {
@@ -276,16 +380,17 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
                 for (int i = 0; i < H; i += 4) quad4(vc + qc * H + i, 32 * c + qc * H + i, b0, b1);
                 float x0, x1, x2, x3;
                 unpack2(b0, x0, x1); unpack2(b1, x2, x3);
-                store(c * (32 / H) + qc, (x0 + x1) + (x2 + x3));
+                store(c * (32 / H) + qc, s, (x0 + x1) + (x2 + x3));
               }
             }
             if (c + 1 < C::CHUNKS) tmem_ld_wait();
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty(ab));
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty(ab));
         ++acc_cnt;
+      }
       }
       if (!ok) break;
       __syncwarp();
