@@ -10,22 +10,24 @@
 //     (18 x tcgen05.mma M128 N64 K16 per tile of 64 keys), then swaps its partial with the
 //     partner through distributed shared memory; both add the two partials in the same
 //     order, so both hold the same scores, softmax and P;
-//   * accumulates O[:, 256c .. 256c+255] = P V in TMEM (2 x M128 N256 K16 per tile, V read
-//     MN-major straight from the gathered rows);
-//     (P.V: 4 x M128 N256 K16 per tile)
+//   * accumulates O[:, 256c .. 256c+255] = P V in TMEM (4 x M128 N256 K16 per tile, P read
+//     from TMEM, V read MN-major straight from the gathered rows);
 //   * gathers only the row columns it needs: c = 0 columns 0..287, c = 1 columns 256..575.
-// Per CTA: a 3-stage ring of 40 KB key tiles; TMEM 64 score + 144 q + 256 output columns.
+// Per CTA: a 4-stage ring of 40 KB key tiles; TMEM 64 score + 144 q + 32 P + 256 output
+// columns.
 //
-//   warps 0-3  softmax: thread = head.  Partial scores from TMEM -> a local stage -> per warp,
-//              one 8 KB bulk copy into the partner (completing that warp's barrier there);
-//              partner's partial
-//              + own -> masked scores; running max moved only when a tile exceeds it by more
-//              than 2^8 (then O is rescaled in TMEM); P = exp2(S - m) as bf16 in one of two
-//              shared-memory buffers, so a tile's softmax overlaps the previous tile's P.V; at the end O / l is written out (or a split partial with its lse).
-//              First, each thread stores its head's q columns into TMEM.
+//   warps 0-3  softmax: thread = head.  First each thread stores its head's q columns into
+//              TMEM.  Per tile j: (1) the partner's partial of tile j (sent a tile earlier)
+//              + our own -> masked scores and their max; a relaxed remote arrive, ordered
+//              after every read of the partner's rows by a data dependency, frees its buffer;
+//              (2) our partial of tile j+1 from TMEM -> a local stage -> per warp, one 8 KB
+//              bulk copy into the partner (completing that warp's barrier there), in flight
+//              while (3) the running max moves only when a tile exceeds it by more than 2^8
+//              (then O is rescaled in TMEM) and P = exp2(S - m) goes to TMEM as bf16 pairs.
+//              At the end O / l is written out (or a split partial with its lse).
 //   warps 4-6  gather: 16-byte cp.async of the selected rows into the 128-byte-swizzled
 //              K-major layout the tensor core reads (also V's MN-major layout).
-//   warp 7     TMEM owner and MMA issuer.
+//   warp 7     TMEM owner and MMA issuer: S_0, S_1, then per tile S_{j+2} ahead of P_j.V_j.
 // Every wait is bounded (tc_common.cuh); the two CTAs meet at cluster barriers only at start
 // and end.
 #include "common.cuh"
@@ -39,20 +41,18 @@ using namespace tc;
 
 constexpr int HQ = 128, DQK = 576, DV = 512, DVH = 256;
 constexpr int NK = 64;                  // keys per tile
-constexpr int NS = 3;                   // key-tile stages
+constexpr int NS = 4;                   // key-tile stages
 constexpr int BLKS = 5;                 // 64-column blocks of a key row held per CTA
 constexpr int K_BLK = NK * 128;         // 64 rows x 128 B
 constexpr int KSTEPS = 18;              // 288 score columns / 16 per MMA
 constexpr int KV_STAGE = BLKS * K_BLK;                 // 40960
 constexpr int OFF_KV = 0;
-constexpr int OFF_P = OFF_KV + NS * KV_STAGE;          // 2 P buffers: rows of 128 B (64 keys bf16)
-constexpr int P_BYTES = HQ * NK * 2;                   // 16384
 constexpr int X_BYTES = HQ * NK * 4;                   // 32768: one tile of fp32 partial scores
-constexpr int OFF_XS = OFF_P + 2 * P_BYTES;            // own partial, staged for the bulk copy out
+constexpr int OFF_XS = OFF_KV + NS * KV_STAGE;         // own partial, staged for the bulk copy out
 constexpr int OFF_X = OFF_XS + X_BYTES;                // partner's partial, copied in
 constexpr int OFF_IDS = OFF_X + X_BYTES;
 constexpr int OFF_BAR = OFF_IDS + NS * NK * 4 + 16 * NS;   // ids + an all-valid flag per stage
-constexpr int NBARS = 3 * NS + 22;
+constexpr int NBARS = 3 * NS + 13;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;       // + alignment slack
 constexpr int THREADS = 256;            // 8 warps: 2 per SM sub-partition, so up to 255 registers
@@ -61,16 +61,17 @@ constexpr int MMA_WARP = 7;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S = 0;      // partial scores, NK columns
 constexpr uint32_t COL_Q = 64;     // this CTA's 288 q columns as packed bf16 pairs: 144 columns
+constexpr uint32_t COL_P = 224;    // P of one tile as packed bf16 pairs (the P.V MMA's A operand): 32 columns
 constexpr uint32_t COL_O = 256;    // DVH output columns
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
 
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert((OFF_P % 1024) == 0 && (OFF_KV % 1024) == 0 && (OFF_X % 128) == 0 && (OFF_XS % 128) == 0, "alignment");
-static_assert(COL_Q + 144 <= COL_O && COL_S + NK <= COL_Q, "TMEM map");
+static_assert((OFF_KV % 1024) == 0 && (OFF_X % 128) == 0 && (OFF_XS % 128) == 0, "alignment");
+static_assert(COL_S + NK <= COL_Q && COL_Q + 144 <= COL_P && COL_P + NK / 2 <= COL_O, "TMEM map");
 
 constexpr uint32_t IDESC_S = instr_desc(128, NK, 1);                   // bf16, K-major A and B
-constexpr uint32_t IDESC_PV = instr_desc(128, DVH, 1) | (1u << 16);    // B (V) MN-major
+constexpr uint32_t IDESC_PV = instr_desc(128, DVH, 1) | (1u << 16);    // A (P) from TMEM, B (V) MN-major
 
 __device__ __forceinline__ uint64_t smem_desc_lbo(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
@@ -128,12 +129,13 @@ __device__ __forceinline__ uint32_t map_to_cta(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+// Relaxed arrive on a barrier in the partner CTA: no cluster-scope fence.  `dep` is a value
+// computed from every shared-memory load the arrive must follow, so those loads have returned
+// their data (and can no longer observe a later write) before the arrive is issued.
+__device__ __forceinline__ void mbar_arrive_cluster_after(uint32_t cluster_bar, float dep) {
+  asm volatile("{\n\t.reg .f32 d;\n\tmov.f32 d, %1;\n\t"
+               "mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];\n\t}\n" ::"r"(cluster_bar), "f"(dep)
                : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_bar) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -162,13 +164,6 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
     }
   }
 }
-// 16-byte asynchronous store into a cluster peer's shared memory; completes `bytes` of the
-// peer barrier's transaction count when it lands (no fence on the issuing side).
-__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t remote_bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];\n"
-               ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
-               : "memory");
-}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -193,12 +188,12 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   auto ids_ready = [&](int s) { return bar0 + 8u * (2 * NS + s); };
   const uint32_t s_full = bar0 + 8u * (3 * NS);
   const uint32_t s_empty = bar0 + 8u * (3 * NS + 1);
+  const uint32_t p_full = bar0 + 8u * (3 * NS + 2);
+  const uint32_t pv_done = bar0 + 8u * (3 * NS + 3);
+  const uint32_t q_ready = bar0 + 8u * (3 * NS + 4);
   // per softmax warp w (rows 32w..32w+31): the partner's rows landed / the partner read ours
-  auto x_full = [&](int w) { return bar0 + 8u * (3 * NS + 13 + w); };
-  auto x_free = [&](int w) { return bar0 + 8u * (3 * NS + 17 + w); };
-  auto p_full = [&](int s) { return bar0 + 8u * (3 * NS + 6 + s); };
-  auto pv_done = [&](int s) { return bar0 + 8u * (3 * NS + 8 + s); };
-  const uint32_t q_ready = bar0 + 8u * (3 * NS + 10);
+  auto x_full = [&](int w) { return bar0 + 8u * (3 * NS + 5 + w); };
+  auto x_free = [&](int w) { return bar0 + 8u * (3 * NS + 9 + w); };
   volatile int* ids_s = reinterpret_cast<volatile int*>(sgen + OFF_IDS);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(sgen + OFF_MISC + 4);
@@ -229,10 +224,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       mbar_init(x_full(w), 1);   // one expect-tx arrival per use, plus the partner's 8 KB
       mbar_init(x_free(w), 1);   // the partner's warp w, once it has read our rows
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(p_full(s), 4);
-      mbar_init(pv_done(s), 1);
-    }
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
     mbar_init(q_ready, 4);
     *abort = 0;
     fence_barrier_init();
@@ -295,32 +288,15 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     cp_async_wait<0>();
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
+    // Order: S_0, S_1, then for each tile j: S_{j+2} (as soon as the softmax has read S_{j+1})
+    // ahead of P_j.V_j (once P_j is in TMEM), so the next tile's scores are always ready when
+    // the softmax asks for them.  The key ring holds tiles j .. j+2 meanwhile.
     bool ok = true;
-    auto issue_pv = [&](int jj) -> bool {
-      const int pb = jj & 1;
-      if (!mbar_wait(p_full(pb), (jj >> 1) & 1, abort, kWaitLimitNs)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t stage = sbase + OFF_KV + (jj % NS) * KV_STAGE;
-#pragma unroll
-        for (int kk = 0; kk < NK / 16; ++kk) {
-          const uint64_t ad = smem_desc(sbase + OFF_P + pb * P_BYTES + kk * 32, 1024, kLayoutSw128);
-          // V columns 256*half .. +255 are the stage's blocks 0..3 for both CTAs; keys 16kk..
-          const uint64_t bd = smem_desc_lbo(stage + kk * 2048, K_BLK, 1024, kLayoutSw128);
-          mma_bf16(tmem + COL_O, ad, bd, IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(kv_empty(jj % NS));
-        mma_commit(pv_done(pb));
-      }
-      __syncwarp();
-      return true;
-    };
     const int ks0 = half * KSTEPS;
-    if (ntiles > 0) ok = mbar_wait(q_ready, 0, abort, kWaitLimitNs);
-    for (int j = 0; j < ntiles && ok; ++j) {
-      const int st = j % NS;
-      if (!(ok = mbar_wait(kv_full(st), (j / NS) & 1, abort, kWaitLimitNs))) break;
-      if (!(ok = mbar_wait(s_empty, (j & 1) ^ 1, abort, kWaitLimitNs))) break;
+    auto issue_s = [&](int jj) -> bool {
+      const int st = jj % NS;
+      if (!mbar_wait(kv_full(st), (jj / NS) & 1, abort, kWaitLimitNs)) return false;
+      if (!mbar_wait(s_empty, (jj & 1) ^ 1, abort, kWaitLimitNs)) return false;
       tc_fence_after();
       fence_proxy_async();
       if (lane == 0) {
@@ -336,9 +312,32 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         mma_commit(s_full);
       }
       __syncwarp();
-      if (j >= 1) ok = issue_pv(j - 1);
+      return true;
+    };
+    auto issue_pv = [&](int jj) -> bool {
+      if (!mbar_wait(p_full, jj & 1, abort, kWaitLimitNs)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t stage = sbase + OFF_KV + (jj % NS) * KV_STAGE;
+#pragma unroll
+        for (int kk = 0; kk < NK / 16; ++kk) {
+          // V columns 256*half .. +255 are the stage's blocks 0..3 for both CTAs; keys 16kk..
+          const uint64_t bd = smem_desc_lbo(stage + kk * 2048, K_BLK, 1024, kLayoutSw128);
+          mma_bf16_ts(tmem + COL_O, tmem + COL_P + 8u * kk, bd, IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(kv_empty(jj % NS));
+        mma_commit(pv_done);
+      }
+      __syncwarp();
+      return true;
+    };
+    if (ntiles > 0) ok = mbar_wait(q_ready, 0, abort, kWaitLimitNs);
+    if (ok && ntiles > 0) ok = issue_s(0);
+    if (ok && ntiles > 1) ok = issue_s(1);
+    for (int j = 0; j < ntiles && ok; ++j) {
+      if (j + 2 < ntiles && !(ok = issue_s(j + 2))) break;
+      ok = issue_pv(j);
     }
-    if (ok && ntiles > 0) ok = issue_pv(ntiles - 1);
   } else {
     // ------------------------------------------------------------ softmax + epilogue (warps 0-3)
     const int row = warp * 32 + lane;  // head
@@ -378,49 +377,50 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       if (lane == 0) mbar_arrive(q_ready);
     }
     const uint32_t sw = (uint32_t)(row & 7);
-    for (int j = 0; j < ntiles; ++j) {
-      const int xb = j & 1, pb = j & 1, st = j % NS;
-      if (!(ok = mbar_wait(s_full, j & 1, abort, kWaitLimitNs))) break;
+    // S_jj from TMEM into sv, then this warp's 32 rows of it into the partner's exchange buffer
+    // jj&1: staged locally, one 8 KB bulk copy that completes the partner's per-warp barrier.
+    // Sent one tile ahead, so the copy is in flight while the current tile is finished.
+    auto load_send = [&](int jj, float (&sv)[NK]) -> bool {
+      if (!mbar_wait(s_full, jj & 1, abort, kWaitLimitNs)) return false;
       tc_fence_after();
-      float s[NK];
-      tmem_ld32(tmem + lane_off + COL_S, *reinterpret_cast<float(*)[32]>(s));
-      tmem_ld32(tmem + lane_off + COL_S + 32, *reinterpret_cast<float(*)[32]>(s + 32));
+      tmem_ld32(tmem + lane_off + COL_S, *reinterpret_cast<float(*)[32]>(sv));
+      tmem_ld32(tmem + lane_off + COL_S + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_empty);
-      // ---- send this warp's 32 partial rows to the partner's warp: stage locally, one 8 KB
-      //      bulk copy that completes the partner's per-warp barrier (no CTA-wide sync)
-      {
-        if (lane == 0 && j >= 1) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
-        __syncwarp();
-        const uint32_t xs_row = sbase + OFF_XS + row * 256;
+      if (lane == 0 && jj >= 1) asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");  // stage free
+      __syncwarp();
+      const uint32_t xs_row = sbase + OFF_XS + row * 256;
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-          asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};\n" ::"r"(xs_row + ((c ^ sw) << 4)), "f"(s[4 * c]),
-                       "f"(s[4 * c + 1]), "f"(s[4 * c + 2]), "f"(s[4 * c + 3]));
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) {
-          // the partner's warp has read our previous rows out of its buffer
-          ok = mbar_wait_cluster(x_free(warp), (j & 1) ^ 1, abort);
-          if (ok) {
-            const uint32_t off = (uint32_t)(warp * 32 * 256);
-            asm volatile(
-                "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
-                "cp.async.bulk.commit_group;\n"
-                ::"r"(map_to_cta(sbase + OFF_X + off, partner)), "r"(sbase + OFF_XS + off), "r"((uint32_t)(X_BYTES / 4)),
-                  "r"(map_to_cta(x_full(warp), partner))
-                : "memory");
-          }
+      for (int c = 0; c < 16; ++c)
+        asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};\n" ::"r"(xs_row + ((c ^ sw) << 4)), "f"(sv[4 * c]),
+                     "f"(sv[4 * c + 1]), "f"(sv[4 * c + 2]), "f"(sv[4 * c + 3]));
+      fence_proxy_async();
+      __syncwarp();
+      bool good = true;
+      if (lane == 0) {
+        // the partner's warp has read what we sent last (tile jj-1): it read it before sending
+        // tile jj itself, so this wait is short
+        good = mbar_wait_cluster(x_free(warp), (jj & 1) ^ 1, abort);
+        if (good) {
+          const uint32_t off = (uint32_t)(warp * 32 * 256);
+          asm volatile(
+              "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+              "cp.async.bulk.commit_group;\n"
+              ::"r"(map_to_cta(sbase + OFF_X + off, partner)), "r"(sbase + OFF_XS + off),
+                "r"((uint32_t)(X_BYTES / 4)), "r"(map_to_cta(x_full(warp), partner))
+              : "memory");
         }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok) break;
       }
-      // ---- receive the partner's rows for this warp
-      if (!(ok = mbar_wait_cluster(x_full(warp), j & 1, abort))) break;
-      float o4[NK];
+      return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+    };
+    // Tile jj, first half: the partner's partial + ours -> masked scores and their max.
+    auto part1 = [&](int jj, float (&sv)[NK], float& mt) -> bool {
+      const int st = jj % NS;
+      if (!mbar_wait_cluster(x_full(warp), jj & 1, abort)) return false;
       {
+        // both CTAs add the partials in column order (0..287 first): the same scores in both
         const uint32_t xrow = sbase + OFF_X + row * 256;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
@@ -428,21 +428,17 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
           asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
                        : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                        : "r"(xrow + ((c ^ sw) << 4)));
-          o4[4 * c] = v.x; o4[4 * c + 1] = v.y; o4[4 * c + 2] = v.z; o4[4 * c + 3] = v.w;
+          sv[4 * c] = half == 0 ? sv[4 * c] + v.x : v.x + sv[4 * c];
+          sv[4 * c + 1] = half == 0 ? sv[4 * c + 1] + v.y : v.y + sv[4 * c + 1];
+          sv[4 * c + 2] = half == 0 ? sv[4 * c + 2] + v.z : v.z + sv[4 * c + 2];
+          sv[4 * c + 3] = half == 0 ? sv[4 * c + 3] + v.w : v.w + sv[4 * c + 3];
         }
       }
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(x_full(warp), X_BYTES / 4);        // arm this warp's next exchange
-        mbar_arrive_cluster(map_to_cta(x_free(warp), partner));  // the partner's warp may copy in again
-      }
-      // ---- masked full scores: both CTAs add the partials in column order (0..287 first)
-      if (!(ok = mbar_wait(ids_ready(st), (j / NS) & 1, abort, kWaitLimitNs))) break;
-      float mt = -INFINITY;   // in the log2 domain (scaled)
-      {
+      if (lane == 0) mbar_arrive_expect_tx(x_full(warp), X_BYTES / 4);   // arm the next exchange
+      if (!mbar_wait(ids_ready(st), (jj / NS) & 1, abort, kWaitLimitNs)) return false;
+      {   // tile max in the log2 domain (scaled)
         const bool all_valid = ids_s[NS * NK + 4 * st] != 0;
-#pragma unroll
-        for (int i = 0; i < NK; ++i) s[i] = half == 0 ? s[i] + o4[i] : o4[i] + s[i];   // same order in both CTAs
         if (!all_valid) {
           const uint32_t ids_addr = sbase + OFF_IDS + st * NK * 4;
 #pragma unroll
@@ -450,26 +446,35 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
             int4 id4;
             asm volatile("ld.shared.v4.s32 {%0,%1,%2,%3}, [%4];\n"
                          : "=r"(id4.x), "=r"(id4.y), "=r"(id4.z), "=r"(id4.w) : "r"(ids_addr + 16 * c));
-            if (id4.x < 0) s[4 * c] = -INFINITY;
-            if (id4.y < 0) s[4 * c + 1] = -INFINITY;
-            if (id4.z < 0) s[4 * c + 2] = -INFINITY;
-            if (id4.w < 0) s[4 * c + 3] = -INFINITY;
+            if (id4.x < 0) sv[4 * c] = -INFINITY;
+            if (id4.y < 0) sv[4 * c + 1] = -INFINITY;
+            if (id4.z < 0) sv[4 * c + 2] = -INFINITY;
+            if (id4.w < 0) sv[4 * c + 3] = -INFINITY;
           }
         }
         float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
         for (int i = 0; i < NK; i += 4) {
-          m0 = fmaxf(m0, s[i]); m1 = fmaxf(m1, s[i + 1]); m2 = fmaxf(m2, s[i + 2]); m3 = fmaxf(m3, s[i + 3]);
+          m0 = fmaxf(m0, sv[i]); m1 = fmaxf(m1, sv[i + 1]); m2 = fmaxf(m2, sv[i + 2]); m3 = fmaxf(m3, sv[i + 3]);
         }
         mt = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * scale_log2;   // scale > 0 commutes with max
       }
-      // ---- P buffer pb was last read by P.V of tile j-2
-      if (j >= 2 && !(ok = mbar_wait(pv_done(pb), ((j >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
+      // every value of the partner's rows has been read (mt depends on all of them, in every
+      // lane of this warp): the partner's warp may copy in again
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster_after(map_to_cta(x_free(warp), partner), mt);
+      return true;
+    };
+    // Tile jj, second half: running max, P_jj = exp2(s - m) into TMEM.
+    auto part2 = [&](int jj, float (&sv)[NK], float mt) -> bool {
+      // P.V of tile jj-1 has finished: the P columns are free and O holds tiles < jj
+      if (jj >= 1) {
+        if (!mbar_wait(pv_done, (jj - 1) & 1, abort, kWaitLimitNs)) return false;
+        tc_fence_after();
+      }
       if (mt > m_use + kRescaleLog2 || (m_use == -INFINITY && mt > -INFINITY)) {
         const float alpha = (m_use == -INFINITY) ? 0.f : ex2(m_use - mt);
-        if (j >= 1 && m_use != -INFINITY) {   // O already holds earlier tiles: rescale it
-          if (!(ok = mbar_wait(pv_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort, kWaitLimitNs))) break;
-          tc_fence_after();
+        if (jj >= 1 && m_use != -INFINITY) {   // O already holds earlier tiles: rescale it
 #pragma unroll 1
           for (int c = 0; c < DVH; c += 32) {
             float o[32];
@@ -479,36 +484,46 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
             tmem_st32(tmem + lane_off + COL_O + c, o);
           }
-          tmem_st_wait();
         }
         l_run *= alpha;
         m_use = mt;
       }
-      // ---- P = exp2(s - m_use) as bf16, one 128-byte swizzled row per head
+      // ---- P = exp2(s - m_use) as bf16 pairs (even key in the low half) into this lane's
+      //      32 P columns: the A operand of the P.V MMA
       {
-        const uint32_t prow = sbase + OFF_P + pb * P_BYTES + row * 128;
         const bool live = m_use != -INFINITY;
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0v = live ? ex2(fmaf(s[8 * c + 2 * e], scale_log2, -m_use)) : 0.f;
-            const float p1v = live ? ex2(fmaf(s[8 * c + 2 * e + 1], scale_log2, -m_use)) : 0.f;
-            l_run += p0v + p1v;
-            pk[e] = pack2_bf16(p0v, p1v);
-          }
-          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(prow + ((c ^ sw) << 4)), "r"(pk[0]),
-                       "r"(pk[1]), "r"(pk[2]), "r"(pk[3]));
+        for (int i = 0; i < 32; ++i) {
+          const float p0v = live ? ex2(fmaf(sv[2 * i], scale_log2, -m_use)) : 0.f;
+          const float p1v = live ? ex2(fmaf(sv[2 * i + 1], scale_log2, -m_use)) : 0.f;
+          l_run += p0v + p1v;
+          pk[i] = pack2_bf16(p0v, p1v);
         }
+        tmem_st32u(tmem + lane_off + COL_P, pk);
+        tmem_st_wait();
       }
-      fence_proxy_async();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full(pb));
+      if (lane == 0) mbar_arrive(p_full);
+      return true;
+    };
+    // Per tile j: part1(j), then the next tile's scores go out (their copy overlaps part2(j)),
+    // then part2(j).  Two score arrays alternate between the tiles.
+    float sa[NK], sb[NK];
+    float mt = -INFINITY;
+    if (ntiles > 0) ok = load_send(0, sa);
+    for (int j = 0; j < ntiles && ok; j += 2) {
+      if (!(ok = part1(j, sa, mt))) break;
+      if (j + 1 < ntiles && !(ok = load_send(j + 1, sb))) break;
+      if (!(ok = part2(j, sa, mt))) break;
+      if (j + 1 >= ntiles) break;
+      if (!(ok = part1(j + 1, sb, mt))) break;
+      if (j + 2 < ntiles && !(ok = load_send(j + 2, sa))) break;
+      if (!(ok = part2(j + 1, sb, mt))) break;
     }
     // ---- epilogue: wait for the last P.V, normalise, write
-    if (ok && ntiles > 0) ok = mbar_wait(pv_done((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1, abort, kWaitLimitNs);
+    if (ok && ntiles > 0) ok = mbar_wait(pv_done, (ntiles - 1) & 1, abort, kWaitLimitNs);
     tc_fence_after();
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
     const float lse_r = l_run > 0.f ? (m_use + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
