@@ -472,9 +472,14 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         if (!mbar_wait(pv_done, (jj - 1) & 1, abort, kWaitLimitNs)) return false;
         tc_fence_after();
       }
-      if (mt > m_use + kRescaleLog2 || (m_use == -INFINITY && mt > -INFINITY)) {
-        const float alpha = (m_use == -INFINITY) ? 0.f : ex2(m_use - mt);
-        if (jj >= 1 && m_use != -INFINITY) {   // O already holds earlier tiles: rescale it
+      // Lazy rescale, decided for the whole warp: the O round trip through TMEM is a
+      // warp-collective operation.  Every lane then moves to max(m_use, mt) with its own
+      // alpha (1 where its max did not move; O and l are still 0 where m_use was -inf).
+      const bool want = mt > m_use + kRescaleLog2 || (m_use == -INFINITY && mt > -INFINITY);
+      if (__any_sync(0xffffffffu, want)) {
+        const float m_new = fmaxf(m_use, mt);
+        const float alpha = (m_use == -INFINITY) ? 0.f : ex2(m_use - m_new);
+        if (jj >= 1) {   // O already holds earlier tiles: rescale it
 #pragma unroll 1
           for (int c = 0; c < DVH; c += 32) {
             float o[32];
@@ -486,7 +491,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
           }
         }
         l_run *= alpha;
-        m_use = mt;
+        m_use = m_new;
       }
       // ---- P = exp2(s - m_use) as bf16 pairs (even key in the low half) into this lane's
       //      32 P columns: the A operand of the P.V MMA
@@ -524,6 +529,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     }
     // ---- epilogue: wait for the last P.V, normalise, write
     if (ok && ntiles > 0) ok = mbar_wait(pv_done, (ntiles - 1) & 1, abort, kWaitLimitNs);
+    ok = __all_sync(0xffffffffu, ok);   // the TMEM reads below are warp-collective
     tc_fence_after();
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
     const float lse_r = l_run > 0.f ? (m_use + log2f(l_run)) * 0.69314718055994531f : -INFINITY;

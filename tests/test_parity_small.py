@@ -185,3 +185,24 @@ def test_attention_skips_negative_ids_anywhere():
                                P.to_np(lse[0, t]).astype(np.float64))
         assert msg is None, f"row {t}: {msg}"
     assert (P.bf16_np(out[0, 3]) == 0).all() and np.isneginf(P.to_np(lse[0, 3])).all()
+
+
+@pytest.mark.parametrize("q_scale", [6.0, 12.0, 20.0])
+def test_mla_peaked_softmax(q_scale):
+    """Logits 6-20x the unit-variance workload's (a peaked softmax: a few keys carry most of
+    the weight, and the running max moves by more than the lazy-rescale threshold inside a
+    row, so O is rescaled in TMEM mid-row).  Outputs reach |O| ~ 5, so the bf16 bounds are
+    taken in units of max(1, max|O|); the lse bound is unchanged."""
+    wl = W.WORKLOADS["prefill32k"].replace(T=256, ctx=4096)
+    L = W.make_attn_inputs(wl, 0, device=DEV)
+    q = (L["q"].float() * q_scale).to(torch.bfloat16)
+    g = torch.Generator(device="cpu").manual_seed(11)
+    idx = torch.stack([torch.randperm(4096 - 256, generator=g)[: wl.topk] for _ in range(wl.T)]).to(torch.int32)
+    idx = idx.view(1, wl.T, wl.topk).to(DEV)
+    out, lse = dsa.dsa_sparse_attn(q, L["kv"], idx, wl.sm_scale, wl.d_v, want_lse=True)
+    K = P.bf16_np(L["kv"][0])
+    idx_h = P.to_np(idx)
+    for t in (0, 1, 77, 128, 255):
+        msg = P.check_attn_row(P.bf16_np(out[0, t]), P.bf16_np(q[0, t]), K, K[:, : wl.d_v], idx_h[0, t], wl.sm_scale,
+                               P.to_np(lse[0, t]).astype(np.float64), out_scaled=True)
+        assert msg is None, f"row {t}: {msg}"
