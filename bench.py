@@ -230,7 +230,7 @@ def run_ours(args, rank, world, dev):
         "clocks": clk.summary(),
         "breakdown_ms": brk,
     }
-    res["roofline"] = roofline(wl, brk, pk)
+    res["roofline"] = roofline(wl, brk, pk, t_chunk)
     del g, ws
     torch.cuda.empty_cache()
     return res, wl, ind, lays
@@ -283,7 +283,14 @@ def breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, reps):
     return out
 
 
-def roofline(wl, brk, pk):
+# DRAM bytes (read + write) per query, from one ncu capture of the current kernels with the
+# bench's 131072-row context and 2048 queries (dram__bytes_read.sum + dram__bytes_write.sum per
+# launch / queries).  Per-query traffic does not depend on the number of queries, so a launch's
+# traffic is this figure times its queries.  Other contexts: not measured (None).
+TRAFFIC_PER_QUERY = {("prefill128k", "attn"): 552.3e3, ("prefill128k", "indexer"): 510.6e3}
+
+
+def roofline(wl, brk, pk, t_chunk):
     """Roofline of the kernel with the largest share of the step."""
     fp8_peak = 2.0 * pk["bf16_sus"]   # nominal fp8:bf16 ratio 2 on the measured bf16 figure
     ent = {
@@ -301,6 +308,9 @@ def roofline(wl, brk, pk):
                           "achieved": (wl.B * wl.S * wl.d_I + wl.B * wl.T * wl.H_I * (wl.d_I + 4))
                           / (brk["indexer"] * 1e-3) / 1e9,
                           "peak": pk["hbm_gbs"], "unit": "GB/s", "traffic": None, "peak_src": f"{pk['src']} copy"}
+    for k, queries in (("attn", wl.B * wl.T), ("indexer", wl.B * min(t_chunk, wl.T))):
+        per_q = TRAFFIC_PER_QUERY.get((wl.name, k))
+        ent[k]["traffic"] = None if per_q is None else per_q * queries   # bytes per launch
     top = max(("indexer", "attn"), key=lambda k: brk[k])
     r = dict(ent[top])
     r["kernel"] = top
@@ -366,7 +376,7 @@ def run_secondary(args, name, dev, steps=3, per_layer=False):
         ms = time_region(fn, steps, stream) / steps
         brk = breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, 3)
         r = {"workload": name, "value": wl.B * wl.T / (ms / 1e3), "unit": "query tok/s", "ms_per_step": ms,
-             "steps": steps, "breakdown_ms": brk, "roofline": roofline(wl, brk, peaks())}
+             "steps": steps, "breakdown_ms": brk, "roofline": roofline(wl, brk, peaks(), t_chunk)}
         del g, ws, ind, lays
         torch.cuda.empty_cache()
         return r
