@@ -14,7 +14,8 @@ Multi-GPU (torchrun, one process per GPU): every rank runs its own replica of th
 max-over-ranks time, scaling "weak".
 
 The JSON line also carries: the decode line (32 x 256K), the per-layer-indexer comparator
-at 128K with the IndexShare speedup, a per-kernel breakdown from CUDA events, the roofline
+at 128K with the IndexShare speedup, chunked prefill at a 1M-token cache without and with
+IndexPool (and that speedup), a per-kernel breakdown from CUDA events, the roofline
 of the dominant kernel, SM clocks sampled during the timed region, and the CPU oracle's
 throughput on a bounded sample (cpu_baseline).
 """
@@ -533,6 +534,14 @@ def main():
         except torch.cuda.OutOfMemoryError as e:  # pragma: no cover
             res["per_layer_indexer"] = {"error": str(e)[:200]}
         res["decode256k"] = run_secondary(args, "decode256k", dev, steps=10)
+        # IndexPool at a 1M-token cache: 8192 new queries, without and with pooling of 4 keys
+        for name in ("chunk1m", "chunk1m_pool"):
+            try:
+                res[name] = run_secondary(args, name, dev, steps=2)
+            except torch.cuda.OutOfMemoryError as e:  # pragma: no cover
+                res[name] = {"error": str(e)[:200]}
+        if "ms_per_step" in res["chunk1m"] and "ms_per_step" in res["chunk1m_pool"]:
+            res["indexpool_speedup_1m"] = res["chunk1m"]["ms_per_step"] / res["chunk1m_pool"]["ms_per_step"]
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
         v, rows, cores, spent = oracle_sample(W.WORKLOADS[args.workload], args.cpu_seconds)
         res["cpu_baseline"] = {"value": v, "unit": "query tok/s", "cores": cores, "kind": "oracle",

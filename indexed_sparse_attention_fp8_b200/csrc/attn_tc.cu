@@ -28,6 +28,11 @@
 //   warps 4-6  gather: 16-byte cp.async of the selected rows into the 128-byte-swizzled
 //              K-major layout the tensor core reads (also V's MN-major layout).
 //   warp 7     TMEM owner and MMA issuer: S_0, S_1, then per tile S_{j+2} ahead of P_j.V_j.
+// Persistent: one cluster per two SMs serves work items (query, key split) in turn, and every
+// barrier phase counts tiles over all its items.  At an item boundary the next query's q
+// (prefetched to L2 an item earlier) goes into TMEM before the previous query's O is read out,
+// so the MMA computes the next query's first scores meanwhile, and the gather warps run
+// straight on into the next query's rows.
 // Every wait is bounded (tc_common.cuh); the two CTAs meet at cluster barriers only at start
 // and end.
 #include "common.cuh"
@@ -173,10 +178,115 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
 
+// q[bt, head, 288*half .. +287] -> TMEM lane `head` (bf16 pairs packed per 32-bit column),
+// then this warp's arrival on q_ready.  Out of line: it runs once per query, and inlined its
+// registers would crowd the per-tile loop.
+__device__ __noinline__ void attn_load_q(const __nv_bfloat16* __restrict__ q, int bt, int row, int half, uint32_t tmem,
+                                         uint32_t lane_off, uint32_t q_ready, int lane) {
+      // q[head, 288*half .. +287] -> TMEM lane `head`, bf16 pairs packed per 32-bit column
+  const uint4* qsrc = reinterpret_cast<const uint4*>(q + ((int64_t)bt * HQ + row) * DQK + 288 * half);
+      // two batches of loads (16 + 20 x 16 B; the rows were prefetched to L2 an item earlier)
+      {
+        uint4 qa[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) qa[i] = __ldg(qsrc + i);
+        uint32_t w[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { w[4 * i] = qa[i].x; w[4 * i + 1] = qa[i].y; w[4 * i + 2] = qa[i].z; w[4 * i + 3] = qa[i].w; }
+        tmem_st32u(tmem + lane_off + COL_Q, w);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { w[4 * i] = qa[8 + i].x; w[4 * i + 1] = qa[8 + i].y; w[4 * i + 2] = qa[8 + i].z; w[4 * i + 3] = qa[8 + i].w; }
+        tmem_st32u(tmem + lane_off + COL_Q + 32, w);
+      }
+      {
+        uint4 qb[20];
+#pragma unroll
+        for (int i = 0; i < 20; ++i) qb[i] = __ldg(qsrc + 16 + i);
+        uint32_t w[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { w[4 * i] = qb[i].x; w[4 * i + 1] = qb[i].y; w[4 * i + 2] = qb[i].z; w[4 * i + 3] = qb[i].w; }
+        tmem_st32u(tmem + lane_off + COL_Q + 64, w);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { w[4 * i] = qb[8 + i].x; w[4 * i + 1] = qb[8 + i].y; w[4 * i + 2] = qb[8 + i].z; w[4 * i + 3] = qb[8 + i].w; }
+        tmem_st32u(tmem + lane_off + COL_Q + 96, w);
+        uint32_t w16[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { w16[4 * i] = qb[16 + i].x; w16[4 * i + 1] = qb[16 + i].y; w16[4 * i + 2] = qb[16 + i].z; w16[4 * i + 3] = qb[16 + i].w; }
+        tmem_st16u(tmem + lane_off + COL_Q + 128, w16);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
+
+// Epilogue of one item: waits for its last P.V, then O / l (or the split partial and its lse)
+// out of TMEM.  Out of line for the same reason as attn_load_q.
+__device__ __noinline__ bool attn_epilogue(int bt, int sp, int ntiles, float m_fin, float l_fin, uint32_t g_last,
+                                           bool good, int nbt, int row, int half, uint32_t tmem, uint32_t lane_off,
+                                           uint32_t pv_done, volatile int* abort, __nv_bfloat16* __restrict__ out,
+                                           float* __restrict__ lse, float* __restrict__ part_o,
+                                           float* __restrict__ part_lse) {
+      if (good && ntiles > 0) good = mbar_wait(pv_done, g_last & 1, abort, kWaitLimitNs);
+      good = __all_sync(0xffffffffu, good);   // the TMEM reads below are warp-collective
+      tc_fence_after();
+      const float inv = l_fin > 0.f ? 1.f / l_fin : 0.f;
+      const float lse_r = l_fin > 0.f ? (m_fin + log2f(l_fin)) * 0.69314718055994531f : -INFINITY;
+      const bool have_o = good && ntiles > 0;
+      const int64_t orow = (int64_t)bt * HQ + row;
+      if (part_o == nullptr) {
+        __nv_bfloat16* dst = out + orow * DV + half * DVH;
+#pragma unroll 1
+        for (int c = 0; c < DVH; c += 32) {
+          float o[32];
+          if (have_o) {
+            tmem_ld32(tmem + lane_off + COL_O + c, o);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 v;
+            v.x = pack2_bf16(o[i] * inv, o[i + 1] * inv);
+            v.y = pack2_bf16(o[i + 2] * inv, o[i + 3] * inv);
+            v.z = pack2_bf16(o[i + 4] * inv, o[i + 5] * inv);
+            v.w = pack2_bf16(o[i + 6] * inv, o[i + 7] * inv);
+            *reinterpret_cast<uint4*>(dst + c + i) = v;
+          }
+        }
+        if (lse != nullptr && half == 0) lse[orow] = lse_r;
+      } else {
+        const int64_t rows = (int64_t)nbt * HQ;
+        float* dst = part_o + ((int64_t)sp * rows + orow) * DV + half * DVH;
+#pragma unroll 1
+        for (int c = 0; c < DVH; c += 32) {
+          float o[32];
+          if (have_o) {
+            tmem_ld32(tmem + lane_off + COL_O + c, o);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + c + i) = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+        }
+        if (half == 0) part_lse[(int64_t)sp * rows + orow] = lse_r;
+      }
+      return good;
+    }
+
+struct Item {
+  int bt, sp, b, kbeg, kend, ntiles;
+};
+
 __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(THREADS, 1)
 sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv, int64_t kv_rs,
-                     int64_t kv_bs, const int32_t* __restrict__ idx, int T, int k, int keys_per_split,
-                     float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+                     int64_t kv_bs, const int32_t* __restrict__ idx, int T, int nbt, int items, int k,
+                     int keys_per_split, float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
                      float* __restrict__ part_o, float* __restrict__ part_lse) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
@@ -201,13 +311,19 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int half = (int)cluster_rank();       // 0 or 1: score columns 288*half.., output columns 256*half..
   const uint32_t partner = (uint32_t)(half ^ 1);
-  const int bt = blockIdx.x;
-  const int sp = blockIdx.z;
-  const int b = bt / T;
-  const int kbeg = sp * keys_per_split;
-  const int kend = min(k, kbeg + keys_per_split);
-  const int ntiles = kend > kbeg ? (kend - kbeg + NK - 1) / NK : 0;
-  const int32_t* irow = idx + (int64_t)bt * k;
+  // Work item it = (query bt = it % nbt, key split sp = it / nbt); the cluster takes items
+  // blockIdx.x, blockIdx.x + gridDim.x, ..  Every barrier phase below counts tiles (g) or
+  // items with tiles, over all the items this CTA has served.
+  auto geom = [&](int it) {
+    Item I;
+    I.bt = it % nbt;
+    I.sp = it / nbt;
+    I.b = I.bt / T;
+    I.kbeg = I.sp * keys_per_split;
+    I.kend = min(k, I.kbeg + keys_per_split);
+    I.ntiles = I.kend > I.kbeg ? (I.kend - I.kbeg + NK - 1) / NK : 0;
+    return I;
+  };
   const int blk0 = half == 0 ? 0 : 4;             // first 64-column block held by this CTA
   const int ch_lo = half == 0 ? 0 : 32;           // gathered 16-byte chunks [ch_lo, ch_hi) of a row
   const int ch_hi = half == 0 ? 36 : 72;
@@ -247,19 +363,23 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     // range, so each row is read with coalesced requests.  A tile's ids come from one
     // coalesced load per warp, issued a tile ahead, and reach the rows through shuffles.
     const int gw = warp - 4;
-    const __nv_bfloat16* kvb = kv + (int64_t)b * kv_bs;
+    bool ok = true;
+    uint32_t g = 0;   // tiles gathered so far
+    for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
+    const Item I = geom(it);
+    const __nv_bfloat16* kvb = kv + (int64_t)I.b * kv_bs;
+    const int32_t* irow = idx + (int64_t)I.bt * k;
     auto load_id = [&](int j, int r) -> int {
-      const int p = kbeg + j * NK + r;
-      return (j < ntiles && p < kend) ? __ldg(irow + p) : -1;
+      const int p = I.kbeg + j * NK + r;
+      return (j < I.ntiles && p < I.kend) ? __ldg(irow + p) : -1;
     };
     int id_next0 = load_id(0, lane), id_next1 = load_id(0, lane + 32);
-    bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      const int st = j % NS;
+    for (int j = 0; j < I.ntiles; ++j, ++g) {
+      const int st = g % NS;
       const int id0 = id_next0, id1 = id_next1;
       id_next0 = load_id(j + 1, lane);
       id_next1 = load_id(j + 1, lane + 32);
-      if (!(ok = mbar_wait(kv_empty(st), ((j / NS) & 1) ^ 1, abort, kWaitLimitNs))) break;
+      if (!(ok = mbar_wait(kv_empty(st), ((g / NS) & 1) ^ 1, abort, kWaitLimitNs))) break;
       if (gw == 0) {
         ids_s[st * NK + lane] = id0;
         ids_s[st * NK + 32 + lane] = id1;
@@ -285,6 +405,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       }
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(kv_full(st)) : "memory");
     }
+    }
     cp_async_wait<0>();
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
@@ -293,10 +414,10 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     // the softmax asks for them.  The key ring holds tiles j .. j+2 meanwhile.
     bool ok = true;
     const int ks0 = half * KSTEPS;
-    auto issue_s = [&](int jj) -> bool {
-      const int st = jj % NS;
-      if (!mbar_wait(kv_full(st), (jj / NS) & 1, abort, kWaitLimitNs)) return false;
-      if (!mbar_wait(s_empty, (jj & 1) ^ 1, abort, kWaitLimitNs)) return false;
+    auto issue_s = [&](uint32_t gg) -> bool {
+      const int st = gg % NS;
+      if (!mbar_wait(kv_full(st), (gg / NS) & 1, abort, kWaitLimitNs)) return false;
+      if (!mbar_wait(s_empty, (gg & 1) ^ 1, abort, kWaitLimitNs)) return false;
       tc_fence_after();
       fence_proxy_async();
       if (lane == 0) {
@@ -314,29 +435,36 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       __syncwarp();
       return true;
     };
-    auto issue_pv = [&](int jj) -> bool {
-      if (!mbar_wait(p_full, jj & 1, abort, kWaitLimitNs)) return false;
+    auto issue_pv = [&](uint32_t gg, bool first) -> bool {
+      if (!mbar_wait(p_full, gg & 1, abort, kWaitLimitNs)) return false;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t stage = sbase + OFF_KV + (jj % NS) * KV_STAGE;
+        const uint32_t stage = sbase + OFF_KV + (gg % NS) * KV_STAGE;
 #pragma unroll
         for (int kk = 0; kk < NK / 16; ++kk) {
           // V columns 256*half .. +255 are the stage's blocks 0..3 for both CTAs; keys 16kk..
           const uint64_t bd = smem_desc_lbo(stage + kk * 2048, K_BLK, 1024, kLayoutSw128);
-          mma_bf16_ts(tmem + COL_O, tmem + COL_P + 8u * kk, bd, IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + COL_O, tmem + COL_P + 8u * kk, bd, IDESC_PV, (!first || kk > 0) ? 1u : 0u);
         }
-        mma_commit(kv_empty(jj % NS));
+        mma_commit(kv_empty(gg % NS));
         mma_commit(pv_done);
       }
       __syncwarp();
       return true;
     };
-    if (ntiles > 0) ok = mbar_wait(q_ready, 0, abort, kWaitLimitNs);
-    if (ok && ntiles > 0) ok = issue_s(0);
-    if (ok && ntiles > 1) ok = issue_s(1);
-    for (int j = 0; j < ntiles && ok; ++j) {
-      if (j + 2 < ntiles && !(ok = issue_s(j + 2))) break;
-      ok = issue_pv(j);
+    uint32_t g = 0, nq = 0;   // tiles, and items with tiles, issued so far
+    for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
+      const Item I = geom(it);
+      if (I.ntiles == 0) continue;
+      if (!(ok = mbar_wait(q_ready, nq & 1, abort, kWaitLimitNs))) break;   // this item's q is in TMEM
+      ++nq;
+      ok = issue_s(g);
+      if (ok && I.ntiles > 1) ok = issue_s(g + 1);
+      for (int j = 0; j < I.ntiles && ok; ++j) {
+        if (j + 2 < I.ntiles && !(ok = issue_s(g + j + 2))) break;
+        ok = issue_pv(g + j, j == 0);
+      }
+      g += I.ntiles;
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue (warps 0-3)
@@ -344,43 +472,11 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     float m_use = -INFINITY, l_run = 0.f;
     bool ok = true;
-    {
-      // q[head, 288*half .. +287] -> TMEM lane `head`, bf16 pairs packed per 32-bit column
-      const uint4* qsrc = reinterpret_cast<const uint4*>(q + ((int64_t)bt * HQ + row) * DQK + 288 * half);
-      uint4 qa[16], qb[20];   // all 36 loads in flight together
-#pragma unroll
-      for (int i = 0; i < 16; ++i) qa[i] = __ldg(qsrc + i);
-#pragma unroll
-      for (int i = 0; i < 20; ++i) qb[i] = __ldg(qsrc + 16 + i);
-      {
-        uint32_t w[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) { w[4 * i] = qa[i].x; w[4 * i + 1] = qa[i].y; w[4 * i + 2] = qa[i].z; w[4 * i + 3] = qa[i].w; }
-        tmem_st32u(tmem + lane_off + COL_Q, w);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) { w[4 * i] = qa[8 + i].x; w[4 * i + 1] = qa[8 + i].y; w[4 * i + 2] = qa[8 + i].z; w[4 * i + 3] = qa[8 + i].w; }
-        tmem_st32u(tmem + lane_off + COL_Q + 32, w);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) { w[4 * i] = qb[i].x; w[4 * i + 1] = qb[i].y; w[4 * i + 2] = qb[i].z; w[4 * i + 3] = qb[i].w; }
-        tmem_st32u(tmem + lane_off + COL_Q + 64, w);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) { w[4 * i] = qb[8 + i].x; w[4 * i + 1] = qb[8 + i].y; w[4 * i + 2] = qb[8 + i].z; w[4 * i + 3] = qb[8 + i].w; }
-        tmem_st32u(tmem + lane_off + COL_Q + 96, w);
-        uint32_t w16[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) { w16[4 * i] = qb[16 + i].x; w16[4 * i + 1] = qb[16 + i].y; w16[4 * i + 2] = qb[16 + i].z; w16[4 * i + 3] = qb[16 + i].w; }
-        tmem_st16u(tmem + lane_off + COL_Q + 128, w16);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(q_ready);
-    }
     const uint32_t sw = (uint32_t)(row & 7);
     // S_jj from TMEM into sv, then this warp's 32 rows of it into the partner's exchange buffer
     // jj&1: staged locally, one 8 KB bulk copy that completes the partner's per-warp barrier.
     // Sent one tile ahead, so the copy is in flight while the current tile is finished.
-    auto load_send = [&](int jj, float (&sv)[NK]) -> bool {
+    auto load_send = [&](uint32_t jj, float (&sv)[NK]) -> bool {
       if (!mbar_wait(s_full, jj & 1, abort, kWaitLimitNs)) return false;
       tc_fence_after();
       tmem_ld32(tmem + lane_off + COL_S, *reinterpret_cast<float(*)[32]>(sv));
@@ -416,7 +512,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
     };
     // Tile jj, first half: the partner's partial + ours -> masked scores and their max.
-    auto part1 = [&](int jj, float (&sv)[NK], float& mt) -> bool {
+    auto part1 = [&](uint32_t jj, float (&sv)[NK], float& mt) -> bool {
       const int st = jj % NS;
       if (!mbar_wait_cluster(x_full(warp), jj & 1, abort)) return false;
       {
@@ -465,9 +561,9 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       if (lane == 0) mbar_arrive_cluster_after(map_to_cta(x_free(warp), partner), mt);
       return true;
     };
-    // Tile jj, second half: running max, P_jj = exp2(s - m) into TMEM.
-    auto part2 = [&](int jj, float (&sv)[NK], float mt) -> bool {
-      // P.V of tile jj-1 has finished: the P columns are free and O holds tiles < jj
+    // Tile jj (the item's tile j), second half: running max, P_jj = exp2(s - m) into TMEM.
+    auto part2 = [&](uint32_t jj, int j, float (&sv)[NK], float mt) -> bool {
+      // P.V of tile jj-1 has finished: the P columns are free and O holds the item's tiles < j
       if (jj >= 1) {
         if (!mbar_wait(pv_done, (jj - 1) & 1, abort, kWaitLimitNs)) return false;
         tc_fence_after();
@@ -479,7 +575,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       if (__any_sync(0xffffffffu, want)) {
         const float m_new = fmaxf(m_use, mt);
         const float alpha = (m_use == -INFINITY) ? 0.f : ex2(m_use - m_new);
-        if (jj >= 1) {   // O already holds earlier tiles: rescale it
+        if (j >= 1) {   // O already holds earlier tiles of this item: rescale it
 #pragma unroll 1
           for (int c = 0; c < DVH; c += 32) {
             float o[32];
@@ -513,69 +609,53 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       if (lane == 0) mbar_arrive(p_full);
       return true;
     };
-    // Per tile j: part1(j), then the next tile's scores go out (their copy overlaps part2(j)),
-    // then part2(j).  Two score arrays alternate between the tiles.
+    // Per item: the next item's q goes to L2 ahead of time; this item's q into TMEM (the S MMAs
+    // of the previous item have all finished: its last S has been read); then the previous
+    // item's O out of TMEM, while the MMA already computes this item's first scores; then the
+    // tiles.  Per tile j: part1(j), then the next tile's scores go out (their copy overlaps
+    // part2(j)), then part2(j).  Two score arrays alternate between the tiles.
     float sa[NK], sb[NK];
-    float mt = -INFINITY;
-    if (ntiles > 0) ok = load_send(0, sa);
-    for (int j = 0; j < ntiles && ok; j += 2) {
-      if (!(ok = part1(j, sa, mt))) break;
-      if (j + 1 < ntiles && !(ok = load_send(j + 1, sb))) break;
-      if (!(ok = part2(j, sa, mt))) break;
-      if (j + 1 >= ntiles) break;
-      if (!(ok = part1(j + 1, sb, mt))) break;
-      if (j + 2 < ntiles && !(ok = load_send(j + 2, sa))) break;
-      if (!(ok = part2(j + 1, sb, mt))) break;
-    }
-    // ---- epilogue: wait for the last P.V, normalise, write
-    if (ok && ntiles > 0) ok = mbar_wait(pv_done, (ntiles - 1) & 1, abort, kWaitLimitNs);
-    ok = __all_sync(0xffffffffu, ok);   // the TMEM reads below are warp-collective
-    tc_fence_after();
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    const float lse_r = l_run > 0.f ? (m_use + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
-    const bool have_o = ok && ntiles > 0;
-    const int64_t orow = (int64_t)bt * HQ + row;
-    if (part_o == nullptr) {
-      __nv_bfloat16* dst = out + orow * DV + half * DVH;
-#pragma unroll 1
-      for (int c = 0; c < DVH; c += 32) {
-        float o[32];
-        if (have_o) {
-          tmem_ld32(tmem + lane_off + COL_O + c, o);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0.f;
-        }
-#pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          uint4 v;
-          v.x = pack2_bf16(o[i] * inv, o[i + 1] * inv);
-          v.y = pack2_bf16(o[i + 2] * inv, o[i + 3] * inv);
-          v.z = pack2_bf16(o[i + 4] * inv, o[i + 5] * inv);
-          v.w = pack2_bf16(o[i + 6] * inv, o[i + 7] * inv);
-          *reinterpret_cast<uint4*>(dst + c + i) = v;
-        }
+    uint32_t g = 0;   // tiles served so far
+    int prev_it = -1;   // the item written out at the start of the next pass
+    float prev_m = -INFINITY, prev_l = 0.f;
+    // one pass more than there are items: the last pass only writes out the last item
+    for (int it = blockIdx.x;; it += gridDim.x) {
+      const bool real = it < items && ok;
+      Item I{};
+      if (real) I = geom(it);
+      if (real && warp == 0 && lane == 0 && it + (int)gridDim.x < items) {
+        const int bt_next = (it + (int)gridDim.x) % nbt;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(q + (int64_t)bt_next * HQ * DQK),
+                     "r"((uint32_t)(HQ * DQK * 2))
+                     : "memory");
       }
-      if (lse != nullptr && half == 0) lse[orow] = lse_r;
-    } else {
-      const int64_t rows = (int64_t)gridDim.x * HQ;
-      float* dst = part_o + ((int64_t)sp * rows + orow) * DV + half * DVH;
-#pragma unroll 1
-      for (int c = 0; c < DVH; c += 32) {
-        float o[32];
-        if (have_o) {
-          tmem_ld32(tmem + lane_off + COL_O + c, o);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0.f;
-        }
-#pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(dst + c + i) = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+      if (I.ntiles > 0) attn_load_q(q, I.bt, row, half, tmem, lane_off, q_ready, lane);
+      if (prev_it >= 0) {
+        const Item P = geom(prev_it);
+        ok = attn_epilogue(P.bt, P.sp, P.ntiles, prev_m, prev_l, g - 1, ok, nbt, row, half, tmem, lane_off, pv_done,
+                           abort, out, lse, part_o, part_lse);
       }
-      if (half == 0) part_lse[(int64_t)sp * rows + orow] = lse_r;
+      if (!real || !ok) break;
+      m_use = -INFINITY;
+      l_run = 0.f;
+      if (I.ntiles > 0) {
+        const uint32_t g0 = g;
+        float mt = -INFINITY;
+        ok = load_send(g0, sa);
+        for (int j = 0; j < I.ntiles && ok; j += 2) {
+          if (!(ok = part1(g0 + j, sa, mt))) break;
+          if (j + 1 < I.ntiles && !(ok = load_send(g0 + j + 1, sb))) break;
+          if (!(ok = part2(g0 + j, j, sa, mt))) break;
+          if (j + 1 >= I.ntiles) break;
+          if (!(ok = part1(g0 + j + 1, sb, mt))) break;
+          if (j + 2 < I.ntiles && !(ok = load_send(g0 + j + 2, sa))) break;
+          if (!(ok = part2(g0 + j + 1, j + 1, sb, mt))) break;
+        }
+        g += I.ntiles;
+      }
+      prev_it = it;
+      prev_m = m_use;
+      prev_l = l_run;
     }
   }
 
@@ -611,10 +691,14 @@ int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, i
     part_o = reinterpret_cast<float*>(ws);
     part_lse = part_o + (int64_t)splits * rows * DV;
   }
-  dim3 grid((unsigned)(B * T), 2, splits);
+  // persistent: one cluster (CTA pair) per two SMs, each serving items (query, key split) in turn
+  const int nbt = B * T;
+  const int items = nbt * splits;
+  const int nclu = std::max(1, std::min(items, num_sms() / 2));
+  dim3 grid((unsigned)nclu, 2, 1);
   sparse_mla_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(
-      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(kv), kv_rs, kv_bs, idx, T, k,
-      kps, sm_scale * 1.4426950408889634f, reinterpret_cast<__nv_bfloat16*>(out), lse, part_o, part_lse);
+      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(kv), kv_rs, kv_bs, idx, T, nbt,
+      items, k, kps, sm_scale * 1.4426950408889634f, reinterpret_cast<__nv_bfloat16*>(out), lse, part_o, part_lse);
   int st = check_launch();
   if (st != DSA_OK || splits == 1) return st;
   return launch_attn_combine(part_o, part_lse, splits, rows, DV, out, lse, stream);
