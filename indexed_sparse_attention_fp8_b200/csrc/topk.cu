@@ -54,17 +54,31 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_buf, int* total)
   return excl;
 }
 
-// Calls fn(i, score) for every i in [0, n), 16-byte loads where the row allows.
+// Calls fn(i, score) for every i in [0, n), 16-byte loads where the row allows.  Each thread
+// issues TK_UNROLL loads before it consumes any, so a pass over a long row is not a chain of
+// one-load round trips to L2.
+constexpr int TK_UNROLL = 4;
 template <typename F>
 __device__ __forceinline__ void for_each_score(const float* __restrict__ row, int n, F&& fn) {
   const int n4 = n >> 2;
   const float4* r4 = reinterpret_cast<const float4*>(row);
-  for (int v = threadIdx.x; v < n4; v += TK_THREADS) {
-    const float4 f = __ldcs(r4 + v);
-    fn(4 * v + 0, f.x);
-    fn(4 * v + 1, f.y);
-    fn(4 * v + 2, f.z);
-    fn(4 * v + 3, f.w);
+  for (int v0 = threadIdx.x; v0 < n4; v0 += TK_UNROLL * TK_THREADS) {
+    float4 f[TK_UNROLL];
+#pragma unroll
+    for (int u = 0; u < TK_UNROLL; ++u) {
+      const int v = v0 + u * TK_THREADS;
+      if (v < n4) f[u] = __ldcs(r4 + v);
+    }
+#pragma unroll
+    for (int u = 0; u < TK_UNROLL; ++u) {
+      const int v = v0 + u * TK_THREADS;
+      if (v < n4) {
+        fn(4 * v + 0, f[u].x);
+        fn(4 * v + 1, f[u].y);
+        fn(4 * v + 2, f[u].z);
+        fn(4 * v + 3, f[u].w);
+      }
+    }
   }
   for (int i = 4 * n4 + threadIdx.x; i < n; i += TK_THREADS) fn(i, __ldcs(row + i));
 }

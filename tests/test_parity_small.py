@@ -206,3 +206,24 @@ def test_mla_peaked_softmax(q_scale):
         msg = P.check_attn_row(P.bf16_np(out[0, t]), P.bf16_np(q[0, t]), K, K[:, : wl.d_v], idx_h[0, t], wl.sm_scale,
                                P.to_np(lse[0, t]).astype(np.float64), out_scaled=True)
         assert msg is None, f"row {t}: {msg}"
+
+
+def test_topk_long_rows_exact_with_ties():
+    """Long rows given as fp32 scores directly: the selected set must equal the oracle's
+    exactly, with exact ties resolved to the lowest indices (an all-tied row, and a row of
+    small integers with thousands of keys tied at the pivot), ids ascending and -1 padding; a
+    row with fewer visible keys than k selects them all."""
+    S, k, B, T = 20000, 2048, 4, 1
+    g = torch.Generator(device="cpu").manual_seed(3)
+    sc = torch.randn(B, T, S, generator=g)
+    sc[0] = 0.0                                                       # all tied: ids 0..2047
+    sc[1, 0] = torch.randint(0, 50, (S,), generator=g).float()        # heavy ties at the pivot
+    ctx = torch.tensor([S, S, 15000, 1500], dtype=torch.int32)
+    idx = dsa.dsa_topk(sc.to(DEV), ctx.to(DEV), T, S, k)
+    for b in range(B):
+        n_valid = min(S, int(ctx[b]))
+        ref = O.topk_row(sc[b, 0].numpy(), n_valid, k)
+        got = P.to_np(idx[b, 0])
+        valid = got[got >= 0]
+        assert np.array_equal(np.sort(valid), np.sort(ref[ref >= 0])), f"row {b}"
+        assert (np.diff(valid) > 0).all() and (got[valid.size:] == -1).all(), f"row {b}"
