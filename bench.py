@@ -288,7 +288,7 @@ def breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, reps):
 # bench's 131072-row context and 2048 queries (dram__bytes_read.sum + dram__bytes_write.sum per
 # launch / queries).  Per-query traffic does not depend on the number of queries, so a launch's
 # traffic is this figure times its queries.  Other contexts: not measured (None).
-TRAFFIC_PER_QUERY = {("prefill128k", "attn"): 552.3e3, ("prefill128k", "indexer"): 510.6e3}
+TRAFFIC_PER_QUERY = {("prefill128k", "attn"): 587.6e3, ("prefill128k", "indexer"): 510.5e3}
 
 
 def roofline(wl, brk, pk, t_chunk):
