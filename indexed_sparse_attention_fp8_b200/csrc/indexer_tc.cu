@@ -248,13 +248,22 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
                                  ((uint32_t)(quad * 32 + (st & 1) * 16) << 16) + (uint32_t)((st >> 1) * H),
                              dst);
         };
-        auto store = [&](int ql, int s, float val) {
+        // per query of this warp: its score row, its causal limit (last visible key row) and
+        // whether it exists in this block; a store is then an add, a compare and a select
+        float* qrow[C::QPH];
+        int lim[C::QPH];
+        bool qok[C::QPH];
+#pragma unroll
+        for (int ql = 0; ql < C::QPH; ++ql) {
           const int qq = half * C::QPH + ql;
-          if (qq < g.nq && s < S_max) {
-            const int t = g.t0 + qq;
-            const int pos = ctx_b - T + t;
-            scores[((int64_t)g.b * t_count + (t - t_begin)) * ld + s] = (s * pool <= pos) ? val : -INFINITY;
-          }
+          const int t = g.t0 + qq;
+          qok[ql] = qq < g.nq;
+          qrow[ql] = scores + ((int64_t)g.b * t_count + (t - t_begin)) * ld;
+          const int pos = ctx_b - T + t;
+          lim[ql] = pos < 0 ? -1 : pos / pool;   // s * pool <= pos  <=>  s <= pos / pool
+        }
+        auto store = [&](int ql, int s, float val) {
+          if (qok[ql] && s < S_max) qrow[ql][s] = (s <= lim[ql]) ? val : -INFINITY;
         };
         if (g.kt0 < g.kt1) {
           if (!(ok = mbar_wait(acc_full(acc_cnt & 1), (acc_cnt >> 1) & 1, abort, kWaitLimitNs))) break;

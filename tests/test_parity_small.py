@@ -212,13 +212,16 @@ def test_topk_long_rows_exact_with_ties():
     """Long rows given as fp32 scores directly: the selected set must equal the oracle's
     exactly, with exact ties resolved to the lowest indices (an all-tied row, and a row of
     small integers with thousands of keys tied at the pivot), ids ascending and -1 padding; a
-    row with fewer visible keys than k selects them all."""
-    S, k, B, T = 20000, 2048, 4, 1
+    row with fewer visible keys than k selects them all.  Rows this long and this few are split
+    over a cluster of CTAs, so the tied winners also span the CTAs' slices."""
+    S, k, B, T = 20000, 2048, 5, 1
     g = torch.Generator(device="cpu").manual_seed(3)
     sc = torch.randn(B, T, S, generator=g)
     sc[0] = 0.0                                                       # all tied: ids 0..2047
     sc[1, 0] = torch.randint(0, 50, (S,), generator=g).float()        # heavy ties at the pivot
-    ctx = torch.tensor([S, S, 15000, 1500], dtype=torch.int32)
+    sc[4] = 0.0
+    sc[4, 0, ::7] = 1.0                                               # the winners: every 7th id up to 14329
+    ctx = torch.tensor([S, S, 15000, 1500, S], dtype=torch.int32)
     idx = dsa.dsa_topk(sc.to(DEV), ctx.to(DEV), T, S, k)
     for b in range(B):
         n_valid = min(S, int(ctx[b]))
