@@ -4,10 +4,13 @@
 //
 // One CTA per row.  Radix select on order-preserving 32-bit keys (larger float -> larger
 // unsigned key), three digit passes (11 + 11 + 10 bits) with shared-memory histograms, each
-// pass restricted to the keys that share the digits fixed so far, stopping as soon as the
-// pivot bucket is taken whole.  Then one pass emits the winners: every key above the pivot
-// prefix, plus the lowest-indexed keys equal to it (the same tie rule as a sort by
-// (score desc, index asc)).  The winners are sorted ascending in shared memory (bitonic)
+// restricted to the keys that share the digits fixed so far, stopping as soon as the pivot
+// bucket is taken whole.  When the first digit's pivot bucket fits (TK_CAP keys), one more
+// pass over the row takes every key above it as a winner and copies the bucket (key, id) to
+// shared memory; the other digits and the ties are then resolved on the copy, so a row is
+// read twice instead of up to five times.  Otherwise the digits run over the row and a last
+// pass emits the winners.  Either way the winners are every key above the pivot prefix plus
+// the lowest-indexed keys equal to it (the same tie rule as a sort by (score desc, index asc)).  The winners are sorted ascending in shared memory (bitonic)
 // so the attention gathers walk the KV cache in address order, and written out, expanded
 // to token ids when the scores were over IndexPool blocks.
 #include "common.cuh"
@@ -21,6 +24,8 @@ namespace {
 constexpr int TK_THREADS = 1024;
 constexpr int TK_KMAX = 2048;
 constexpr int TK_BINS = 2048;
+constexpr int TK_CAP = 8192;   // candidate buffer (keys, ids, tie ids) in dynamic shared memory
+constexpr int TK_DYN_SMEM = 3 * TK_CAP * 4;
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f);
@@ -137,20 +142,31 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __
     return;
   }
   const float* row = scores + (int64_t)row_id * ld;
+  extern __shared__ uint32_t cand_smem[];
+  uint32_t* ck = cand_smem;                                            // candidate keys
+  int* ci = reinterpret_cast<int*>(cand_smem + TK_CAP);                 // their row indices
+  int* tie = reinterpret_cast<int*>(cand_smem + 2 * TK_CAP);            // ids tied at the pivot
 
   // ---- radix select of the k-th largest key
   uint32_t prefix = 0, mask = 0;
   int kk = k;          // winners still to find among keys matching `prefix` under `mask`
   int eq_count = 0;    // keys matching the final prefix
   const int shifts[3] = {21, 10, 0};
-  for (int p = 0; p < 3; ++p) {
-    const int shift = shifts[p];
+  // one digit pass over the keys matching prefix/mask (from the row, or from the candidates)
+  auto digit_pass = [&](int shift, bool from_cand, int ncand) {
     for (int i = tid; i < TK_BINS; i += TK_THREADS) hist[i] = 0u;
     __syncthreads();
-    for_each_score(row, n_valid, [&](int, float f) {
-      const uint32_t key = order_key(f);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (TK_BINS - 1)], 1u);
-    });
+    if (from_cand) {
+      for (int j = tid; j < ncand; j += TK_THREADS) {
+        const uint32_t key = ck[j];
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (TK_BINS - 1)], 1u);
+      }
+    } else {
+      for_each_score(row, n_valid, [&](int, float f) {
+        const uint32_t key = order_key(f);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (TK_BINS - 1)], 1u);
+      });
+    }
     __syncthreads();
     // thread tid owns bins hb and hb-1, scanned from the top bin down
     const int hb = TK_BINS - 1 - 2 * tid;
@@ -167,176 +183,83 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __
     prefix |= (uint32_t)sh_bin << shift;
     mask |= (uint32_t)(TK_BINS - 1) << shift;
     eq_count = sh_cnt;
-    if (eq_count == kk) break;  // the whole pivot bucket is selected (block-uniform)
-  }
+  };
 
-  // ---- emit winners: all keys above the prefix, then kk of the keys equal to it
-  if (tid == 0) { sh_ngt = 0; sh_neq = 0; }
-  __syncthreads();
-  const int n_gt = k - kk;
-  const bool take_all_eq = (eq_count == kk);
-  for_each_score(row, n_valid, [&](int i, float f) {
-    const uint32_t m = order_key(f) & mask;
-    if (m > prefix) {
-      sel[atomicAdd(&sh_ngt, 1)] = i;
-    } else if (take_all_eq && m == prefix) {
-      sel[n_gt + atomicAdd(&sh_neq, 1)] = i;
+  digit_pass(shifts[0], false, 0);
+  const int n_gt_1 = k - kk;   // keys above the first pivot digit: all winners
+  if (eq_count != kk && eq_count <= TK_CAP) {
+    // ---- the pivot bucket fits in shared memory: one more pass over the row takes the keys
+    //      above it as winners and copies the bucket; the rest works on the copy
+    if (tid == 0) { sh_ngt = 0; sh_neq = 0; }
+    __syncthreads();
+    for_each_score(row, n_valid, [&](int i, float f) {
+      const uint32_t key = order_key(f);
+      const uint32_t m = key & mask;
+      if (m > prefix) {
+        sel[atomicAdd(&sh_ngt, 1)] = i;
+      } else if (m == prefix) {
+        const int j = atomicAdd(&sh_neq, 1);
+        ck[j] = key;
+        ci[j] = i;
+      }
+    });
+    __syncthreads();
+    const int ncand = sh_neq;   // == eq_count
+    for (int p = 1; p < 3 && eq_count != kk; ++p) digit_pass(shifts[p], true, ncand);
+    // winners among the candidates: above the final prefix, then the ties (all, or the kk
+    // lowest ids)
+    const bool take_all_eq = (eq_count == kk);
+    if (tid == 0) { sh_ngt = n_gt_1; sh_neq = 0; }
+    __syncthreads();
+    for (int j = tid; j < ncand; j += TK_THREADS) {
+      const uint32_t m = ck[j] & mask;
+      if (m > prefix) {
+        sel[atomicAdd(&sh_ngt, 1)] = ci[j];
+      } else if (m == prefix) {
+        tie[atomicAdd(&sh_neq, 1)] = ci[j];
+      }
     }
-  });
-  if (!take_all_eq) {
-    // exact ties at the k-th key: the lowest indices win (ordered block compaction)
-    int base = 0;
-    for (int c0 = 0; c0 < n_valid && base < kk; c0 += TK_THREADS) {
-      const int i = c0 + tid;
-      const int eq = (i < n_valid) && ((order_key(row[i]) & mask) == prefix);
-      int total;
-      const int r = block_excl_scan(eq, warp_buf, &total);
-      if (eq && base + r < kk) sel[n_gt + base + r] = i;
-      base += total;
+    __syncthreads();
+    const int n_gt = sh_ngt, nties = sh_neq;   // n_gt == k - kk
+    if (!take_all_eq) sort_ascending(tie, nties);   // the lowest ids win
+    __syncthreads();
+    for (int j = tid; j < kk; j += TK_THREADS) sel[n_gt + j] = tie[j];
+    __syncthreads();
+  } else {
+    // ---- the pivot bucket is taken whole, or too large to copy: digit passes over the row
+    for (int p = 1; p < 3 && eq_count != kk; ++p) digit_pass(shifts[p], false, 0);
+
+    // ---- emit winners: all keys above the prefix, then kk of the keys equal to it
+    if (tid == 0) { sh_ngt = 0; sh_neq = 0; }
+    __syncthreads();
+    const int n_gt = k - kk;
+    const bool take_all_eq = (eq_count == kk);
+    for_each_score(row, n_valid, [&](int i, float f) {
+      const uint32_t m = order_key(f) & mask;
+      if (m > prefix) {
+        sel[atomicAdd(&sh_ngt, 1)] = i;
+      } else if (take_all_eq && m == prefix) {
+        sel[n_gt + atomicAdd(&sh_neq, 1)] = i;
+      }
+    });
+    if (!take_all_eq) {
+      // exact ties at the k-th key: the lowest indices win (ordered block compaction)
+      int base = 0;
+      for (int c0 = 0; c0 < n_valid && base < kk; c0 += TK_THREADS) {
+        const int i = c0 + tid;
+        const int eq = (i < n_valid) && ((order_key(row[i]) & mask) == prefix);
+        int total;
+        const int r = block_excl_scan(eq, warp_buf, &total);
+        if (eq && base + r < kk) sel[n_gt + base + r] = i;
+        base += total;
+      }
     }
+    __syncthreads();
   }
-  __syncthreads();
 
   // ---- ascending bitonic sort of the k winners
   sort_ascending(sel, k);
   for (int i = tid; i < k; i += TK_THREADS) write_expanded(out, i, sel[i], pool, pos);
-}
-
-// ---- few long rows (decode): a cluster of TK_CL CTAs per row, each over a 1/TK_CL slice
-constexpr int TK_CL = 4;
-
-__device__ __forceinline__ uint32_t cl_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cl_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
-}
-// A 32-bit word of CTA `rank`'s shared memory at the address of `p` in this CTA.
-__device__ __forceinline__ uint32_t ld_cluster_u32(const void* p, uint32_t rank) {
-  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
-  uint32_t r, v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(a), "r"(rank));
-  asm volatile("ld.shared::cluster.u32 %0, [%1];\n" : "=r"(v) : "r"(r) : "memory");
-  return v;
-}
-
-// The selection of topk_rows_kernel with the row split over the TK_CL CTAs of a cluster:
-// each pass sums the CTAs' histograms through distributed shared memory (every CTA derives
-// the same pivot), and the winners come out in index order because CTA c's slice holds lower
-// indices than CTA c+1's: each CTA takes its keys above the pivot prefix plus its share of
-// the lowest-indexed ties, sorts them, and writes them after the lower CTAs' winners.
-__global__ void __cluster_dims__(TK_CL, 1, 1) __launch_bounds__(TK_THREADS, 1)
-topk_rows_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ ctx_len,
-                         int T, int S_max, int pool, int t_begin, int t_count, int k,
-                         int32_t* __restrict__ idx_out) {
-  __shared__ uint32_t hist[TK_BINS];
-  __shared__ int sel[TK_KMAX];
-  __shared__ int warp_buf[32];
-  __shared__ int sh_bin, sh_above, sh_cnt, sh_ngt, sh_neq;
-  __shared__ int sh_counts[2];   // this CTA's keys above the prefix / equal to it
-
-  const int tid = threadIdx.x;
-  const uint32_t rank = cl_rank();
-  const int row_id = blockIdx.x / TK_CL;
-  const int b = row_id / t_count;
-  const int t = t_begin + row_id % t_count;
-  const int pos = ctx_len[b] - T + t;
-  const int n_valid = pos < 0 ? 0 : min(S_max, pos / pool + 1);
-  int32_t* out = idx_out + ((int64_t)b * T + t) * (int64_t)k * pool;
-
-  if (n_valid <= k) {  // every visible key is selected (the same for the whole cluster)
-    for (int i = (int)rank * TK_THREADS + tid; i < k; i += TK_CL * TK_THREADS)
-      write_expanded(out, i, i < n_valid ? i : -1, pool, pos);
-    return;
-  }
-  // this CTA's slice [lo, lo + len), 4-aligned so the 16-byte loads stay aligned
-  const int per = ((n_valid + TK_CL - 1) / TK_CL + 3) & ~3;
-  const int lo = min(n_valid, (int)rank * per);
-  const int len = min(n_valid, lo + per) - lo;
-  const float* row = scores + (int64_t)row_id * ld + lo;
-
-  uint32_t prefix = 0, mask = 0;
-  int kk = k;
-  int eq_count = 0;
-  const int shifts[3] = {21, 10, 0};
-  for (int p = 0; p < 3; ++p) {
-    const int shift = shifts[p];
-    for (int i = tid; i < TK_BINS; i += TK_THREADS) hist[i] = 0u;
-    __syncthreads();
-    for_each_score(row, len, [&](int, float f) {
-      const uint32_t key = order_key(f);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (TK_BINS - 1)], 1u);
-    });
-    cl_sync();   // every CTA's histogram is complete
-    const int hb = TK_BINS - 1 - 2 * tid;
-    int h0 = 0, h1 = 0;
-#pragma unroll
-    for (int r = 0; r < TK_CL; ++r) {
-      h0 += (int)ld_cluster_u32(&hist[hb], (uint32_t)r);
-      h1 += (int)ld_cluster_u32(&hist[hb - 1], (uint32_t)r);
-    }
-    cl_sync();   // every CTA has read every histogram before any is cleared again
-    int total;
-    const int excl = block_excl_scan(h0 + h1, warp_buf, &total);
-    if (excl < kk && kk <= excl + h0) {
-      sh_bin = hb; sh_above = excl; sh_cnt = h0;
-    } else if (excl + h0 < kk && kk <= excl + h0 + h1) {
-      sh_bin = hb - 1; sh_above = excl + h0; sh_cnt = h1;
-    }
-    __syncthreads();
-    kk -= sh_above;
-    prefix |= (uint32_t)sh_bin << shift;
-    mask |= (uint32_t)(TK_BINS - 1) << shift;
-    eq_count = sh_cnt;
-    if (eq_count == kk) break;  // the same merged histogram in every CTA: cluster-uniform
-  }
-
-  // ---- this CTA's counts above / equal to the prefix, shared with the cluster
-  if (tid == 0) { sh_ngt = 0; sh_neq = 0; }
-  __syncthreads();
-  for_each_score(row, len, [&](int, float f) {
-    const uint32_t m = order_key(f) & mask;
-    if (m > prefix) atomicAdd(&sh_ngt, 1);
-    else if (m == prefix) atomicAdd(&sh_neq, 1);
-  });
-  __syncthreads();
-  if (tid == 0) { sh_counts[0] = sh_ngt; sh_counts[1] = sh_neq; }
-  cl_sync();
-  // the lowest-indexed kk ties win: CTA c takes ties after those of the lower CTAs
-  int out_off = 0, eq_before = 0;
-  for (int r = 0; r < (int)rank; ++r) {
-    const int gt_r = (int)ld_cluster_u32(&sh_counts[0], (uint32_t)r);
-    const int eq_r = (int)ld_cluster_u32(&sh_counts[1], (uint32_t)r);
-    out_off += gt_r + min(eq_r, max(0, kk - eq_before));
-    eq_before += eq_r;
-  }
-  const int my_gt = sh_counts[0];
-  const int my_eq_take = min(sh_counts[1], max(0, kk - eq_before));
-  cl_sync();   // the counts have been read before any CTA may leave
-
-  // ---- collect this CTA's winners (row indices), sort, write after the lower CTAs' winners
-  if (tid == 0) sh_ngt = 0;
-  __syncthreads();
-  for_each_score(row, len, [&](int i, float f) {
-    if ((order_key(f) & mask) > prefix) sel[atomicAdd(&sh_ngt, 1)] = lo + i;
-  });
-  {
-    int base = 0;   // ordered compaction of the slice's first my_eq_take ties
-    for (int c0 = 0; c0 < len && base < my_eq_take; c0 += TK_THREADS) {
-      const int i = c0 + tid;
-      const int eq = (i < len) && ((order_key(row[i]) & mask) == prefix);
-      int total;
-      const int r = block_excl_scan(eq, warp_buf, &total);
-      if (eq && base + r < my_eq_take) sel[my_gt + base + r] = lo + i;
-      base += total;
-    }
-  }
-  __syncthreads();
-  const int mine = my_gt + my_eq_take;
-  sort_ascending(sel, mine);
-  for (int i = tid; i < mine; i += TK_THREADS) write_expanded(out, out_off + i, sel[i], pool, pos);
 }
 
 }  // namespace
@@ -345,13 +268,15 @@ int launch_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, 
                 int pool, int t_begin, int t_count, int k, int32_t* idx, cudaStream_t stream) {
   if (B * t_count == 0) return DSA_OK;
   const int rows = B * t_count;
-  if (rows * TK_CL <= num_sms() && S_max / pool >= TK_CL * 4 * TK_THREADS) {
-    // few long rows (decode): a cluster per row, the whole grid in one wave
-    topk_rows_cluster_kernel<<<rows * TK_CL, TK_THREADS, 0, stream>>>(scores, ld, ctx_len, T, S_max, pool, t_begin,
-                                                                      t_count, k, idx);
-    return check_launch();
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TK_DYN_SMEM);
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  topk_rows_kernel<<<rows, TK_THREADS, 0, stream>>>(scores, ld, ctx_len, T, S_max, pool, t_begin, t_count, k, idx);
+  topk_rows_kernel<<<rows, TK_THREADS, TK_DYN_SMEM, stream>>>(scores, ld, ctx_len, T, S_max, pool, t_begin, t_count,
+                                                               k, idx);
   return check_launch();
 }
 

@@ -208,20 +208,24 @@ def test_mla_peaked_softmax(q_scale):
         assert msg is None, f"row {t}: {msg}"
 
 
-def test_topk_long_rows_exact_with_ties():
+@pytest.mark.parametrize("reps", [1, 8])
+def test_topk_long_rows_exact_with_ties(reps):
     """Long rows given as fp32 scores directly: the selected set must equal the oracle's
     exactly, with exact ties resolved to the lowest indices (an all-tied row, and a row of
     small integers with thousands of keys tied at the pivot), ids ascending and -1 padding; a
-    row with fewer visible keys than k selects them all.  Rows this long and this few are split
-    over a cluster of CTAs, so the tied winners also span the CTAs' slices."""
-    S, k, B, T = 20000, 2048, 5, 1
+    row with fewer visible keys than k selects them all.  The pivot bucket is copied to shared
+    memory when it fits (the every-7th and integer rows) and not for the all-tied row; five and
+    forty rows."""
+    S, k, T = 20000, 2048, 1
+    B = 5 * reps
     g = torch.Generator(device="cpu").manual_seed(3)
     sc = torch.randn(B, T, S, generator=g)
-    sc[0] = 0.0                                                       # all tied: ids 0..2047
-    sc[1, 0] = torch.randint(0, 50, (S,), generator=g).float()        # heavy ties at the pivot
-    sc[4] = 0.0
-    sc[4, 0, ::7] = 1.0                                               # the winners: every 7th id up to 14329
-    ctx = torch.tensor([S, S, 15000, 1500, S], dtype=torch.int32)
+    ctx = torch.tensor([S, S, 15000, 1500, S] * reps, dtype=torch.int32)
+    for r in range(reps):
+        sc[5 * r] = 0.0                                                     # all tied: ids 0..2047
+        sc[5 * r + 1, 0] = torch.randint(0, 50, (S,), generator=g).float()  # heavy ties at the pivot
+        sc[5 * r + 4] = 0.0
+        sc[5 * r + 4, 0, ::7] = 1.0                                         # winners: every 7th id up to 14329
     idx = dsa.dsa_topk(sc.to(DEV), ctx.to(DEV), T, S, k)
     for b in range(B):
         n_valid = min(S, int(ctx[b]))
