@@ -80,6 +80,24 @@ def test_e4m3_encode_matches_torch_in_range():
     assert np.array_equal(O.f32_to_e4m3(x), ref)
 
 
+def test_e4m3_encode_every_rounding_class():
+    """Every decision the encoder makes, enumerated: for each fp32 exponent from far below the
+    e4m3 subnormals to beyond saturation, every value of the 5 leading mantissa bits (what an
+    e4m3 normal keeps plus the round bit; more for subnormals, covered by the exponent sweep),
+    a zero, a 1-ulp and a full sticky tail, both signs.  Compared with torch's RNE cast."""
+    bits = []
+    for e in range(127 - 20, 127 + 10):          # 2^-20 .. 2^9
+        for head in range(32):
+            for tail in (0, 1, (1 << 18) - 1):
+                bits.append((e << 23) | (head << 18) | tail)
+    u = np.array(bits, dtype=np.uint32)
+    x = np.concatenate([u, u | np.uint32(0x80000000)]).view(np.float32)
+    x = x[np.abs(x) < 464.0]                     # beyond 464 both sides saturate (pinned below)
+    ref = torch.from_numpy(x.copy()).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert x.size > 5_000
+    assert np.array_equal(O.f32_to_e4m3(x), ref)
+
+
 def test_e4m3_encode_saturates():
     x = np.array([448.0, 455.9, 464.0, 479.0, 1e9, np.inf, -600.0, -np.inf], dtype=np.float32)
     assert list(O.f32_to_e4m3(x)) == [0x7E] * 6 + [0xFE] * 2

@@ -150,6 +150,17 @@ def test_indexpool_small():
     _check_rows(wl, ind, lays, idx, outs, [(0, t) for t in (0, 1, 2, 3, 100, 255, 256, 511)])
 
 
+def test_indexpool_every_code_bit_exact():
+    """Pooling of keys drawn uniformly over all 254 finite e4m3 codes (so sums cancel,
+    saturate and land on ties of every binade): the pooled codes equal the oracle's bit for
+    bit."""
+    g = torch.Generator(device="cpu").manual_seed(17)
+    codes = torch.randint(0, 254, (2, 1 << 17, 128), generator=g, dtype=torch.int32)
+    codes = torch.where(codes >= 0x7F, codes + 1, codes).to(torch.uint8)   # skip 0x7F (NaN); 0xFF is never drawn
+    kp = dsa.dsa_index_pool(codes.to(DEV))
+    assert np.array_equal(P.to_np(kp), O.index_pool(codes.numpy()))
+
+
 def test_mla_shapes_small_prefill():
     wl = W.WORKLOADS["prefill32k"].replace(T=2500, ctx=3000)
     ind, lays = _inputs(wl, layers=2)
