@@ -302,6 +302,10 @@ def roofline(wl, brk, pk, t_chunk):
                  "peak": pk["bf16_sus"], "unit": "TFLOP/s", "dtype": "bf16", "traffic": None,
                  "peak_src": f"{pk['src']} bf16 sustained"},
     }
+    # top-k: reads every visible score once and writes k ids per row (HBM-bound)
+    topk_bytes = 4 * causal_pairs(wl) + 4 * wl.B * wl.T * wl.topk * wl.pool
+    ent["topk"] = {"bound": "hbm", "achieved": topk_bytes / (brk["topk"] * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                   "unit": "GB/s", "traffic": None, "peak_src": f"{pk['src']} copy"}
     if wl.B * wl.T <= 64:   # decode: the attention reads every gathered row once; HBM-bound
         ent["attn"] = {"bound": "hbm", "achieved": attn_bytes(wl) / (brk["per_launch"]["attn_layer"] * 1e-3) / 1e9,
                        "peak": pk["hbm_gbs"], "unit": "GB/s", "traffic": None, "peak_src": f"{pk['src']} copy"}
@@ -312,7 +316,7 @@ def roofline(wl, brk, pk, t_chunk):
     for k, queries in (("attn", wl.B * wl.T), ("indexer", wl.B * min(t_chunk, wl.T))):
         per_q = TRAFFIC_PER_QUERY.get((wl.name, k))
         ent[k]["traffic"] = None if per_q is None else per_q * queries   # bytes per launch
-    top = max(("indexer", "attn"), key=lambda k: brk[k])
+    top = max(("indexer", "attn", "topk"), key=lambda k: brk[k])
     r = dict(ent[top])
     r["kernel"] = top
     r["frac"] = r["achieved"] / r["peak"]

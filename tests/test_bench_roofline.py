@@ -1,0 +1,56 @@
+"""bench.py's work counts and roofline arithmetic on CPU: the causal-pair and selected-key
+counts against their closed forms, and the roofline entries computed from a given per-kernel
+breakdown (no GPU involved)."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from indexed_sparse_attention_fp8_b200 import workloads as W  # noqa: E402
+
+PK = {"hbm_gbs": 6535.7, "bf16": 1672.2, "bf16_sus": 1382.4, "src": "measured"}
+
+
+def test_work_counts_closed_forms():
+    wl = W.WORKLOADS["prefill128k"]
+    L, k = wl.T, wl.topk
+    assert bench.causal_pairs(wl) == L * (L + 1) // 2                 # query t sees t + 1 keys
+    assert bench.selected_pairs(wl) == k * (k + 1) // 2 + (L - k) * k  # min(k, t + 1) summed
+    d = W.WORKLOADS["decode256k"]
+    assert bench.causal_pairs(d) == d.B * d.S                          # one query at the end of each cache
+    p = W.WORKLOADS["chunk1m_pool"]
+    first = p.ctx - p.T                                                # position of the first new query
+    assert bench.causal_pairs(p) == sum(pos // 4 + 1 for pos in range(first, p.ctx))
+
+
+def test_roofline_prefill_entries():
+    wl = W.WORKLOADS["prefill128k"]
+    brk = {"indexer": 89.3, "topk": 30.7, "attn": 451.4,
+           "per_launch": {"indexer_chunk": 11.16, "topk_chunk": 3.84, "attn_layer": 112.85}}
+    r = bench.roofline(wl, brk, PK, 16384)
+    assert r["kernel"] == "attn" and r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    flops = 128 * 2 * (576 + 512) * bench.selected_pairs(wl)
+    assert r["achieved"] == pytest.approx(flops / 112.85e-3 / 1e12)
+    assert r["peak"] == 1382.4 and r["frac"] == pytest.approx(r["achieved"] / 1382.4)
+    assert r["traffic"] == pytest.approx(bench.TRAFFIC_PER_QUERY[("prefill128k", "attn")] * wl.B * wl.T)
+    ix, tk = r["others"]["indexer"], r["others"]["topk"]
+    assert ix["achieved"] == pytest.approx(2 * 64 * 128 * bench.causal_pairs(wl) / 89.3e-3 / 1e12)
+    assert ix["peak"] == pytest.approx(2 * 1382.4)
+    assert ix["traffic"] == pytest.approx(bench.TRAFFIC_PER_QUERY[("prefill128k", "indexer")] * 16384)
+    assert tk["bound"] == "hbm"
+    assert tk["achieved"] == pytest.approx((4 * bench.causal_pairs(wl) + 4 * wl.T * 2048) / 30.7e-3 / 1e9)
+    assert tk["frac"] == pytest.approx(tk["achieved"] / 6535.7)
+
+
+def test_roofline_decode_is_hbm_bound():
+    wl = W.WORKLOADS["decode256k"]
+    brk = {"indexer": 0.186, "topk": 0.079, "attn": 0.218,
+           "per_launch": {"indexer_chunk": 0.186, "topk_chunk": 0.079, "attn_layer": 0.0545}}
+    r = bench.roofline(wl, brk, PK, 1)
+    assert r["kernel"] == "attn" and r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(bench.attn_bytes(wl) / 0.0545e-3 / 1e9)
+    assert r["traffic"] is None                        # no capture at this context
+    assert r["others"]["indexer"]["bound"] == "hbm"
