@@ -183,42 +183,42 @@ __device__ __forceinline__ void cluster_sync() {
 // registers would crowd the per-tile loop.
 __device__ __noinline__ void attn_load_q(const __nv_bfloat16* __restrict__ q, int bt, int row, int half, uint32_t tmem,
                                          uint32_t lane_off, uint32_t q_ready, int lane) {
-      // q[head, 288*half .. +287] -> TMEM lane `head`, bf16 pairs packed per 32-bit column
+  // q[head, 288*half .. +287] -> TMEM lane `head`, bf16 pairs packed per 32-bit column
   const uint4* qsrc = reinterpret_cast<const uint4*>(q + ((int64_t)bt * HQ + row) * DQK + 288 * half);
-      // two batches of loads (16 + 20 x 16 B; the rows were prefetched to L2 an item earlier)
-      {
-        uint4 qa[16];
+  // two batches of loads (16 + 20 x 16 B; the rows were prefetched to L2 an item earlier)
+  {
+    uint4 qa[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) qa[i] = __ldg(qsrc + i);
-        uint32_t w[32];
+    for (int i = 0; i < 16; ++i) qa[i] = __ldg(qsrc + i);
+    uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) { w[4 * i] = qa[i].x; w[4 * i + 1] = qa[i].y; w[4 * i + 2] = qa[i].z; w[4 * i + 3] = qa[i].w; }
-        tmem_st32u(tmem + lane_off + COL_Q, w);
+    for (int i = 0; i < 8; ++i) { w[4 * i] = qa[i].x; w[4 * i + 1] = qa[i].y; w[4 * i + 2] = qa[i].z; w[4 * i + 3] = qa[i].w; }
+    tmem_st32u(tmem + lane_off + COL_Q, w);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) { w[4 * i] = qa[8 + i].x; w[4 * i + 1] = qa[8 + i].y; w[4 * i + 2] = qa[8 + i].z; w[4 * i + 3] = qa[8 + i].w; }
-        tmem_st32u(tmem + lane_off + COL_Q + 32, w);
-      }
-      {
-        uint4 qb[20];
+    for (int i = 0; i < 8; ++i) { w[4 * i] = qa[8 + i].x; w[4 * i + 1] = qa[8 + i].y; w[4 * i + 2] = qa[8 + i].z; w[4 * i + 3] = qa[8 + i].w; }
+    tmem_st32u(tmem + lane_off + COL_Q + 32, w);
+  }
+  {
+    uint4 qb[20];
 #pragma unroll
-        for (int i = 0; i < 20; ++i) qb[i] = __ldg(qsrc + 16 + i);
-        uint32_t w[32];
+    for (int i = 0; i < 20; ++i) qb[i] = __ldg(qsrc + 16 + i);
+    uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) { w[4 * i] = qb[i].x; w[4 * i + 1] = qb[i].y; w[4 * i + 2] = qb[i].z; w[4 * i + 3] = qb[i].w; }
-        tmem_st32u(tmem + lane_off + COL_Q + 64, w);
+    for (int i = 0; i < 8; ++i) { w[4 * i] = qb[i].x; w[4 * i + 1] = qb[i].y; w[4 * i + 2] = qb[i].z; w[4 * i + 3] = qb[i].w; }
+    tmem_st32u(tmem + lane_off + COL_Q + 64, w);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) { w[4 * i] = qb[8 + i].x; w[4 * i + 1] = qb[8 + i].y; w[4 * i + 2] = qb[8 + i].z; w[4 * i + 3] = qb[8 + i].w; }
-        tmem_st32u(tmem + lane_off + COL_Q + 96, w);
-        uint32_t w16[16];
+    for (int i = 0; i < 8; ++i) { w[4 * i] = qb[8 + i].x; w[4 * i + 1] = qb[8 + i].y; w[4 * i + 2] = qb[8 + i].z; w[4 * i + 3] = qb[8 + i].w; }
+    tmem_st32u(tmem + lane_off + COL_Q + 96, w);
+    uint32_t w16[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) { w16[4 * i] = qb[16 + i].x; w16[4 * i + 1] = qb[16 + i].y; w16[4 * i + 2] = qb[16 + i].z; w16[4 * i + 3] = qb[16 + i].w; }
-        tmem_st16u(tmem + lane_off + COL_Q + 128, w16);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(q_ready);
-    }
+    for (int i = 0; i < 4; ++i) { w16[4 * i] = qb[16 + i].x; w16[4 * i + 1] = qb[16 + i].y; w16[4 * i + 2] = qb[16 + i].z; w16[4 * i + 3] = qb[16 + i].w; }
+    tmem_st16u(tmem + lane_off + COL_Q + 128, w16);
+  }
+  tmem_st_wait();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(q_ready);
+}
 
 // Epilogue of one item: waits for its last P.V, then O / l (or the split partial and its lse)
 // out of TMEM.  Out of line for the same reason as attn_load_q.
@@ -227,57 +227,57 @@ __device__ __noinline__ bool attn_epilogue(int bt, int sp, int ntiles, float m_f
                                            uint32_t pv_done, volatile int* abort, __nv_bfloat16* __restrict__ out,
                                            float* __restrict__ lse, float* __restrict__ part_o,
                                            float* __restrict__ part_lse) {
-      if (good && ntiles > 0) good = mbar_wait(pv_done, g_last & 1, abort, kWaitLimitNs);
-      good = __all_sync(0xffffffffu, good);   // the TMEM reads below are warp-collective
-      tc_fence_after();
-      const float inv = l_fin > 0.f ? 1.f / l_fin : 0.f;
-      const float lse_r = l_fin > 0.f ? (m_fin + log2f(l_fin)) * 0.69314718055994531f : -INFINITY;
-      const bool have_o = good && ntiles > 0;
-      const int64_t orow = (int64_t)bt * HQ + row;
-      if (part_o == nullptr) {
-        __nv_bfloat16* dst = out + orow * DV + half * DVH;
+  if (good && ntiles > 0) good = mbar_wait(pv_done, g_last & 1, abort, kWaitLimitNs);
+  good = __all_sync(0xffffffffu, good);   // the TMEM reads below are warp-collective
+  tc_fence_after();
+  const float inv = l_fin > 0.f ? 1.f / l_fin : 0.f;
+  const float lse_r = l_fin > 0.f ? (m_fin + log2f(l_fin)) * 0.69314718055994531f : -INFINITY;
+  const bool have_o = good && ntiles > 0;
+  const int64_t orow = (int64_t)bt * HQ + row;
+  if (part_o == nullptr) {
+    __nv_bfloat16* dst = out + orow * DV + half * DVH;
 #pragma unroll 1
-        for (int c = 0; c < DVH; c += 32) {
-          float o[32];
-          if (have_o) {
-            tmem_ld32(tmem + lane_off + COL_O + c, o);
-            tmem_ld_wait();
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = 0.f;
-          }
-#pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint4 v;
-            v.x = pack2_bf16(o[i] * inv, o[i + 1] * inv);
-            v.y = pack2_bf16(o[i + 2] * inv, o[i + 3] * inv);
-            v.z = pack2_bf16(o[i + 4] * inv, o[i + 5] * inv);
-            v.w = pack2_bf16(o[i + 6] * inv, o[i + 7] * inv);
-            *reinterpret_cast<uint4*>(dst + c + i) = v;
-          }
-        }
-        if (lse != nullptr && half == 0) lse[orow] = lse_r;
+    for (int c = 0; c < DVH; c += 32) {
+      float o[32];
+      if (have_o) {
+        tmem_ld32(tmem + lane_off + COL_O + c, o);
+        tmem_ld_wait();
       } else {
-        const int64_t rows = (int64_t)nbt * HQ;
-        float* dst = part_o + ((int64_t)sp * rows + orow) * DV + half * DVH;
-#pragma unroll 1
-        for (int c = 0; c < DVH; c += 32) {
-          float o[32];
-          if (have_o) {
-            tmem_ld32(tmem + lane_off + COL_O + c, o);
-            tmem_ld_wait();
-          } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = 0.f;
-          }
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(dst + c + i) = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
-        }
-        if (half == 0) part_lse[(int64_t)sp * rows + orow] = lse_r;
+        for (int i = 0; i < 32; ++i) o[i] = 0.f;
       }
-      return good;
+#pragma unroll
+      for (int i = 0; i < 32; i += 8) {
+        uint4 v;
+        v.x = pack2_bf16(o[i] * inv, o[i + 1] * inv);
+        v.y = pack2_bf16(o[i + 2] * inv, o[i + 3] * inv);
+        v.z = pack2_bf16(o[i + 4] * inv, o[i + 5] * inv);
+        v.w = pack2_bf16(o[i + 6] * inv, o[i + 7] * inv);
+        *reinterpret_cast<uint4*>(dst + c + i) = v;
+      }
     }
+    if (lse != nullptr && half == 0) lse[orow] = lse_r;
+  } else {
+    const int64_t rows = (int64_t)nbt * HQ;
+    float* dst = part_o + ((int64_t)sp * rows + orow) * DV + half * DVH;
+#pragma unroll 1
+    for (int c = 0; c < DVH; c += 32) {
+      float o[32];
+      if (have_o) {
+        tmem_ld32(tmem + lane_off + COL_O + c, o);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4*>(dst + c + i) = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+    }
+    if (half == 0) part_lse[(int64_t)sp * rows + orow] = lse_r;
+  }
+  return good;
+}
 
 struct Item {
   int bt, sp, b, kbeg, kend, ntiles;
