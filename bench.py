@@ -258,12 +258,13 @@ def breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, reps):
             marks.append(("pool", a, b))
         for t0 in range(0, wl.T, t_chunk):
             tc = min(t_chunk, wl.T - t0)
+            sc = scores.view(-1)[: wl.B * tc * ld].view(wl.B, tc, ld)   # [B, tc, ld], batch stride tc * ld
             a, b, c = ev(), ev(), ev()
             a.record(stream)
             dsa.dsa_index_scores(ind["q_idx"], ind["w"], keys, ind["ctx_len"], pool=wl.pool, t_begin=t0, t_count=tc,
-                                 scores=scores[:, :tc], stream=stream)
+                                 scores=sc, stream=stream)
             b.record(stream)
-            dsa.dsa_topk(scores[:, :tc], ind["ctx_len"], wl.T, S_eff, wl.topk, pool=wl.pool, t_begin=t0, idx=g.idx,
+            dsa.dsa_topk(sc, ind["ctx_len"], wl.T, S_eff, wl.topk, pool=wl.pool, t_begin=t0, idx=g.idx,
                          stream=stream)
             c.record(stream)
             marks += [("indexer", a, b), ("topk", b, c)]

@@ -129,7 +129,8 @@ int dsa_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, int
  *   q    [B, T, Hq, d_qk] bf16 (contiguous)
  *   kv   K rows: element (b, s, c) at kv[b*kv_batch_stride + s*kv_row_stride + c], c < d_qk
  *   v    V rows, same form with v_* strides; NULL means V = the first d_v columns of kv
- *   idx  [B, T, k] int32, entries in [0, ctx_len[b]) or < 0
+ *   idx  [B, T, k] int32, entries in [0, ctx_len[b]) or < 0 (entries are not range-checked on
+ *        the device: one at or beyond the end of the cache reads memory outside it)
  *   out  [B, T, Hq, d_v] bf16          lse  [B, T, Hq] fp32 or NULL
  *   ws   scratch of at least dsa_sparse_attn_workspace_size(B, T, Hq, d_v, k) bytes
  *        (zero for long prefill; split-key partials for few-query batches such as decode)

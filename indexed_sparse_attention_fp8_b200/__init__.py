@@ -99,6 +99,34 @@ def _ptr(t: Optional[torch.Tensor]):
     return t.data_ptr()
 
 
+def _layout(name: str, t: Optional[torch.Tensor], dtype: torch.dtype, shape: Sequence[int],
+            strides: Optional[Sequence[int]] = None) -> None:
+    """Checks that a tensor has the dtype, shape and element strides the C ABI assumes for it
+    (row-major contiguous unless `strides` is given; -1 in `shape` or `strides` matches any)."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.dim() != len(shape) or any(want not in (-1, got) for want, got in zip(shape, t.shape)):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if strides is None:
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: must be contiguous (strides {t.stride()})")
+    elif any(want not in (-1, got) for want, got in zip(strides, t.stride())):
+        raise ValueError(f"{name}: strides {t.stride()}, expected {tuple(strides)}")
+
+
+def _kv_layout(name: str, t: Optional[torch.Tensor], B: int, width: int) -> None:
+    """A K or V cache [B, S, >= width] bf16 with unit inner stride and row / batch strides that
+    are multiples of 8 elements (16 bytes)."""
+    if t is None:
+        return
+    _layout(name, t, torch.bfloat16, (B, -1, -1), (-1, -1, 1))
+    if t.shape[2] < width or t.stride(1) < width or t.stride(1) % 8 or t.stride(0) % 8:
+        raise ValueError(f"{name}: shape {tuple(t.shape)} strides {t.stride()} cannot hold {width}-wide rows "
+                         "at 16-byte aligned row and batch strides")
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -132,10 +160,15 @@ def dsa_index_scores(q_idx: torch.Tensor, w: torch.Tensor, k_idx: torch.Tensor, 
     S = k_idx.shape[1]
     tc = T - t_begin if t_count is None else t_count
     ld = (S + 3) // 4 * 4
+    _layout("q_idx", q_idx, torch.uint8, (B, T, H, D))
+    _layout("w", w, torch.float32, (B, T, H))
+    _layout("k_idx", k_idx, torch.uint8, (B, S, D))
+    _layout("ctx_len", ctx_len, torch.int32, (B,))
     if scores is None:
         scores = torch.empty((B, tc, ld), dtype=torch.float32, device=q_idx.device)
     else:
         ld = scores.stride(1)
+        _layout("scores", scores, torch.float32, (B, tc, -1), (tc * ld, ld, 1))
     _check("dsa_index_scores", _lib().dsa_index_scores(
         _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(ctx_len), B, T, S, H, D, pool, t_begin, tc, _ptr(scores), ld,
         _stream(stream)))
@@ -146,11 +179,24 @@ def dsa_topk(scores: torch.Tensor, ctx_len: torch.Tensor, T: int, S_max: int, k:
              t_begin: int = 0, idx: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Top-k token ids [B, T, k*pool] int32 (rows t_begin .. t_begin + scores.shape[1] written)."""
     B, tc, ld = scores.shape
+    _layout("scores", scores, torch.float32, (B, tc, -1), (tc * scores.stride(1), -1, 1))
+    _layout("ctx_len", ctx_len, torch.int32, (B,))
     if idx is None:
         idx = torch.full((B, T, k * pool), -1, dtype=torch.int32, device=scores.device)
+    _layout("idx", idx, torch.int32, (B, T, k * pool))
     _check("dsa_topk", _lib().dsa_topk(_ptr(scores), scores.stride(1), _ptr(ctx_len), B, T, S_max, pool, t_begin,
                                        tc, k, _ptr(idx), _stream(stream)))
     return idx
+
+
+def _attn_layouts(q, kv, v, idx, d_v, out, lse) -> None:
+    B, T, Hq, Dqk = q.shape
+    _layout("q", q, torch.bfloat16, (B, T, Hq, Dqk))
+    _kv_layout("kv", kv, B, Dqk)
+    _kv_layout("v", v, B, d_v)
+    _layout("idx", idx, torch.int32, (B, T, -1))
+    _layout("out", out, torch.bfloat16, (B, T, Hq, d_v))
+    _layout("lse", lse, torch.float32, (B, T, Hq))
 
 
 def dsa_sparse_attn_workspace_size(B: int, T: int, Hq: int, d_v: int, k: int) -> int:
@@ -165,6 +211,7 @@ def dsa_sparse_attn(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, sm_sca
     idx [B,T,k] int32.  Returns (out [B,T,Hq,d_v] bf16, lse [B,T,Hq] f32 or None)."""
     B, T, Hq, Dqk = q.shape
     k = idx.shape[-1]
+    _attn_layouts(q, kv, v, idx, d_v, out, lse)
     if out is None:
         out = torch.empty((B, T, Hq, d_v), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
@@ -189,6 +236,7 @@ def dsa_sparse_attn_noalloc(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor
     calls that may overlap on one GPU share that scratch and must be serialised."""
     B, T, Hq, Dqk = q.shape
     k = idx.shape[-1]
+    _attn_layouts(q, kv, v, idx, d_v, out, lse)
     if out is None:
         out = torch.empty((B, T, Hq, d_v), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
@@ -204,8 +252,10 @@ def dsa_sparse_attn_noalloc(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor
 def dsa_index_pool(k_idx: torch.Tensor, pool: int = 4, k_pool: Optional[torch.Tensor] = None, stream=None):
     """IndexPool: [B, S, d_I] e4m3 keys -> [B, S/4, d_I] pooled e4m3 keys."""
     B, S, D = k_idx.shape
+    _layout("k_idx", k_idx, torch.uint8, (B, S, D))
     if k_pool is None:
         k_pool = torch.empty((B, S // pool, D), dtype=torch.uint8, device=k_idx.device)
+    _layout("k_pool", k_pool, torch.uint8, (B, S // pool, D))
     _check("dsa_index_pool", _lib().dsa_index_pool(_ptr(k_idx), B, S, D, pool, _ptr(k_pool), _stream(stream)))
     return k_pool
 
@@ -221,6 +271,21 @@ class Group:
         self.layers = list(layers)
         q0, kv0 = layers[0]["q"], layers[0]["kv"]
         Hq, Dqk = q0.shape[2], q0.shape[3]
+        _layout("q_idx", q_idx, torch.uint8, (B, T, H, D))
+        _layout("w", w, torch.float32, (B, T, H))
+        _layout("k_idx", k_idx, torch.uint8, (B, S, D))
+        _layout("ctx_len", ctx_len, torch.int32, (B,))
+        _layout("idx", idx, torch.int32, (B, T, topk * pool))
+        v0 = layers[0].get("v")
+        for l, lay in enumerate(self.layers):
+            # one set of K/V strides describes every layer's caches
+            _attn_layouts(lay["q"], lay["kv"], lay.get("v"), torch.empty((B, T, 0), dtype=torch.int32), d_v,
+                          lay.get("out"), lay.get("lse"))
+            if lay["q"].shape != q0.shape or lay["kv"].stride() != kv0.stride():
+                raise ValueError(f"layer {l}: q shape or kv strides differ from layer 0's")
+            vl = lay.get("v")
+            if (vl is None) != (v0 is None) or (vl is not None and vl.stride() != v0.stride()):
+                raise ValueError(f"layer {l}: v presence or strides differ from layer 0's")
         for lay in self.layers:
             if lay.get("out") is None:
                 lay["out"] = torch.empty((B, T, Hq, d_v), dtype=torch.bfloat16, device=q0.device)
