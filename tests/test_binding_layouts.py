@@ -103,3 +103,27 @@ def test_group_layers_share_one_set_of_strides():
     with pytest.raises(ValueError, match="idx: shape"):
         dsa.Group(q_idx, w, k_idx, ctx, K, [{"q": q, "kv": kv, "v": v}], 0.1, DV, pool=4,
                   idx=torch.zeros(B, T, K, dtype=torch.int32))
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny", dict(T=64, ctx=128)),
+    ("prefill32k", dict(T=16, ctx=64)),
+    ("decode256k", dict(B=3, ctx=64)),
+    ("chunk1m_pool", dict(T=16, ctx=256)),
+])
+def test_workload_tensors_pass_the_layout_checks(name, over):
+    """The seeded workload tensors the tests and the bench hand to the binding (built here on
+    the CPU at reduced sizes) have the layouts it accepts: every call gets to the device check."""
+    from indexed_sparse_attention_fp8_b200 import workloads as W
+    wl = W.WORKLOADS[name].replace(**over)
+    ind = W.make_indexer_inputs(wl, device="cpu")
+    lays = [W.make_attn_inputs(wl, l, device="cpu") for l in range(2)]
+    args = [{"q": L["q"], "kv": L["kv"], "v": None if wl.kv_latent else L["v"]} for L in lays]
+    with pytest.raises(ValueError, match="CUDA device"):
+        dsa.Group(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk, args, wl.sm_scale, wl.d_v,
+                  pool=wl.pool)
+    with pytest.raises(ValueError, match="CUDA device"):
+        dsa.dsa_index_scores(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], t_begin=0, t_count=1)
+    idx = torch.zeros(wl.B, wl.T, wl.topk * wl.pool, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA device"):
+        dsa.dsa_sparse_attn(lays[0]["q"], lays[0]["kv"], idx, wl.sm_scale, wl.d_v, v=args[0]["v"], want_lse=True)
