@@ -92,6 +92,75 @@ def _expand_no_mask(block_ids, pos, pool):
     return out
 
 
+def _pool_max(k_idx, pool=4):
+    kf = OD._orig["e4m3_to_f64"](k_idx).astype(np.float32)
+    S = kf.shape[-2]; g = kf.reshape(kf.shape[:-2] + (S // 4, 4, kf.shape[-1]))
+    return OD._orig["f32_to_e4m3"](g.max(axis=-2))
+
+
+def _select_pool_last_block_dropped(q_idx_t, w_t, k_dec, pos, k, pool=1, k_pool_dec=None):
+    if pool == 1:
+        return OD._orig["select_row"](q_idx_t, w_t, k_dec, pos, k, pool, k_pool_dec)
+    sc = OD.index_scores_row(q_idx_t, w_t, k_pool_dec, pos, pool=pool)
+    blocks = OD.topk_row(sc, min(k_pool_dec.shape[0], pos // pool), k)        # off by one block
+    return OD.expand_blocks(blocks, pos, pool), sc
+
+
+def _attn_no_max_subtraction(q_t, K, V, idx_row, sm_scale):
+    sel = np.asarray([i for i in idx_row if i >= 0], dtype=np.int64)
+    if sel.size == 0:
+        return np.zeros((q_t.shape[0], V.shape[1])), np.full(q_t.shape[0], -np.inf)
+    with np.errstate(over="ignore", invalid="ignore"):
+        p = np.exp((q_t @ K[sel].T) * sm_scale)
+        d = p.sum(axis=1, keepdims=True)
+        return (p @ V[sel]) / d, np.log(d)[:, 0]
+
+
+def _group_first_layer_query(q_idx_t, w_t, k_dec, pos, k, layers, sm_scale, pool=1, k_pool_dec=None):
+    idx, _ = OD.select_row(q_idx_t, w_t, k_dec, pos, k, pool, k_pool_dec)
+    return idx, [OD.sparse_attn_row(layers[0]["q"], L["K"], L["V"], idx, sm_scale) for L in layers]
+
+
+def _per_layer_first_layer_indexer(indexer_inputs, pos, k, layers, sm_scale):
+    return OD._orig["per_layer_forward_row"]([indexer_inputs[0]] * len(layers), pos, k, layers, sm_scale)
+
+
+def _set_ok_no_missed_rule(gpu_idx, scores_ref, n_valid, k, pos, rel_band=1e-3, pool=1):
+    sel = np.asarray([i for i in gpu_idx if i >= 0], dtype=np.int64)
+    keff = min(k, n_valid)
+    if sel.size != keff or np.unique(sel).size != sel.size or (sel.size and sel.max() >= n_valid):
+        return False, "shape"
+    if keff == n_valid:
+        return True, "all"
+    s = np.asarray(scores_ref[:n_valid], dtype=np.float64)
+    tau = np.sort(s)[::-1][keff - 1]
+    return (not (s[sel] < tau - rel_band * abs(tau)).any()), "below only"
+
+
+def _set_ok_no_count_rule(gpu_idx, scores_ref, n_valid, k, pos, rel_band=1e-3, pool=1):
+    sel = np.asarray([i for i in gpu_idx if i >= 0], dtype=np.int64)
+    keff = min(k, n_valid)
+    if np.unique(sel).size != sel.size or (sel.size and sel.max() >= n_valid):
+        return False, "dup/range"
+    s = np.asarray(scores_ref[:n_valid], dtype=np.float64)
+    tau = np.sort(s)[::-1][keff - 1]
+    band = rel_band * abs(tau)
+    if not np.isin(np.nonzero(s > tau + band)[0], sel).all():
+        return False, "missed"
+    return (not (s[sel] < tau - band).any()), "no count"
+
+
+def _score_close_abs(gpu, ref, dense_mag, rel=1e-3, floor_rel=1e-5):
+    d = np.abs(np.asarray(gpu, np.float64) - np.asarray(ref, np.float64))
+    return d <= rel, 0
+
+
+def _magnitude_signed_w(q_t, w_t, k, pos, pool=1):
+    S = k.shape[0]; n = min(S, pos // pool + 1); out = np.zeros(S)
+    out[:n] = np.maximum(k[:n] @ q_t.T, 0.0) @ np.asarray(w_t, np.float64)
+    return out
+
+
 MUTANTS = [
     ("index_scores_row", _scores_no_relu, ["test_indexer_single_head_unit_weight_is_relu_dot", "test_indexer_hand_worked_example"]),
     ("index_scores_row", _scores_excl_self, ["test_indexer_causal_rule_includes_self", "test_indexer_brute_force_tiny"]),
@@ -105,13 +174,24 @@ MUTANTS = [
     ("e4m3_to_f64", _decode_bias8, ["test_e4m3_decode_all_codes_match_torch", "test_e4m3_decode_format_values"]),
     ("f32_to_e4m3", _encode_truncate, ["test_e4m3_encode_matches_torch_in_range"]),
     ("index_pool", _pool_half, ["test_pool_brute_force_and_library_requantisation"]),
-    ("expand_blocks", _expand_no_mask, ["test_pool_validity_and_expansion"]),
+    ("expand_blocks", _expand_no_mask, ["test_pool_validity_and_expansion",
+                                        "test_select_row_pool_last_block_visible_from_its_first_token"]),
+    ("index_pool", _pool_max, ["test_pool_mean_is_exact_then_one_rounding", "test_pool_brute_force_and_library_requantisation"]),
+    ("select_row", _select_pool_last_block_dropped, ["test_select_row_pool_last_block_visible_from_its_first_token"]),
+    ("sparse_attn_row", _attn_no_max_subtraction, ["test_attention_huge_logits_pick_the_argmax_key"]),
+    ("group_forward_row", _group_first_layer_query, ["test_indexshare_group_reuses_one_selection"]),
+    ("per_layer_forward_row", _per_layer_first_layer_indexer, ["test_per_layer_comparator_selects_with_each_layers_own_indexer"]),
+    ("topk_set_ok", _set_ok_no_missed_rule, ["test_topk_acceptance_rule"]),
+    ("topk_set_ok", _set_ok_no_count_rule, ["test_topk_acceptance_rule"]),
+    ("score_close", _score_close_abs, ["test_score_tolerance_rule_closed_form"]),
+    ("score_magnitude_row", _magnitude_signed_w, ["test_score_magnitude_closed_form"]),
 ]
 
 if not hasattr(OD, "_orig"):
     OD._orig = {n: getattr(OD, n) for n in
                 ["index_scores_row", "topk_row", "sparse_attn_row", "e4m3_to_f64", "f32_to_e4m3",
-                 "index_pool", "expand_blocks"]}
+                 "index_pool", "expand_blocks", "select_row", "group_forward_row", "per_layer_forward_row",
+                 "topk_set_ok", "score_close", "score_magnitude_row"]}
 
 
 @pytest.mark.parametrize("fn,mutant,pins", MUTANTS, ids=[m[1].__name__ for m in MUTANTS])

@@ -202,6 +202,32 @@ def test_topk_acceptance_rule():
     s2 = s.copy(); order = np.argsort(-s2); s2[order[50]] = s2[order[49]] * (1 - 1e-4 * np.sign(s2[order[49]]))
     idx2 = O.topk_row(s2, 500, 50); sw = idx2.copy(); sw[list(idx2).index(order[49])] = order[50]
     assert O.topk_set_ok(sw, s2, 500, 50, 499)[0]
+    # missing a key far above the k-th score is wrong even when its replacement sits inside
+    # the band (nothing selected lies below tau - band, so only the "missed" rule rejects it)
+    miss = idx2.copy(); miss[list(idx2).index(order[0])] = order[50]
+    assert not O.topk_set_ok(miss, s2, 500, 50, 499)[0]
+    assert not O.topk_set_ok(np.where(np.arange(50) == 49, -1, idx), s, 500, 50, 499)[0]   # one short
+    assert not O.topk_set_ok(np.r_[idx[:49], 500], s, 500, 50, 499)[0]                    # beyond n_valid
+    # fewer valid keys than k: every valid key, nothing else
+    assert O.topk_set_ok(np.r_[np.arange(7), [-1] * 3], s, 7, 10, 6)[0]
+    assert not O.topk_set_ok(np.r_[np.arange(6), [-1] * 4], s, 7, 10, 6)[0]
+
+
+def test_score_tolerance_rule_closed_form():
+    # relative rule: |gpu - ref| <= 1e-3 |ref|; floor rule: |gpu - ref| <= 1e-5 * D where D is
+    # the score's absolute magnitude sum_j |w_j| relu(q_j . k)
+    ref = np.array([1000.0, 1000.0, 1.0, 0.0, 0.0, -50.0])
+    gpu = np.array([1000.9, 1001.1, 1.01, 0.009, 0.011, -50.04])
+    mag = np.array([1000.0, 1000.0, 1.0, 1000.0, 1000.0, 60.0])
+    ok, nfloor = O.score_close(gpu, ref, mag, rel=1e-3, floor_rel=1e-5)
+    assert list(ok) == [True, False, False, True, False, True] and nfloor == 1
+
+
+def test_score_magnitude_closed_form():
+    # two heads, w = (1, -2): D = |1| relu(q0.k) + |-2| relu(q1.k)
+    q = np.array([[1.0, 0.0], [0.0, 1.0]]); w = np.array([1.0, -2.0], np.float32)
+    k = np.array([[3.0, 2.0], [-1.0, 5.0], [2.0, -4.0], [9.0, 9.0]])
+    assert list(O.score_magnitude_row(q, w, k, pos=2)) == [3 + 2 * 2, 0 + 2 * 5, 2 + 0, 0.0]
 
 
 # ---------------------------------------------------------------- IndexPool
@@ -223,6 +249,36 @@ def test_pool_brute_force_and_library_requantisation():
                 m = ((a + bb) + (c + e)) * 0.25                    # torch fp32 scalar ops
                 ref = m.reshape(1).to(torch.float8_e4m3fn).view(torch.uint8).item()
                 assert got[b, g, d] == ref
+
+
+def test_pool_mean_is_exact_then_one_rounding():
+    """Four e4m3 values are integer multiples of 2^-9 below 2^11 in magnitude, so their fp32
+    sum and its quarter are exact: the pooled code is the exact rational mean rounded once by
+    torch's e4m3 cast, whatever order the four keys come in."""
+    from fractions import Fraction
+    k = rand_codes((32, 24), scale=40.0)                       # wide range: subnormals to 448
+    got = O.index_pool(k)
+    kv = torch_e4m3(k)
+    for g in range(8):
+        for d in range(24):
+            mean = sum(Fraction(float(kv[4 * g + r, d])) for r in range(4)) / 4
+            ref = torch.tensor([float(mean)], dtype=torch.float64).to(torch.float32).to(torch.float8_e4m3fn)
+            assert float(mean) == float(np.float32(float(mean)))     # exact in fp32
+            assert got[g, d] == ref.view(torch.uint8).item()
+    perm = k.reshape(8, 4, 24)[:, [2, 0, 3, 1]].reshape(32, 24)
+    assert np.array_equal(O.index_pool(perm), got)
+
+
+def test_select_row_pool_last_block_visible_from_its_first_token():
+    # block b is a candidate from position 4b on (its first token visible), never before; the
+    # expanded ids keep only tokens <= pos
+    D = 16
+    q = np.zeros((1, D)); q[0, 0] = 1.0; w = np.ones(1, np.float32)
+    kp = np.zeros((6, D)); kp[:, 0] = [1.0, 2.0, 3.0, 100.0, 0.5, 0.25]     # block 3 scores highest
+    for pos, want in [(12, [12, -1, -1, -1]), (13, [12, 13, -1, -1]), (15, [12, 13, 14, 15]), (11, [8, 9, 10, 11])]:
+        idx, sc = O.select_row(q, w, None, pos, 2, pool=4, k_pool_dec=kp)
+        assert list(idx[:4]) == want, (pos, list(idx))
+        assert np.isneginf(sc[pos // 4 + 1:]).all()
 
 
 def test_pool_validity_and_expansion():
@@ -273,6 +329,17 @@ def test_attention_zero_query_is_mean_of_v_and_duplicates_count():
     np.testing.assert_allclose(o, np.repeat(((V[3] + 2 * V[5] + V[11]) / 4)[None], 4, axis=0), rtol=1e-14)
 
 
+def test_attention_huge_logits_pick_the_argmax_key():
+    # logit gaps of ~1000 (exp(-1000) is 0 in float64): the output is exactly V of the
+    # best key and lse is exactly the best logit
+    K = np.zeros((5, 4)); K[:, 0] = [1.0, 3.0, -2.0, 2.0, 0.0]
+    V = rng.standard_normal((5, 3))
+    q = np.array([[1000.0, 0, 0, 0], [-1000.0, 0, 0, 0]])
+    o, lse = O.sparse_attn_row(q, K, V, np.array([0, 1, 2, 3, 4]), 1.0)
+    assert np.array_equal(o[0], V[1]) and np.array_equal(o[1], V[2])
+    assert list(lse) == [3000.0, 2000.0]
+
+
 def test_attention_brute_force_and_permutation():
     q, K, V = _attn_inputs(3, 6, 4, 15, latent=True)
     idx = rng.permutation(15)[:9]
@@ -304,3 +371,21 @@ def test_indexshare_group_reuses_one_selection():
     # the comparator with the same indexer inputs at every layer selects the same keys
     per = O.per_layer_forward_row([(qi, w, kd)] * 4, 33, k, layers, 0.25)
     assert all(np.array_equal(p[0], idx) for p in per)
+
+
+def test_per_layer_comparator_selects_with_each_layers_own_indexer():
+    # layer l's keys are built so that key 5l+3 dominates its own indexer: each layer's
+    # selection must contain its own planted key, and the layers' selections differ
+    S, H, D, Hq, Dq, Dv, k = 30, 1, 4, 2, 6, 3, 3
+    q = np.zeros((H, D)); q[0, 0] = 1.0; w = np.ones(H, np.float32)
+    ins = []
+    for l in range(4):
+        kd = np.zeros((S, D)); kd[:, 0] = rng.uniform(-1, 1, S); kd[5 * l + 3, 0] = 50.0
+        ins.append((q, w, kd))
+    layers = [dict(zip("qKV", _attn_inputs(Hq, Dq, Dv, S, latent=False))) for _ in range(4)]
+    per = O.per_layer_forward_row(ins, 29, k, layers, 0.5)
+    for l, (idx, (o, lse)) in enumerate(per):
+        assert 5 * l + 3 in set(idx.tolist())
+        o2, l2 = O.sparse_attn_row(layers[l]["q"], layers[l]["K"], layers[l]["V"], idx, 0.5)
+        assert np.array_equal(o, o2) and np.array_equal(lse, l2)
+    assert len({tuple(p[0].tolist()) for p in per}) == 4
