@@ -285,11 +285,13 @@ def breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, reps):
     return out
 
 
-# DRAM bytes (read + write) per query, from one ncu capture of the current kernels with the
-# bench's 131072-row context and 2048 queries (dram__bytes_read.sum + dram__bytes_write.sum per
-# launch / queries).  Per-query traffic does not depend on the number of queries, so a launch's
-# traffic is this figure times its queries.  Other contexts: not measured (None).
-TRAFFIC_PER_QUERY = {("prefill128k", "attn"): 587.6e3, ("prefill128k", "indexer"): 510.5e3}
+# DRAM bytes (read + write) per query, from one ncu capture with the bench's 131072-row context
+# and 2048 queries (dram__bytes_read.sum + dram__bytes_write.sum per launch / queries).
+# Per-query traffic does not depend on the number of queries, so a launch's traffic is this
+# figure times its queries.  Only kernels unchanged since that capture are listed: the indexer
+# and the top-k have changed since (their traffic is reported as None until re-captured), and
+# other contexts were not measured.
+TRAFFIC_PER_QUERY = {("prefill128k", "attn"): 587.6e3}
 
 
 def roofline(wl, brk, pk, t_chunk):

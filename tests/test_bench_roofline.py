@@ -39,7 +39,7 @@ def test_roofline_prefill_entries():
     ix, tk = r["others"]["indexer"], r["others"]["topk"]
     assert ix["achieved"] == pytest.approx(2 * 64 * 128 * bench.causal_pairs(wl) / 89.3e-3 / 1e12)
     assert ix["peak"] == pytest.approx(2 * 1382.4)
-    assert ix["traffic"] == pytest.approx(bench.TRAFFIC_PER_QUERY[("prefill128k", "indexer")] * 16384)
+    assert ix["traffic"] is None   # the indexer changed after the traffic capture
     assert tk["bound"] == "hbm"
     assert tk["achieved"] == pytest.approx((4 * bench.causal_pairs(wl) + 4 * wl.T * 2048) / 30.7e-3 / 1e9)
     assert tk["frac"] == pytest.approx(tk["achieved"] / 6535.7)
