@@ -203,7 +203,8 @@ typedef struct dsa_group_args {
   const uint16_t* const* v;   /* NULL, or per-layer V (NULL entries alias kv) */
   uint16_t* const* out;       /* [B, T, Hq, d_v] bf16 */
   float* const* lse;          /* NULL, or per-layer [B, T, Hq] fp32 (NULL entries skip) */
-  int64_t kv_row_stride, kv_batch_stride, v_row_stride, v_batch_stride;
+  int64_t kv_row_stride, kv_batch_stride, v_row_stride, v_batch_stride;   /* elements; the same
+                                                                             for every layer */
   int32_t Hq, d_qk, d_v;
   float sm_scale;
   int32_t* idx;            /* [B, T, topk*pool] int32 out: the shared selection */
