@@ -92,6 +92,19 @@ def _expand_no_mask(block_ids, pos, pool):
     return out
 
 
+def _encode_ties_away(x):
+    # round half away from zero instead of half to even: move every exact tie to the code
+    # above it in magnitude
+    x = np.asarray(x, np.float32)
+    codes = OD._orig["f32_to_e4m3"](x)
+    v = OD._orig["e4m3_to_f64"](codes)
+    a = np.abs(x.astype(np.float64))
+    up = (codes & 0x7F) + 1
+    nxt = OD._orig["e4m3_to_f64"](np.minimum(up, 0x7E).astype(np.uint8))
+    tie_down = (np.abs(v) < a) & np.isclose(a - np.abs(v), nxt - a, rtol=0, atol=0) & ((codes & 0x7F) < 0x7E)
+    return np.where(tie_down, (codes & 0x80) | up, codes).astype(np.uint8)
+
+
 def _pool_max(k_idx, pool=4):
     kf = OD._orig["e4m3_to_f64"](k_idx).astype(np.float32)
     S = kf.shape[-2]; g = kf.reshape(kf.shape[:-2] + (S // 4, 4, kf.shape[-1]))
@@ -176,7 +189,10 @@ MUTANTS = [
     ("index_pool", _pool_half, ["test_pool_brute_force_and_library_requantisation"]),
     ("expand_blocks", _expand_no_mask, ["test_pool_validity_and_expansion",
                                         "test_select_row_pool_last_block_visible_from_its_first_token"]),
-    ("index_pool", _pool_max, ["test_pool_mean_is_exact_then_one_rounding", "test_pool_brute_force_and_library_requantisation"]),
+    ("index_pool", _pool_max, ["test_pool_mean_is_exact_then_one_rounding", "test_pool_brute_force_and_library_requantisation",
+                               "test_pool_hand_worked_example"]),
+    ("index_pool", _pool_half, ["test_pool_hand_worked_example"]),
+    ("f32_to_e4m3", _encode_ties_away, ["test_e4m3_encode_matches_torch_in_range", "test_pool_hand_worked_example"]),
     ("select_row", _select_pool_last_block_dropped, ["test_select_row_pool_last_block_visible_from_its_first_token"]),
     ("sparse_attn_row", _attn_no_max_subtraction, ["test_attention_huge_logits_pick_the_argmax_key"]),
     ("group_forward_row", _group_first_layer_query, ["test_indexshare_group_reuses_one_selection"]),

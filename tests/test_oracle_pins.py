@@ -251,6 +251,12 @@ def test_pool_brute_force_and_library_requantisation():
                 assert got[b, g, d] == ref
 
 
+def test_pool_hand_worked_example():
+    g = json.load(open(os.path.join(GOLDEN, "indexpool_hand.json")))
+    k = np.array(g["groups_codes"], dtype=np.uint8).reshape(-1, 1)     # [4 * groups, d = 1]
+    assert list(O.index_pool(k)[:, 0]) == g["expected_codes"]
+
+
 def test_pool_mean_is_exact_then_one_rounding():
     """Four e4m3 values are integer multiples of 2^-9 below 2^11 in magnitude, so their fp32
     sum and its quarter are exact: the pooled code is the exact rational mean rounded once by
