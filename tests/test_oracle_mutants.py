@@ -64,6 +64,11 @@ def _attn_drop_last(q_t, K, V, idx_row, sm_scale):
     return OD._orig["sparse_attn_row"](q_t, K, V, np.array(r[:-1] if len(r) > 1 else r), sm_scale)
 
 
+def _attn_dedup(q_t, K, V, idx_row, sm_scale):
+    r = np.unique(np.asarray([i for i in idx_row if i >= 0], dtype=np.int64))
+    return OD._orig["sparse_attn_row"](q_t, K, V, r if r.size else np.array([-1]), sm_scale)
+
+
 def _decode_bias8(codes):
     v = OD._orig["e4m3_to_f64"](codes)
     c = np.asarray(codes, np.uint8)
@@ -195,6 +200,11 @@ MUTANTS = [
     ("f32_to_e4m3", _encode_ties_away, ["test_e4m3_encode_matches_torch_in_range", "test_pool_hand_worked_example"]),
     ("select_row", _select_pool_last_block_dropped, ["test_select_row_pool_last_block_visible_from_its_first_token"]),
     ("sparse_attn_row", _attn_no_max_subtraction, ["test_attention_huge_logits_pick_the_argmax_key"]),
+    ("sparse_attn_row", _attn_no_scale, ["test_attention_hand_worked_example"]),
+    ("sparse_attn_row", _attn_drop_last, ["test_attention_hand_worked_example"]),
+    ("sparse_attn_row", _attn_k_as_v, ["test_attention_hand_worked_example"]),
+    ("sparse_attn_row", _attn_dedup, ["test_attention_hand_worked_example",
+                                      "test_attention_zero_query_is_mean_of_v_and_duplicates_count"]),
     ("group_forward_row", _group_first_layer_query, ["test_indexshare_group_reuses_one_selection"]),
     ("per_layer_forward_row", _per_layer_first_layer_indexer, ["test_per_layer_comparator_selects_with_each_layers_own_indexer"]),
     ("topk_set_ok", _set_ok_no_missed_rule, ["test_topk_acceptance_rule"]),

@@ -335,6 +335,21 @@ def test_attention_zero_query_is_mean_of_v_and_duplicates_count():
     np.testing.assert_allclose(o, np.repeat(((V[3] + 2 * V[5] + V[11]) / 4)[None], 4, axis=0), rtol=1e-14)
 
 
+def test_attention_hand_worked_example():
+    from fractions import Fraction
+    g = json.load(open(os.path.join(GOLDEN, "attention_hand.json")))
+    K, V, q = (np.array(g[n], dtype=np.float64) for n in ("K", "V", "q"))
+    for r, idx in enumerate(g["idx"]):
+        o, lse = O.sparse_attn_row(q, K, V, np.array(idx), math.log(2.0))
+        exp_o = np.array([[float(Fraction(x)) for x in h] for h in g["expected_O"][r]])
+        np.testing.assert_allclose(o, exp_o, rtol=1e-13, atol=1e-13)
+        for h, z in enumerate(g["expected_lse_of"][r]):
+            if z == 0:
+                assert lse[h] == -np.inf
+            else:
+                assert abs(lse[h] - math.log(z)) < 1e-13
+
+
 def test_attention_huge_logits_pick_the_argmax_key():
     # logit gaps of ~1000 (exp(-1000) is 0 in float64): the output is exactly V of the
     # best key and lse is exactly the best logit
