@@ -33,7 +33,9 @@ notes of the repository):
     index list count twice; -1 entries are skipped;
   * IndexPool: pooled key b = e4m3(((k[4b]+k[4b+1]) + (k[4b+2]+k[4b+3])) * 0.25) computed
     in fp32 from the decoded keys; block b is valid for query position p iff 4b <= p; the
-    top blocks expand to tokens 4b..4b+3, tokens beyond p become -1.
+    top blocks expand to tokens 4b..4b+3, tokens beyond p become -1.  The same mean over
+    P = 2 or 8 keys (a balanced pairwise fp32 sum times 1/P; validity P*b <= p, expansion to
+    P tokens) generalises the pages' factor of four.
 
 Parity status: every function here is pinned by tests that do not re-type its formula
 (library routines, closed forms, brute force on tiny inputs, invariants).
@@ -192,18 +194,22 @@ def expand_blocks(block_ids: np.ndarray, pos: int, pool: int) -> np.ndarray:
 
 
 def index_pool(k_idx: np.ndarray, pool: int = 4) -> np.ndarray:
-    """Pool groups of 4 consecutive indexer keys (e4m3 codes [..., S, d]) into one:
-    decode to fp32, ((k0 + k1) + (k2 + k3)) * 0.25 in fp32, requantise to e4m3 (RNE,
-    saturating).  Groups start at key 0; S must be a multiple of 4."""
-    if pool != 4:
-        raise ValueError("IndexPool pools 4 keys into one")
+    """Pool groups of `pool` consecutive indexer keys (e4m3 codes [..., S, d]) into one:
+    decode to fp32, sum the group as a balanced pairwise tree in fp32 (for the pages' four:
+    ((k0 + k1) + (k2 + k3))), multiply by 1/pool, requantise to e4m3 (RNE, saturating).
+    pool is 4 (the pages' factor) or 2 or 8.  Groups start at key 0; S must be a multiple of
+    pool."""
+    if pool not in (2, 4, 8):
+        raise ValueError("IndexPool pools 2, 4 or 8 keys into one")
     kf = e4m3_to_f64(k_idx).astype(np.float32)            # exact: e4m3 values fit fp32
     S = kf.shape[-2]
     if S % pool:
         raise ValueError("key count must be a multiple of the pool factor")
     g = kf.reshape(kf.shape[:-2] + (S // pool, pool, kf.shape[-1]))
-    a, b, c, d = g[..., 0, :], g[..., 1, :], g[..., 2, :], g[..., 3, :]
-    m = ((a + b) + (c + d)) * np.float32(0.25)            # every op in fp32
+    parts = [g[..., r, :] for r in range(pool)]
+    while len(parts) > 1:                                 # pairwise: (k0+k1), (k2+k3), ...
+        parts = [parts[2 * i] + parts[2 * i + 1] for i in range(len(parts) // 2)]
+    m = parts[0] * np.float32(1.0 / pool)                 # every op in fp32
     return f32_to_e4m3(m)
 
 
@@ -242,8 +248,8 @@ def sparse_attn_row(q_t: np.ndarray, K: np.ndarray, V: np.ndarray, idx_row: np.n
 def select_row(q_idx_t, w_t, k_dec, pos: int, k: int, pool: int = 1, k_pool_dec=None):
     """Indexer + top-k for one query row: returns (idx [k_tokens] int32, scores f32).
 
-    pool == 1: scores over keys, top-k keys.  pool == 4 (IndexPool): scores over pooled
-    keys (k_pool_dec, decoded pooled e4m3), top-k blocks, expanded to 4k tokens."""
+    pool == 1: scores over keys, top-k keys.  pool > 1 (IndexPool): scores over pooled
+    keys (k_pool_dec, decoded pooled e4m3), top-k blocks, expanded to pool*k tokens."""
     if pool == 1:
         sc = index_scores_row(q_idx_t, w_t, k_dec, pos)
         n_valid = min(k_dec.shape[0], pos + 1)

@@ -89,6 +89,21 @@ def _pool_half(k_idx, pool=4):
     return OD._orig["f32_to_e4m3"]((g[..., 0, :] + g[..., 1, :]) * np.float32(0.5))
 
 
+def _pool_fixed_quarter(k_idx, pool=4):
+    # the factor-4 scale kept for every factor: the mean of 2 or 8 keys comes out x2 or x0.5
+    kf = OD._orig["e4m3_to_f64"](k_idx).astype(np.float32)
+    S = kf.shape[-2]; g = kf.reshape(kf.shape[:-2] + (S // pool, pool, kf.shape[-1]))
+    return OD._orig["f32_to_e4m3"](g.sum(axis=-2, dtype=np.float32) * np.float32(0.25))
+
+
+def _pool_first_four_only(k_idx, pool=4):
+    # a group of 8 pooled as if it held only its first 4 keys
+    kf = OD._orig["e4m3_to_f64"](k_idx).astype(np.float32)
+    S = kf.shape[-2]; g = kf.reshape(kf.shape[:-2] + (S // pool, pool, kf.shape[-1]))
+    n = min(pool, 4)
+    return OD._orig["f32_to_e4m3"](g[..., :n, :].sum(axis=-2, dtype=np.float32) * np.float32(1.0 / n))
+
+
 def _expand_no_mask(block_ids, pos, pool):
     out = np.full(block_ids.shape[0] * pool, -1, np.int32)
     for i, b in enumerate(block_ids):
@@ -211,6 +226,11 @@ MUTANTS = [
     ("topk_set_ok", _set_ok_no_count_rule, ["test_topk_acceptance_rule"]),
     ("score_close", _score_close_abs, ["test_score_tolerance_rule_closed_form"]),
     ("score_magnitude_row", _magnitude_signed_w, ["test_score_magnitude_closed_form"]),
+    ("index_pool", _pool_fixed_quarter, [("test_pool_factors_2_and_8_identity_brute_force_and_exact_mean", 2),
+                                         ("test_pool_factors_2_and_8_identity_brute_force_and_exact_mean", 8)]),
+    ("index_pool", _pool_first_four_only, [("test_pool_factors_2_and_8_identity_brute_force_and_exact_mean", 8)]),
+    ("expand_blocks", _expand_no_mask, [("test_pool_factor_validity_and_expansion", 2),
+                                        ("test_pool_factor_validity_and_expansion", 8)]),
 ]
 
 if not hasattr(OD, "_orig"):
@@ -225,5 +245,6 @@ def test_pins_catch_planted_mistake(monkeypatch, fn, mutant, pins):
     monkeypatch.setattr(OD, fn, mutant)
     monkeypatch.setattr(O, fn, mutant)
     for pin in pins:
+        name, args = (pin[0], pin[1:]) if isinstance(pin, tuple) else (pin, ())
         with pytest.raises(AssertionError):
-            getattr(P, pin)()
+            getattr(P, name)(*args)

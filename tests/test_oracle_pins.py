@@ -275,6 +275,55 @@ def test_pool_mean_is_exact_then_one_rounding():
     assert np.array_equal(O.index_pool(perm), got)
 
 
+@pytest.mark.parametrize("P", [2, 8])
+def test_pool_factors_2_and_8_identity_brute_force_and_exact_mean(P):
+    """Pool factors 2 and 8 (the pages' factor is 4): identical keys pool to themselves; each
+    pooled code equals torch fp32 scalar arithmetic (pairwise sum, times 1/P) cast by torch to
+    e4m3; and, since P e4m3 values (integer multiples of 2^-9 below 2^9 in magnitude) sum
+    exactly in fp32 for P <= 8, the code is the exact rational mean rounded once, whatever
+    order the keys come in."""
+    from fractions import Fraction
+    k = rand_codes((5, 32))
+    assert np.array_equal(O.index_pool(np.repeat(k, P, axis=0), pool=P), k)
+    k = rand_codes((P * 6, 12), scale=40.0)
+    got = O.index_pool(k, pool=P)
+    assert got.shape == (6, 12)
+    kt = torch.from_numpy(k).view(torch.float8_e4m3fn).to(torch.float32)
+    for g in range(6):
+        for d in range(12):
+            vals = [kt[P * g + r, d] for r in range(P)]
+            while len(vals) > 1:
+                vals = [vals[2 * i] + vals[2 * i + 1] for i in range(len(vals) // 2)]
+            ref = (vals[0] * (1.0 / P)).reshape(1).to(torch.float8_e4m3fn).view(torch.uint8).item()
+            assert got[g, d] == ref
+            mean = sum(Fraction(float(kt[P * g + r, d])) for r in range(P)) / P
+            assert float(mean) == float(np.float32(float(mean)))          # exact in fp32
+            ex = torch.tensor([float(mean)], dtype=torch.float64).to(torch.float32).to(torch.float8_e4m3fn)
+            assert got[g, d] == ex.view(torch.uint8).item()
+    rng = np.random.default_rng(P)
+    perm = np.stack([rng.permutation(P) for _ in range(6)])
+    shuffled = np.concatenate([k[P * g + perm[g]] for g in range(6)])
+    assert np.array_equal(O.index_pool(shuffled, pool=P), got)
+    with pytest.raises(ValueError):
+        O.index_pool(rand_codes((12, 4)), pool=3)
+
+
+@pytest.mark.parametrize("P", [2, 8])
+def test_pool_factor_validity_and_expansion(P):
+    # block b is a candidate iff P*b <= pos; it expands to tokens P*b .. P*b+P-1, those beyond
+    # pos becoming -1
+    D = 16
+    q = np.zeros((1, D)); q[0, 0] = 1.0; w = np.ones(1, np.float32)
+    kp = np.zeros((6, D)); kp[:, 0] = [1.0, 2.0, 3.0, 100.0, 0.5, 0.25]     # block 3 scores highest
+    pos = 3 * P                                                              # block 3's first token
+    idx, sc = O.select_row(q, w, None, pos, 2, pool=P, k_pool_dec=kp)
+    assert list(idx[:P]) == [3 * P] + [-1] * (P - 1)
+    assert list(idx[P:2 * P]) == list(range(2 * P, 3 * P))                   # runner-up block 2, whole
+    assert np.isneginf(sc[4:]).all() and np.isfinite(sc[:4]).all()
+    idx, _ = O.select_row(q, w, None, pos - 1, 2, pool=P, k_pool_dec=kp)     # block 3 not yet visible
+    assert list(idx[:P]) == list(range(2 * P, 3 * P))
+
+
 def test_select_row_pool_last_block_visible_from_its_first_token():
     # block b is a candidate from position 4b on (its first token visible), never before; the
     # expanded ids keep only tokens <= pos
