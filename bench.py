@@ -9,9 +9,11 @@ layers, all inside one dsa_group_forward call (the C ABI).  Inputs are synthetic
 repeats the step from pinned host buffers with the host<->device copies inside the timed
 region.  Inputs are larger than L2, so no flush is needed between steps.
 
-Multi-GPU (torchrun, one process per GPU): every rank runs its own replica of the workload
-(the path shards by sequence / query block with no exchange), value = all ranks' queries /
-max-over-ranks time, scaling "weak".
+Multi-GPU (torchrun, one process per GPU, --gpus N must equal the world size): the one
+workload is sharded with no exchange step -- prefill query rows in zig-zag contiguous chunks,
+decode sequences in batch slices (indexed_sparse_attention_fp8_b200.shard) -- with the key
+caches replicated; value = the workload's queries / max-over-ranks time, scaling "strong"
+(the total work is fixed).
 
 The JSON line also carries: the decode line (32 x 256K), the per-layer-indexer comparator
 at 128K with the IndexShare speedup, chunked prefill at a 1M-token cache without and with
@@ -36,6 +38,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from indexed_sparse_attention_fp8_b200 import shard  # noqa: E402
 from indexed_sparse_attention_fp8_b200 import workloads as W  # noqa: E402
 
 METRIC = "query tok/s per 4-layer IndexShare group (prefill 128K, decode 256K); % roofline"
@@ -162,6 +165,57 @@ def make_group(wl, dev, dsa, layers=None, indexer_layer=0, share_q=False):
     return ind, lays
 
 
+def rank_boxes(wl, world, rank):
+    """This rank's (b0, b1, t0, t1) boxes of the workload: all of it on one GPU, else its
+    share of the sharding plan (zig-zag query-row chunks for prefill, batch slices for decode)."""
+    return [(0, wl.B, 0, wl.T)] if world == 1 else shard.plan(wl, world, rank)
+
+
+def box_workload(wl, box):
+    """The workload restricted to one box: its rows keep their positions (ctx moves to the
+    chunk's end), so the work counts below apply to it unchanged."""
+    b0, b1, t0, t1 = box
+    return wl.replace(B=b1 - b0, T=t1 - t0, ctx=wl.ctx - (wl.T - t1))
+
+
+class Part:
+    """One box of the rank's share: its sub-workload, its input tensors and its group call."""
+
+    def __init__(self, wl, box, ind, lays, dsa):
+        self.wl, self.box, self.ind, self.lays = box_workload(wl, box), box, ind, lays
+        self.g = dsa.Group(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk, lays, wl.sm_scale,
+                           wl.d_v, pool=wl.pool)
+
+
+def make_parts(wl, dev, dsa, boxes):
+    """Inputs of every box of this rank.  The whole workload keeps its tensors as made; a
+    shard copies its query rows out of the full (identically seeded) tensors, one layer at a
+    time, and views the replicated key caches."""
+    whole = boxes == [(0, wl.B, 0, wl.T)]
+    ind_full = W.make_indexer_inputs(wl, device=dev)
+
+    def rows(x, box):
+        b0, b1, t0, t1 = box
+        return x if whole else x[b0:b1, t0:t1].contiguous()
+
+    inds = [{"q_idx": rows(ind_full["q_idx"], bx), "w": rows(ind_full["w"], bx),
+             "k_idx": ind_full["k_idx"][bx[0]:bx[1]],
+             "ctx_len": ind_full["ctx_len"][bx[0]:bx[1]] - (wl.T - bx[3])} for bx in boxes]
+    lays = [[] for _ in boxes]
+    for l in range(wl.group):
+        a = W.make_attn_inputs(wl, l, device=dev)
+        for i, bx in enumerate(boxes):
+            lays[i].append({"q": rows(a["q"], bx), "kv": a["kv"][bx[0]:bx[1]],
+                            "v": None if a["v"] is None else a["v"][bx[0]:bx[1]]})
+        del a
+    del ind_full
+    return [Part(wl, bx, ind, lay, dsa) for bx, ind, lay in zip(boxes, inds, lays)]
+
+
+def score_t_chunk(args, wl):
+    return args.t_chunk or max(1, min(wl.T, (args.score_ws_gb << 30) // (wl.B * ((wl.S // wl.pool + 3) // 4 * 4) * 4)))
+
+
 def max_over_ranks(x: float, world: int, device) -> float:
     """The slowest rank's value (every rank takes part; world 1 returns x)."""
     if world == 1:
@@ -171,9 +225,17 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def sum_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
 def job_throughput(units_per_rank_step: int, world: int, ms_per_step: float) -> float:
-    """Whole-job units/s: every rank processes its own units each step (weak scaling), and the
-    step takes as long as the slowest rank."""
+    """Whole-job units/s when every rank processes its own units each step (replicas, weak
+    scaling) and the step takes as long as the slowest rank."""
     return units_per_rank_step * world / (ms_per_step / 1e3)
 
 
@@ -196,12 +258,14 @@ def run_ours(args, rank, world, dev):
     wl = W.WORKLOADS[args.workload]
     if args.T:
         wl = wl.replace(T=args.T)
-    ind, lays = make_group(wl, dev, dsa)
-    g = dsa.Group(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk, lays, wl.sm_scale, wl.d_v,
-                  pool=wl.pool)
-    t_chunk = args.t_chunk or max(1, min(wl.T, (args.score_ws_gb << 30) // (wl.B * ((wl.S // wl.pool + 3) // 4 * 4) * 4)))
-    ws = torch.empty(g.workspace_size(t_chunk), dtype=torch.uint8, device=dev)
-    step = lambda: g.forward(ws, stream)  # noqa: E731
+    boxes = rank_boxes(wl, world, rank)
+    parts = make_parts(wl, dev, dsa, boxes)
+    t_chunk = score_t_chunk(args, wl)
+    ws = torch.empty(max([1] + [p.g.workspace_size(t_chunk) for p in parts]), dtype=torch.uint8, device=dev)
+
+    def step():
+        for p in parts:
+            p.g.forward(ws, stream)
 
     for _ in range(args.warmup):
         step()
@@ -214,71 +278,83 @@ def run_ours(args, rank, world, dev):
     launches = dsa.launch_count() - l0
     ms = max_over_ranks(ms, world, dev)
     ms_step = ms / args.steps
-    value = job_throughput(wl.B * wl.T, world, ms_step)
+    # every query row of the workload is processed once per step, spread over the ranks
+    value = wl.B * wl.T / (ms_step / 1e3)
 
     # ---- per-kernel breakdown: the same step as separate C-ABI calls with events between them
-    brk = breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, args.steps if args.steps <= 3 else 3)
+    brk = breakdown(parts, ws, t_chunk, stream, dsa, args.steps if args.steps <= 3 else 3)
 
     res = {
         "metric": METRIC, "value": value, "unit": "query tok/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak" if world == 1 else "strong",
         "vs_baseline": None, "dtype": "fp8-e4m3 indexer / bf16 attention (fp32 accumulate)", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "ctx": wl.ctx, "H_I": wl.H_I, "d_I": wl.d_I,
                    "topk": wl.topk, "pool": wl.pool, "Hq": wl.Hq, "d_qk": wl.d_qk, "d_v": wl.d_v,
-                   "group": wl.group, "t_chunk": t_chunk, "parallelism": f"replicas x{world}",
+                   "group": wl.group, "t_chunk": t_chunk,
+                   "parallelism": "1 GPU" if world == 1 else
+                   (f"query rows sharded zig-zag over {world} ranks" if wl.T > 1 else f"batch sharded over {world} ranks"),
                    "l2": "inputs larger than L2 (126 MB); no flush"},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "breakdown_ms": brk,
     }
-    res["roofline"] = roofline(wl, brk, pk, t_chunk)
-    del g, ws
+    if world > 1:
+        res["config"]["rank0_rows"] = sum(p.wl.B * p.wl.T for p in parts)
+    res["roofline"] = roofline([p.wl for p in parts], brk, pk, t_chunk)
+    del ws
     torch.cuda.empty_cache()
-    return res, wl, ind, lays
+    return res, wl, parts
 
 
-def breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, reps):
-    """Average device time of each kernel family over `reps` steps, CUDA events on `stream`."""
-    S_eff = wl.S // wl.pool
-    ld = (S_eff + 3) // 4 * 4
-    scores = torch.empty((wl.B, t_chunk, ld), dtype=torch.float32, device=ind["q_idx"].device)
-    keys = ind["k_idx"]
+def breakdown(parts, ws, t_chunk, stream, dsa, reps):
+    """Average device time of each kernel family per step over `reps` steps, CUDA events on
+    `stream`, summed over this rank's parts."""
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     tot = {"pool": 0.0, "indexer": 0.0, "topk": 0.0, "attn": 0.0}
     n = {"indexer": 0, "topk": 0, "attn": 0, "pool": 0}
-    attn_ws = torch.empty(max(1, dsa.dsa_sparse_attn_workspace_size(wl.B, wl.T, wl.Hq, wl.d_v, wl.topk * wl.pool)),
-                          dtype=torch.uint8, device=scores.device)
-    for _ in range(reps):
-        marks = []
-        if wl.pool > 1:
-            a, b = ev(), ev()
-            a.record(stream)
-            keys = dsa.dsa_index_pool(ind["k_idx"], stream=stream)
-            b.record(stream)
-            marks.append(("pool", a, b))
-        for t0 in range(0, wl.T, t_chunk):
-            tc = min(t_chunk, wl.T - t0)
-            sc = scores.view(-1)[: wl.B * tc * ld].view(wl.B, tc, ld)   # [B, tc, ld], batch stride tc * ld
-            a, b, c = ev(), ev(), ev()
-            a.record(stream)
-            dsa.dsa_index_scores(ind["q_idx"], ind["w"], keys, ind["ctx_len"], pool=wl.pool, t_begin=t0, t_count=tc,
-                                 scores=sc, stream=stream)
-            b.record(stream)
-            dsa.dsa_topk(sc, ind["ctx_len"], wl.T, S_eff, wl.topk, pool=wl.pool, t_begin=t0, idx=g.idx,
-                         stream=stream)
-            c.record(stream)
-            marks += [("indexer", a, b), ("topk", b, c)]
-        for L in lays:
-            a, b = ev(), ev()
-            a.record(stream)
-            dsa.dsa_sparse_attn(L["q"], L["kv"], g.idx, wl.sm_scale, wl.d_v, v=L["v"], out=L["out"], ws=attn_ws,
-                                stream=stream)
-            b.record(stream)
-            marks.append(("attn", a, b))
-        torch.cuda.synchronize()
-        for name, a, b in marks:
-            tot[name] += a.elapsed_time(b)
-            n[name] += 1
+    dev = ws.device
+    for p in parts:
+        wl, ind, lays, g = p.wl, p.ind, p.lays, p.g
+        S_eff = ind["k_idx"].shape[1] // wl.pool
+        ld = (S_eff + 3) // 4 * 4
+        tc_max = min(t_chunk, wl.T)
+        scores = torch.empty((wl.B, tc_max, ld), dtype=torch.float32, device=dev)
+        attn_ws = torch.empty(max(1, dsa.dsa_sparse_attn_workspace_size(wl.B, wl.T, wl.Hq, wl.d_v, wl.topk * wl.pool)),
+                              dtype=torch.uint8, device=dev)
+        for _ in range(reps):
+            marks = []
+            keys = ind["k_idx"]
+            if wl.pool > 1:
+                a, b = ev(), ev()
+                a.record(stream)
+                keys = dsa.dsa_index_pool(ind["k_idx"], pool=wl.pool, stream=stream)
+                b.record(stream)
+                marks.append(("pool", a, b))
+            for t0 in range(0, wl.T, t_chunk):
+                tc = min(t_chunk, wl.T - t0)
+                sc = scores.view(-1)[: wl.B * tc * ld].view(wl.B, tc, ld)   # [B, tc, ld], batch stride tc * ld
+                a, b, c = ev(), ev(), ev()
+                a.record(stream)
+                dsa.dsa_index_scores(ind["q_idx"], ind["w"], keys, ind["ctx_len"], pool=wl.pool, t_begin=t0,
+                                     t_count=tc, scores=sc, stream=stream)
+                b.record(stream)
+                dsa.dsa_topk(sc, ind["ctx_len"], wl.T, S_eff, wl.topk, pool=wl.pool, t_begin=t0, idx=g.idx,
+                             stream=stream)
+                c.record(stream)
+                marks += [("indexer", a, b), ("topk", b, c)]
+            for L in g.layers:
+                a, b = ev(), ev()
+                a.record(stream)
+                dsa.dsa_sparse_attn(L["q"], L["kv"], g.idx, wl.sm_scale, wl.d_v, v=L["v"], out=L["out"], ws=attn_ws,
+                                    stream=stream)
+                b.record(stream)
+                marks.append(("attn", a, b))
+            torch.cuda.synchronize()
+            for name, a, b in marks:
+                tot[name] += a.elapsed_time(b)
+                n[name] += 1
+        del scores, attn_ws
     out = {k: tot[k] / reps for k in tot if n[k]}
     out["per_launch"] = {"indexer_chunk": tot["indexer"] / max(1, n["indexer"]),
                          "topk_chunk": tot["topk"] / max(1, n["topk"]), "attn_layer": tot["attn"] / max(1, n["attn"])}
@@ -294,29 +370,36 @@ def breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, reps):
 TRAFFIC_PER_QUERY = {("prefill128k", "attn"): 587.6e3}
 
 
-def roofline(wl, brk, pk, t_chunk):
-    """Roofline of the kernel with the largest share of the step."""
+def roofline(wls, brk, pk, t_chunk):
+    """Roofline of the kernel with the largest share of the step; `wls` are the (sub-)workloads
+    this rank ran, whose work adds up."""
+    wls = wls if isinstance(wls, (list, tuple)) else [wls]
+    wl = wls[0]
     fp8_peak = 2.0 * pk["bf16_sus"]   # nominal fp8:bf16 ratio 2 on the measured bf16 figure
+    n_layers = max(1, sum(1 for _ in range(wl.group)))
+    attn_launches = max(1, len(wls) * n_layers)
     ent = {
-        "indexer": {"bound": "tensor", "achieved": indexer_flops(wl) / (brk["indexer"] * 1e-3) / 1e12,
+        "indexer": {"bound": "tensor", "achieved": sum(indexer_flops(w) for w in wls) / (brk["indexer"] * 1e-3) / 1e12,
                     "peak": fp8_peak, "unit": "TFLOP/s", "dtype": "fp8", "traffic": None,
                     "peak_src": f"2 x {pk['src']} bf16 sustained"},
-        "attn": {"bound": "tensor", "achieved": attn_flops(wl) / (brk["per_launch"]["attn_layer"] * 1e-3) / 1e12,
+        "attn": {"bound": "tensor",
+                 "achieved": sum(attn_flops(w) for w in wls) * n_layers / (brk["attn"] * 1e-3) / 1e12,
                  "peak": pk["bf16_sus"], "unit": "TFLOP/s", "dtype": "bf16", "traffic": None,
                  "peak_src": f"{pk['src']} bf16 sustained"},
     }
     # top-k: reads every visible score once and writes k ids per row (HBM-bound)
-    topk_bytes = 4 * causal_pairs(wl) + 4 * wl.B * wl.T * wl.topk * wl.pool
+    topk_bytes = sum(4 * causal_pairs(w) + 4 * w.B * w.T * w.topk * w.pool for w in wls)
     ent["topk"] = {"bound": "hbm", "achieved": topk_bytes / (brk["topk"] * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
                    "unit": "GB/s", "traffic": None, "peak_src": f"{pk['src']} copy"}
-    if wl.B * wl.T <= 64:   # decode: the attention reads every gathered row once; HBM-bound
-        ent["attn"] = {"bound": "hbm", "achieved": attn_bytes(wl) / (brk["per_launch"]["attn_layer"] * 1e-3) / 1e9,
+    rows = sum(w.B * w.T for w in wls)
+    if rows <= 64:   # decode: the attention reads every gathered row once; HBM-bound
+        ent["attn"] = {"bound": "hbm", "achieved": sum(attn_bytes(w) for w in wls) * n_layers / (brk["attn"] * 1e-3) / 1e9,
                        "peak": pk["hbm_gbs"], "unit": "GB/s", "traffic": None, "peak_src": f"{pk['src']} copy"}
         ent["indexer"] = {"bound": "hbm",
-                          "achieved": (wl.B * wl.S * wl.d_I + wl.B * wl.T * wl.H_I * (wl.d_I + 4))
+                          "achieved": sum(w.B * (w.S // w.pool) * w.d_I + w.B * w.T * w.H_I * (w.d_I + 4) for w in wls)
                           / (brk["indexer"] * 1e-3) / 1e9,
                           "peak": pk["hbm_gbs"], "unit": "GB/s", "traffic": None, "peak_src": f"{pk['src']} copy"}
-    for k, queries in (("attn", wl.B * wl.T), ("indexer", wl.B * min(t_chunk, wl.T))):
+    for k, queries in (("attn", rows / len(wls)), ("indexer", min(t_chunk, rows))):
         per_q = TRAFFIC_PER_QUERY.get((wl.name, k))
         ent[k]["traffic"] = None if per_q is None else per_q * queries   # bytes per launch
     top = max(("indexer", "attn", "topk"), key=lambda k: brk[k])
@@ -328,42 +411,48 @@ def roofline(wl, brk, pk, t_chunk):
     return r
 
 
-def run_e2e(args, wl, ind, lays, dev, stream):
-    """Same step from pinned host memory: H2D of every input, the group call, D2H of every output."""
-    import indexed_sparse_attention_fp8_b200 as dsa
-    host = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in ind.items()}
-    for k in host:
-        host[k].copy_(ind[k])
-    hq = torch.empty_like(lays[0]["q"], device="cpu").pin_memory()
-    hkv = torch.empty_like(lays[0]["kv"], device="cpu").pin_memory()
-    hq.copy_(lays[0]["q"])
-    hkv.copy_(lays[0]["kv"])
-    g = dsa.Group(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk, lays, wl.sm_scale, wl.d_v, pool=wl.pool)
-    hout = torch.empty_like(g.layers[0]["out"], device="cpu").pin_memory()
-    t_chunk = args.t_chunk or max(1, min(wl.T, (args.score_ws_gb << 30) // (wl.B * ((wl.S // wl.pool + 3) // 4 * 4) * 4)))
-    ws = torch.empty(g.workspace_size(t_chunk), dtype=torch.uint8, device=dev)
-    h2d = sum(v.numel() * v.element_size() for v in host.values()) + len(lays) * (
-        hq.numel() * hq.element_size() + hkv.numel() * hkv.element_size())
-    d2h = len(lays) * hout.numel() * hout.element_size() + g.idx.numel() * 4
-    hidx = torch.empty_like(g.idx, device="cpu").pin_memory()
+def run_e2e(args, wl, parts, dev, stream, world):
+    """Same step from pinned host memory: per part, H2D of every input, the group call, D2H of
+    every output."""
+    t_chunk = score_t_chunk(args, wl)
+    ws = torch.empty(max([1] + [p.g.workspace_size(t_chunk) for p in parts]), dtype=torch.uint8, device=dev)
+    steps_fns, h2d, d2h = [], 0, 0
+    for p in parts:
+        host = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in p.ind.items()}
+        for k in host:
+            host[k].copy_(p.ind[k])
+        hq = torch.empty_like(p.lays[0]["q"], device="cpu").pin_memory()
+        hkv = torch.empty_like(p.lays[0]["kv"], device="cpu").pin_memory()
+        hq.copy_(p.lays[0]["q"])
+        hkv.copy_(p.lays[0]["kv"])
+        hout = torch.empty_like(p.g.layers[0]["out"], device="cpu").pin_memory()
+        hidx = torch.empty_like(p.g.idx, device="cpu").pin_memory()
+        h2d += sum(v.numel() * v.element_size() for v in host.values()) + len(p.lays) * (
+            hq.numel() * hq.element_size() + hkv.numel() * hkv.element_size())
+        d2h += len(p.lays) * hout.numel() * hout.element_size() + p.g.idx.numel() * 4
+
+        def fn(p=p, host=host, hq=hq, hkv=hkv, hout=hout, hidx=hidx):
+            for k in host:
+                p.ind[k].copy_(host[k], non_blocking=True)
+            for L in p.g.layers:
+                L["q"].copy_(hq, non_blocking=True)
+                L["kv"].copy_(hkv, non_blocking=True)
+            p.g.forward(ws, stream)
+            for L in p.g.layers:
+                hout.copy_(L["out"], non_blocking=True)
+            hidx.copy_(p.g.idx, non_blocking=True)
+        steps_fns.append(fn)
 
     def step():
-        for k in host:
-            ind[k].copy_(host[k], non_blocking=True)
-        for L in g.layers:
-            L["q"].copy_(hq, non_blocking=True)
-            L["kv"].copy_(hkv, non_blocking=True)
-        g.forward(ws, stream)
-        for L in g.layers:
-            hout.copy_(L["out"], non_blocking=True)
-        hidx.copy_(g.idx, non_blocking=True)
+        for fn in steps_fns:
+            fn()
 
     step()
     torch.cuda.synchronize()
     steps = max(1, min(args.steps, args.e2e_steps))
     ms = time_region(step, steps, stream) / steps
-    del ws, g
-    return {"value": job_throughput(wl.B * wl.T, 1, ms), "unit": "query tok/s", "ms_per_step": ms, "steps": steps,
+    del ws
+    return {"value": wl.B * wl.T / (ms / 1e3), "unit": "query tok/s", "ms_per_step": ms, "steps": steps,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
@@ -373,19 +462,18 @@ def run_secondary(args, name, dev, steps=3, per_layer=False):
     stream = torch.cuda.current_stream()
     wl = W.WORKLOADS[name]
     if not per_layer:
-        ind, lays = make_group(wl, dev, dsa)
-        g = dsa.Group(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk, lays, wl.sm_scale, wl.d_v,
-                      pool=wl.pool)
+        parts = make_parts(wl, dev, dsa, rank_boxes(wl, 1, 0))
+        g = parts[0].g
         t_chunk = max(1, min(wl.T, (args.score_ws_gb << 30) // (wl.B * ((wl.S // wl.pool + 3) // 4 * 4) * 4)))
         ws = torch.empty(g.workspace_size(t_chunk), dtype=torch.uint8, device=dev)
         fn = lambda: g.forward(ws, stream)  # noqa: E731
         for _ in range(max(3, args.warmup)):
             fn()
         ms = time_region(fn, steps, stream) / steps
-        brk = breakdown(wl, ind, lays, g, ws, t_chunk, stream, dsa, 3)
+        brk = breakdown(parts, ws, t_chunk, stream, dsa, 3)
         r = {"workload": name, "value": wl.B * wl.T / (ms / 1e3), "unit": "query tok/s", "ms_per_step": ms,
-             "steps": steps, "breakdown_ms": brk, "roofline": roofline(wl, brk, peaks(), t_chunk)}
-        del g, ws, ind, lays
+             "steps": steps, "breakdown_ms": brk, "roofline": roofline([parts[0].wl], brk, peaks(), t_chunk)}
+        del g, ws, parts
         torch.cuda.empty_cache()
         return r
     # per-layer indexer: each layer runs its own indexer + top-k (group_size 1, own indexer inputs)
@@ -513,6 +601,11 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        # one process per GPU: N GPUs need N ranks (torch.distributed.run --nproc-per-node N)
+        sys.stderr.write(f"bench.py --gpus {args.gpus} needs {args.gpus} ranks, found WORLD_SIZE={world}: run it "
+                         f"under python -m torch.distributed.run --nproc-per-node {args.gpus}\n")
+        sys.exit(2)
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl" if args.impl == "ours" else "gloo",
@@ -527,25 +620,29 @@ def main():
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    res, wl, ind, lays = run_ours(args, rank, world, dev)
+    res, wl, parts = run_ours(args, rank, world, dev)
     if not args.no_e2e:
         try:
-            e2e = run_e2e(args, wl, ind, lays, dev, torch.cuda.current_stream())
+            e2e = run_e2e(args, wl, parts, dev, torch.cuda.current_stream(), world)
         except (RuntimeError, torch.cuda.OutOfMemoryError) as e:  # pinned host memory can run out
             e2e = {"error": str(e)[:300]}
         # every rank joins the reduction, a failed one with an infinite time
         ms = max_over_ranks(e2e.get("ms_per_step", math.inf), world, dev)
+        h2d = sum_over_ranks(e2e.get("h2d_bytes_per_step", 0), world, dev)
+        d2h = sum_over_ranks(e2e.get("d2h_bytes_per_step", 0), world, dev)
         if "error" not in e2e:
             if math.isfinite(ms):
-                e2e.update(value=job_throughput(wl.B * wl.T, world, ms), ms_per_step=ms)
+                # every query row crosses once per step, spread over the ranks; bytes of all ranks
+                e2e.update(value=wl.B * wl.T / (ms / 1e3), ms_per_step=ms, h2d_bytes_per_step=int(h2d),
+                           d2h_bytes_per_step=int(d2h))
             else:
                 e2e = {"error": "the end-to-end step failed on another rank"}
         res["e2e"] = e2e
-    del ind, lays
+    del parts
     torch.cuda.empty_cache()
     if world > 1:
         torch.distributed.barrier()
-    if rank == 0 and not args.no_secondary and args.workload == "prefill128k":
+    if world == 1 and not args.no_secondary and args.workload == "prefill128k":
         try:
             pl = run_secondary(args, "prefill128k", dev, steps=2, per_layer=True)
             pl["indexshare_speedup"] = pl["ms_per_step"] / res["ms_per_step"]
@@ -553,6 +650,8 @@ def main():
         except torch.cuda.OutOfMemoryError as e:  # pragma: no cover
             res["per_layer_indexer"] = {"error": str(e)[:200]}
         res["decode256k"] = run_secondary(args, "decode256k", dev, steps=10)
+        # IndexPool at decode: 4 keys pooled into one, top-512 blocks
+        res["decode256k_pool"] = run_secondary(args, "decode256k_pool", dev, steps=10)
         # IndexPool at a 1M-token cache: 8192 new queries, without and with pooling of 4 keys
         for name in ("chunk1m", "chunk1m_pool"):
             try:

@@ -10,7 +10,8 @@
  *   - twiscan.com post on GLM-5.2 (IndexShare): the indexer runs in FP8; one indexer is
  *     shared by a group of 4 layers and the other 3 reuse its selection.
  *   - "GLM-5.3-Flash hybrid sparse-linear attention with IndexPool", section "What
- *     changed": IndexPool pools four indexer keys into one.
+ *     changed": IndexPool pools four indexer keys into one (factors 2 and 8 take the same
+ *     mean over 2 or 8 keys).
  *
  * Conventions shared by every entry point
  *   Positions   Sequence b holds ctx_len[b] keys (rows 0..ctx_len[b]-1 of its caches) and T
@@ -51,7 +52,8 @@ typedef enum {
   DSA_ERR_MISALIGNED = 3,          /* pointer or stride not 16-byte aligned */
   DSA_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes below the size the *_workspace_size call gives */
   DSA_ERR_CUDA = 5,                /* a CUDA launch failed; see dsa_last_cuda_error() */
-  DSA_ERR_TIMEOUT = 6              /* a bounded device-side wait gave up (kernel exited early) */
+  DSA_ERR_TIMEOUT = 6,             /* a bounded device-side wait gave up (kernel exited early) */
+  DSA_ERR_INDEX_RANGE = 7          /* an attention call met a selected id >= its S_kv (skipped) */
 } dsa_status;
 
 /* Static, NUL-terminated description of a status code (thread-safe). */
@@ -65,10 +67,12 @@ int dsa_last_cuda_error(void);
 uint64_t dsa_launch_count(void);
 
 /* Synchronises `stream`, then reads and clears the device status words of the library's
- * kernels on the current device.  Returns DSA_OK, or DSA_ERR_TIMEOUT when a kernel gave up
- * one of its bounded waits since the last call (that launch exited early and its outputs
- * are incomplete), or DSA_ERR_CUDA if the synchronisation failed.  Every wait inside the
- * tensor-core kernels has a time limit, so no launch can hang. */
+ * kernels on the current device.  Returns DSA_OK; DSA_ERR_TIMEOUT when a kernel gave up one
+ * of its bounded waits since the last call (that launch exited early and its outputs are
+ * incomplete); else DSA_ERR_INDEX_RANGE when an attention launch met a selected id at or
+ * beyond its S_kv (that id was skipped like a -1, and nothing outside the cache was read);
+ * or DSA_ERR_CUDA if the synchronisation failed.  Every wait inside the tensor-core kernels
+ * has a time limit, so no launch can hang. */
 int dsa_device_status(void* stream);
 
 /* Test hook for the failure path: enqueues one thread that waits, through the kernels' own
@@ -76,6 +80,27 @@ int dsa_device_status(void* stream);
  * limit_ns (1 ns .. 1 s) and sets the device status word; the next dsa_device_status() then
  * returns DSA_ERR_TIMEOUT.  Faults nothing; the CUDA context stays usable. */
 int dsa_debug_wait_timeout(uint64_t limit_ns, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * Paged caches (optional on every call that reads a cache; NULL = contiguous per sequence).
+ * The serving form of decode and chunked prefill: every cache the call reads (indexer keys
+ * k_idx, latent/K rows kv, separate V rows v) is a pool of num_pages pages of page_size rows
+ * shared by all sequences, and logical row s of sequence b is physical row
+ *     block_table[b * pages_per_seq + s / page_size] * page_size + s % page_size
+ * of each pool (k_idx: rows of d_I bytes; kv and v: rows at the call's row strides; their
+ * batch strides are unused).  A sequence holds up to pages_per_seq * page_size logical rows,
+ * which bounds S_max and S_kv.  page_size is a power of two >= 128, so a key tile of the
+ * indexer never straddles a page.  block_table is a DEVICE array [B, pages_per_seq] of int32
+ * page ids in [0, num_pages); an id outside that range is never followed (the indexer reads
+ * zeros in its place, the attention skips the row) and dsa_device_status() then returns
+ * DSA_ERR_INDEX_RANGE.
+ * ------------------------------------------------------------------------------------ */
+typedef struct dsa_paging {
+  const int32_t* block_table;   /* device [B, pages_per_seq] int32 page ids */
+  int32_t page_size;            /* rows per page: a power of two >= 128 */
+  int32_t pages_per_seq;        /* columns of block_table */
+  int32_t num_pages;            /* pages in each pool */
+} dsa_paging;
 
 /* ------------------------------------------------------------------------------------
  * dsa_index_scores - the lightning indexer (Stage 1, coarse scoring; FP8 per the
@@ -91,13 +116,14 @@ int dsa_debug_wait_timeout(uint64_t limit_ns, void* stream);
  *   scores [B, t_count, ld] fp32 out:  row (b, t - t_begin); entries s < n_valid hold I;
  *          entries from n_valid up to the end of the 128-key tile that holds the last
  *          visible key are -inf; entries beyond are not written.
- *   pool   1, or 4 when k_idx holds IndexPool blocks (validity 4*s <= pos).
+ *   pool   1, or 2, 4 or 8 when k_idx holds IndexPool blocks (validity pool*s <= pos).
+ *   paging NULL, or the page pool k_idx is (pool == 1 only; see dsa_paging).
  * Supported: (H_I, d_I) in {(4, 64), (64, 128)}; ld >= S_max, ld % 4 == 0.
  * ------------------------------------------------------------------------------------ */
 int dsa_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                      const int32_t* ctx_len, int B, int T, int S_max, int H_I, int d_I,
                      int pool, int t_begin, int t_count, float* scores, int64_t ld,
-                     void* stream);
+                     const dsa_paging* paging, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * dsa_topk - Stage 2, fine selection: per query row, the k_eff = min(k, n_valid) keys with
@@ -108,7 +134,7 @@ int dsa_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
  *
  *   scores  [B, t_count, ld] fp32 (as written by dsa_index_scores for the same t_begin)
  *   idx     [B, T, k*pool] int32 out; rows t_begin .. t_begin+t_count-1 are written.
- * Supported: 1 <= k <= 2048, pool in {1, 4}, ld % 4 == 0.
+ * Supported: 1 <= k <= 2048, pool in {1, 2, 4, 8}, ld % 4 == 0.
  * ------------------------------------------------------------------------------------ */
 int dsa_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, int T, int S_max,
              int pool, int t_begin, int t_count, int k, int32_t* idx, void* stream);
@@ -129,32 +155,38 @@ int dsa_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, int
  *   q    [B, T, Hq, d_qk] bf16 (contiguous)
  *   kv   K rows: element (b, s, c) at kv[b*kv_batch_stride + s*kv_row_stride + c], c < d_qk
  *   v    V rows, same form with v_* strides; NULL means V = the first d_v columns of kv
- *   idx  [B, T, k] int32, entries in [0, ctx_len[b]) or < 0 (entries are not range-checked on
- *        the device: one at or beyond the end of the cache reads memory outside it)
+ *   S_kv rows per sequence in the K/V caches (>= 1).  The kernels check every selected id on
+ *        the device: an id >= S_kv is skipped like a -1 (nothing outside the cache is read)
+ *        and the next dsa_device_status() returns DSA_ERR_INDEX_RANGE.
+ *   idx  [B, T, k] int32, entries in [0, S_kv) (normally [0, ctx_len[b])) or < 0
  *   out  [B, T, Hq, d_v] bf16          lse  [B, T, Hq] fp32 or NULL
  *   ws   scratch of at least dsa_sparse_attn_workspace_size(B, T, Hq, d_v, k) bytes
  *        (zero for long prefill; split-key partials for few-query batches such as decode)
+ *   paging NULL, or the page pools kv (and v) are (see dsa_paging; S_kv <= its capacity)
  * Supported: (Hq, d_qk, d_v) in {(16, 128, 128), (128, 576, 512)}; 1 <= k <= 8192.
  * ------------------------------------------------------------------------------------ */
 size_t dsa_sparse_attn_workspace_size(int B, int T, int Hq, int d_v, int k);
 int dsa_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v,
                     int64_t kv_row_stride, int64_t kv_batch_stride, int64_t v_row_stride,
-                    int64_t v_batch_stride, const int32_t* idx, int B, int T, int Hq, int d_qk,
+                    int64_t v_batch_stride, int S_kv, const int32_t* idx, int B, int T, int Hq, int d_qk,
                     int d_v, int k, float sm_scale, uint16_t* out, float* lse, void* ws,
-                    size_t ws_bytes, void* stream);
+                    size_t ws_bytes, const dsa_paging* paging, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * dsa_sparse_attn_noalloc - dsa_sparse_attn for callers that can neither allocate device
  * memory nor pass a workspace (for example an operator inside a runtime that owns all device
  * memory and offers its operators no scratch, or a serving loop that must not call cudaMalloc
  * once it runs).  The method described in the sources has no counterpart to this call: it is
- * a deployment variant.  Same arguments, layouts and results as dsa_sparse_attn minus `ws`;
- * the split-key partials go to a fixed scratch array inside the library instead.
+ * a deployment variant.  Same arguments, layouts, checks and results as dsa_sparse_attn minus
+ * `ws`; the split-key partials go to a fixed scratch array inside the library instead.
  *   - The scratch is dsa_noalloc_scratch_bytes() (16 MiB) per GPU that loads the library,
- *     held until the process exits.  Problems whose partials need more (see
- *     dsa_sparse_attn_workspace_size) return DSA_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
+ *     held until the process exits.  When the default key split of a problem would need more
+ *     partials than that (see dsa_sparse_attn_workspace_size), the call runs at the largest
+ *     split count whose partials fit, down to one split, which needs no scratch: no problem
+ *     is rejected for its size, larger ones only spread over fewer CTAs.
  *   - The first call on a device looks up the scratch's device address (with that device
- *     current) and caches it; make that first call before any stream capture.
+ *     current) and caches it; make that first call before any stream capture.  A
+ *     cudaDeviceReset() invalidates the cached address.
  *   - All calls on a device share the scratch: calls whose kernels may overlap on the GPU
  *     (other streams, other host threads) race on it and must be serialised by the caller.
  *     Nothing in the scratch needs to start at zero; a call ignores what the last one left.
@@ -163,28 +195,30 @@ int dsa_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v,
 size_t dsa_noalloc_scratch_bytes(void);
 int dsa_sparse_attn_noalloc(const uint16_t* q, const uint16_t* kv, const uint16_t* v,
                             int64_t kv_row_stride, int64_t kv_batch_stride, int64_t v_row_stride,
-                            int64_t v_batch_stride, const int32_t* idx, int B, int T, int Hq,
+                            int64_t v_batch_stride, int S_kv, const int32_t* idx, int B, int T, int Hq,
                             int d_qk, int d_v, int k, float sm_scale, uint16_t* out, float* lse,
-                            void* stream);
+                            const dsa_paging* paging, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * dsa_index_pool - IndexPool ("What changed": four indexer keys pooled into one):
  *     k_pool[b, g, :] = e4m3(((k[4g] + k[4g+1]) + (k[4g+2] + k[4g+3])) * 0.25)
- * with the sum in fp32 on the decoded keys and the requantisation round-to-nearest-even,
+ * and for pool = 2 or 8 the same mean over 2 or 8 keys (a balanced pairwise sum times
+ * 1/pool; exact in fp32 before the requantisation, which is the only rounding) * with the sum in fp32 on the decoded keys and the requantisation round-to-nearest-even,
  * saturating at +-448.
- *   k_idx [B, S_max, d_I] e4m3 -> k_pool [B, S_max/4, d_I] e4m3.
- * Supported: pool == 4, S_max % 4 == 0, d_I % 16 == 0.
+ *   k_idx [B, S_max, d_I] e4m3 (or its page pool when paging != NULL)
+ *   -> k_pool [B, S_max/pool, d_I] e4m3 (always contiguous).
+ * Supported: pool in {2, 4, 8}, S_max % pool == 0, d_I % 16 == 0.
  * ------------------------------------------------------------------------------------ */
 int dsa_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool, uint8_t* k_pool,
-                   void* stream);
+                   const dsa_paging* paging, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * dsa_group_forward - one IndexShare group ("IndexShare: Amortizing the Indexer"): the
  * indexer and the top-k run ONCE, and each of the group_size attention layers reads the
  * same index buffer.  Equivalent to dsa_index_scores + dsa_topk over all queries
  * (processed in query chunks sized to the workspace), then group_size x dsa_sparse_attn.
- * With pool == 4 the indexer runs on dsa_index_pool's blocks and `topk` counts blocks
- * (idx then holds 4*topk token ids per row).  The comparator without IndexShare is
+ * With pool > 1 the indexer runs on dsa_index_pool's blocks and `topk` counts blocks
+ * (idx then holds pool*topk token ids per row).  The comparator without IndexShare is
  * group_size calls with group_size = 1 and per-layer indexer tensors.
  * ------------------------------------------------------------------------------------ */
 typedef struct dsa_group_args {
@@ -194,8 +228,8 @@ typedef struct dsa_group_args {
   const uint8_t* k_idx;    /* [B, S_max, d_I] e4m3 */
   const int32_t* ctx_len;  /* device [B] */
   int32_t B, T, S_max, H_I, d_I;
-  int32_t topk;            /* keys (pool 1) or blocks (pool 4) selected per query */
-  int32_t pool;            /* 1 or 4 (IndexPool) */
+  int32_t topk;            /* keys (pool 1) or blocks (pool > 1) selected per query */
+  int32_t pool;            /* 1, or 2, 4 or 8 (IndexPool) */
   int32_t group_size;      /* attention layers sharing the selection, 1..16 */
   /* attention, one entry per layer: HOST arrays of group_size DEVICE pointers */
   const uint16_t* const* q;   /* [B, T, Hq, d_qk] bf16 */
@@ -208,6 +242,8 @@ typedef struct dsa_group_args {
   int32_t Hq, d_qk, d_v;
   float sm_scale;
   int32_t* idx;            /* [B, T, topk*pool] int32 out: the shared selection */
+  dsa_paging paging;       /* block_table NULL: contiguous caches; else k_idx and every
+                              layer's kv (and v) are page pools sharing this table */
 } dsa_group_args;
 
 /* Workspace for dsa_group_forward when the indexer is run over chunks of t_chunk queries

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libdsa_b200.so")
 _c_int, _c_i64, _c_p, _c_sz, _c_f = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
 
 STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED_SHAPE", 3: "DSA_ERR_MISALIGNED",
-          4: "DSA_ERR_WORKSPACE_TOO_SMALL", 5: "DSA_ERR_CUDA", 6: "DSA_ERR_TIMEOUT"}
+          4: "DSA_ERR_WORKSPACE_TOO_SMALL", 5: "DSA_ERR_CUDA", 6: "DSA_ERR_TIMEOUT", 7: "DSA_ERR_INDEX_RANGE"}
 
 
 class DSAError(RuntimeError):
@@ -30,6 +30,27 @@ class DSAError(RuntimeError):
         if status == 5:
             msg += f" (cudaError {_lib().dsa_last_cuda_error()})"
         super().__init__(msg)
+
+
+class Paging(ctypes.Structure):
+    """Mirror of dsa_paging in include/dsa.h: logical row s of sequence b lives at physical row
+    block_table[b, s // page_size] * page_size + s % page_size of each page pool."""
+    _fields_ = [("block_table", _c_p), ("page_size", ctypes.c_int32), ("pages_per_seq", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32)]
+
+
+def paging(block_table: torch.Tensor, page_size: int, num_pages: int) -> Paging:
+    """A page map for the calls below: block_table [B, pages_per_seq] int32 on the device (kept
+    alive by the returned object), page_size a power of two >= 128, num_pages pages per pool."""
+    _layout("block_table", block_table, torch.int32, (-1, -1))
+    p = Paging(block_table=_ptr(block_table), page_size=int(page_size), pages_per_seq=int(block_table.shape[1]),
+               num_pages=int(num_pages))
+    p._table = block_table
+    return p
+
+
+def _paging_ref(p: Optional[Paging]):
+    return None if p is None else ctypes.byref(p)
 
 
 class GroupArgs(ctypes.Structure):
@@ -44,7 +65,7 @@ class GroupArgs(ctypes.Structure):
         ("kv_row_stride", _c_i64), ("kv_batch_stride", _c_i64), ("v_row_stride", _c_i64),
         ("v_batch_stride", _c_i64),
         ("Hq", ctypes.c_int32), ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32), ("sm_scale", _c_f),
-        ("idx", _c_p),
+        ("idx", _c_p), ("paging", Paging),
     ]
 
 
@@ -58,15 +79,17 @@ _SIGS = {
     "dsa_device_status": (_c_int, [_c_p]),
     "dsa_debug_wait_timeout": (_c_int, [ctypes.c_uint64, _c_p]),
     "dsa_index_scores": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
-                                  _c_int, _c_int, _c_p, _c_i64, _c_p]),
+                                  _c_int, _c_int, _c_p, _c_i64, ctypes.POINTER(Paging), _c_p]),
     "dsa_topk": (_c_int, [_c_p, _c_i64, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p]),
     "dsa_sparse_attn_workspace_size": (_c_sz, [_c_int, _c_int, _c_int, _c_int, _c_int]),
-    "dsa_sparse_attn": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_int, _c_int, _c_int,
-                                 _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_sz, _c_p]),
-    "dsa_index_pool": (_c_int, [_c_p, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p]),
+    "dsa_sparse_attn": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_p, _c_int, _c_int,
+                                 _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_sz, ctypes.POINTER(Paging),
+                                 _c_p]),
+    "dsa_index_pool": (_c_int, [_c_p, _c_int, _c_int, _c_int, _c_int, _c_p, ctypes.POINTER(Paging), _c_p]),
     "dsa_noalloc_scratch_bytes": (_c_sz, []),
-    "dsa_sparse_attn_noalloc": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_int, _c_int,
-                                         _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p]),
+    "dsa_sparse_attn_noalloc": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_p, _c_int,
+                                         _c_int, _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p,
+                                         ctypes.POINTER(Paging), _c_p]),
     "dsa_group_workspace_size": (_c_sz, [ctypes.POINTER(GroupArgs), _c_int]),
     "dsa_group_forward": (_c_int, [ctypes.POINTER(GroupArgs), _c_p, _c_sz, _c_p]),
 }
@@ -116,12 +139,19 @@ def _layout(name: str, t: Optional[torch.Tensor], dtype: torch.dtype, shape: Seq
         raise ValueError(f"{name}: strides {t.stride()}, expected {tuple(strides)}")
 
 
-def _kv_layout(name: str, t: Optional[torch.Tensor], B: int, width: int) -> None:
+def _kv_layout(name: str, t: Optional[torch.Tensor], B: int, width: int, pg: Optional[Paging] = None) -> None:
     """A K or V cache [B, S, >= width] bf16 with unit inner stride and row / batch strides that
-    are multiples of 8 elements (16 bytes)."""
+    are multiples of 8 elements (16 bytes); with paging, a page pool [num_pages, page_size,
+    >= width] whose pages follow each other at the row stride."""
     if t is None:
         return
-    _layout(name, t, torch.bfloat16, (B, -1, -1), (-1, -1, 1))
+    if pg is not None:
+        _layout(name, t, torch.bfloat16, (pg.num_pages, pg.page_size, -1), (-1, -1, 1))
+        if t.stride(0) != pg.page_size * t.stride(1):
+            raise ValueError(f"{name}: pages must follow each other at the row stride (strides {t.stride()})")
+        B = pg.num_pages
+    else:
+        _layout(name, t, torch.bfloat16, (B, -1, -1), (-1, -1, 1))
     if t.shape[2] < width or t.stride(1) < width or t.stride(1) % 8 or t.stride(0) % 8:
         raise ValueError(f"{name}: shape {tuple(t.shape)} strides {t.stride()} cannot hold {width}-wide rows "
                          "at 16-byte aligned row and batch strides")
@@ -138,8 +168,9 @@ def launch_count() -> int:
 
 
 def dsa_device_status(stream=None) -> int:
-    """Synchronises the stream and returns (and clears) the kernels' device status: 0, or 6
-    (DSA_ERR_TIMEOUT) when a bounded device wait gave up."""
+    """Synchronises the stream and returns (and clears) the kernels' device status: 0, 6
+    (DSA_ERR_TIMEOUT) when a bounded device wait gave up, or 7 (DSA_ERR_INDEX_RANGE) when an
+    attention call met a selected id beyond its cache and skipped it."""
     return int(_lib().dsa_device_status(_stream(stream)))
 
 
@@ -153,16 +184,21 @@ def dsa_debug_wait_timeout(limit_ns: int, stream=None) -> None:
 
 def dsa_index_scores(q_idx: torch.Tensor, w: torch.Tensor, k_idx: torch.Tensor, ctx_len: torch.Tensor,
                      pool: int = 1, t_begin: int = 0, t_count: Optional[int] = None,
-                     scores: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                     scores: Optional[torch.Tensor] = None, paging: Optional[Paging] = None,
+                     stream=None) -> torch.Tensor:
     """Indexer scores [B, t_count, ld] fp32 of queries t_begin.. (see dsa_index_scores in dsa.h).
-    q_idx [B,T,H_I,d_I] uint8 (e4m3), w [B,T,H_I] f32, k_idx [B,S,d_I] uint8, ctx_len [B] i32."""
+    q_idx [B,T,H_I,d_I] uint8 (e4m3), w [B,T,H_I] f32, k_idx [B,S,d_I] uint8 (or its page pool
+    [num_pages, page_size, d_I] with `paging`), ctx_len [B] i32."""
     B, T, H, D = q_idx.shape
-    S = k_idx.shape[1]
+    S = k_idx.shape[1] if paging is None else paging.pages_per_seq * paging.page_size
     tc = T - t_begin if t_count is None else t_count
     ld = (S + 3) // 4 * 4
     _layout("q_idx", q_idx, torch.uint8, (B, T, H, D))
     _layout("w", w, torch.float32, (B, T, H))
-    _layout("k_idx", k_idx, torch.uint8, (B, S, D))
+    if paging is None:
+        _layout("k_idx", k_idx, torch.uint8, (B, S, D))
+    else:
+        _layout("k_idx", k_idx, torch.uint8, (paging.num_pages, paging.page_size, D))
     _layout("ctx_len", ctx_len, torch.int32, (B,))
     if scores is None:
         scores = torch.empty((B, tc, ld), dtype=torch.float32, device=q_idx.device)
@@ -171,7 +207,7 @@ def dsa_index_scores(q_idx: torch.Tensor, w: torch.Tensor, k_idx: torch.Tensor, 
         _layout("scores", scores, torch.float32, (B, tc, -1), (tc * ld, ld, 1))
     _check("dsa_index_scores", _lib().dsa_index_scores(
         _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(ctx_len), B, T, S, H, D, pool, t_begin, tc, _ptr(scores), ld,
-        _stream(stream)))
+        _paging_ref(paging), _stream(stream)))
     return scores
 
 
@@ -189,11 +225,19 @@ def dsa_topk(scores: torch.Tensor, ctx_len: torch.Tensor, T: int, S_max: int, k:
     return idx
 
 
-def _attn_layouts(q, kv, v, idx, d_v, out, lse) -> None:
+def _cache_rows(kv: torch.Tensor, v: Optional[torch.Tensor], pg: Optional[Paging] = None) -> int:
+    """Rows per sequence of the K/V caches (logical rows when paged): selected ids at or beyond
+    it are skipped on the device."""
+    if pg is not None:
+        return pg.pages_per_seq * pg.page_size
+    return int(kv.shape[1] if v is None else min(kv.shape[1], v.shape[1]))
+
+
+def _attn_layouts(q, kv, v, idx, d_v, out, lse, pg: Optional[Paging] = None) -> None:
     B, T, Hq, Dqk = q.shape
     _layout("q", q, torch.bfloat16, (B, T, Hq, Dqk))
-    _kv_layout("kv", kv, B, Dqk)
-    _kv_layout("v", v, B, d_v)
+    _kv_layout("kv", kv, B, Dqk, pg)
+    _kv_layout("v", v, B, d_v, pg)
     _layout("idx", idx, torch.int32, (B, T, -1))
     _layout("out", out, torch.bfloat16, (B, T, Hq, d_v))
     _layout("lse", lse, torch.float32, (B, T, Hq))
@@ -206,12 +250,13 @@ def dsa_sparse_attn_workspace_size(B: int, T: int, Hq: int, d_v: int, k: int) ->
 def dsa_sparse_attn(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, sm_scale: float, d_v: int,
                     v: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
                     lse: Optional[torch.Tensor] = None, want_lse: bool = False,
-                    ws: Optional[torch.Tensor] = None, stream=None):
-    """Sparse attention: q [B,T,Hq,d_qk] bf16, kv [B,S,*] bf16 (K rows; V = kv[..., :d_v] when v is None),
-    idx [B,T,k] int32.  Returns (out [B,T,Hq,d_v] bf16, lse [B,T,Hq] f32 or None)."""
+                    ws: Optional[torch.Tensor] = None, paging: Optional[Paging] = None, stream=None):
+    """Sparse attention: q [B,T,Hq,d_qk] bf16, kv [B,S,*] bf16 (K rows; V = kv[..., :d_v] when v is None;
+    page pools [num_pages, page_size, *] with `paging`), idx [B,T,k] int32.
+    Returns (out [B,T,Hq,d_v] bf16, lse [B,T,Hq] f32 or None)."""
     B, T, Hq, Dqk = q.shape
     k = idx.shape[-1]
-    _attn_layouts(q, kv, v, idx, d_v, out, lse)
+    _attn_layouts(q, kv, v, idx, d_v, out, lse, paging)
     if out is None:
         out = torch.empty((B, T, Hq, d_v), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
@@ -223,20 +268,23 @@ def dsa_sparse_attn(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, sm_sca
     v_rs = v.stride(1) if v is not None else 0
     v_bs = v.stride(0) if v is not None else 0
     _check("dsa_sparse_attn", _lib().dsa_sparse_attn(
-        _ptr(q), _ptr(kv), _ptr(v), kv.stride(1), kv.stride(0), v_rs, v_bs, _ptr(idx), B, T, Hq, Dqk, d_v, k,
-        float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws), wsb, _stream(stream)))
+        _ptr(q), _ptr(kv), _ptr(v), kv.stride(1), kv.stride(0), v_rs, v_bs, _cache_rows(kv, v, paging), _ptr(idx), B,
+        T, Hq, Dqk, d_v, k,
+        float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws), wsb, _paging_ref(paging), _stream(stream)))
     return out, lse
 
 
 def dsa_sparse_attn_noalloc(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, sm_scale: float, d_v: int,
                             v: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                            lse: Optional[torch.Tensor] = None, want_lse: bool = False, stream=None):
+                            lse: Optional[torch.Tensor] = None, want_lse: bool = False,
+                            paging: Optional[Paging] = None, stream=None):
     """dsa_sparse_attn without a workspace: split partials use the library's fixed scratch
-    (dsa_noalloc_scratch_bytes() per GPU).  For callers that cannot allocate device memory;
-    calls that may overlap on one GPU share that scratch and must be serialised."""
+    (dsa_noalloc_scratch_bytes() per GPU; problems whose default split would not fit run at fewer
+    splits).  For callers that cannot allocate device memory; calls that may overlap on one GPU
+    share that scratch and must be serialised."""
     B, T, Hq, Dqk = q.shape
     k = idx.shape[-1]
-    _attn_layouts(q, kv, v, idx, d_v, out, lse)
+    _attn_layouts(q, kv, v, idx, d_v, out, lse, paging)
     if out is None:
         out = torch.empty((B, T, Hq, d_v), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
@@ -244,19 +292,29 @@ def dsa_sparse_attn_noalloc(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor
     v_rs = v.stride(1) if v is not None else 0
     v_bs = v.stride(0) if v is not None else 0
     _check("dsa_sparse_attn_noalloc", _lib().dsa_sparse_attn_noalloc(
-        _ptr(q), _ptr(kv), _ptr(v), kv.stride(1), kv.stride(0), v_rs, v_bs, _ptr(idx), B, T, Hq, Dqk, d_v, k,
-        float(sm_scale), _ptr(out), _ptr(lse), _stream(stream)))
+        _ptr(q), _ptr(kv), _ptr(v), kv.stride(1), kv.stride(0), v_rs, v_bs, _cache_rows(kv, v, paging), _ptr(idx),
+        B, T, Hq, Dqk, d_v, k,
+        float(sm_scale), _ptr(out), _ptr(lse), _paging_ref(paging), _stream(stream)))
     return out, lse
 
 
-def dsa_index_pool(k_idx: torch.Tensor, pool: int = 4, k_pool: Optional[torch.Tensor] = None, stream=None):
-    """IndexPool: [B, S, d_I] e4m3 keys -> [B, S/4, d_I] pooled e4m3 keys."""
-    B, S, D = k_idx.shape
-    _layout("k_idx", k_idx, torch.uint8, (B, S, D))
+def dsa_index_pool(k_idx: torch.Tensor, pool: int = 4, k_pool: Optional[torch.Tensor] = None,
+                   paging: Optional[Paging] = None, B: Optional[int] = None, stream=None):
+    """IndexPool: [B, S, d_I] e4m3 keys (or their page pool [num_pages, page_size, d_I] with
+    `paging`, for B sequences) -> [B, S/pool, d_I] pooled e4m3 keys (pool 2, 4 or 8)."""
+    if paging is None:
+        B, S, D = k_idx.shape
+        _layout("k_idx", k_idx, torch.uint8, (B, S, D))
+    else:
+        D = k_idx.shape[2]
+        S = paging.pages_per_seq * paging.page_size
+        B = int(B if B is not None else paging._table.shape[0])
+        _layout("k_idx", k_idx, torch.uint8, (paging.num_pages, paging.page_size, D))
     if k_pool is None:
         k_pool = torch.empty((B, S // pool, D), dtype=torch.uint8, device=k_idx.device)
     _layout("k_pool", k_pool, torch.uint8, (B, S // pool, D))
-    _check("dsa_index_pool", _lib().dsa_index_pool(_ptr(k_idx), B, S, D, pool, _ptr(k_pool), _stream(stream)))
+    _check("dsa_index_pool", _lib().dsa_index_pool(_ptr(k_idx), B, S, D, pool, _ptr(k_pool), _paging_ref(paging),
+                                                   _stream(stream)))
     return k_pool
 
 
@@ -264,23 +322,28 @@ class Group:
     """Marshalled arguments of one IndexShare group (keeps the pointer arrays alive)."""
 
     def __init__(self, q_idx, w, k_idx, ctx_len, topk: int, layers: Sequence[dict], sm_scale: float,
-                 d_v: int, pool: int = 1, idx: Optional[torch.Tensor] = None, want_lse: bool = False):
+                 d_v: int, pool: int = 1, idx: Optional[torch.Tensor] = None, want_lse: bool = False,
+                 paging: Optional[Paging] = None):
         B, T, H, D = q_idx.shape
-        S = k_idx.shape[1]
+        S = k_idx.shape[1] if paging is None else paging.pages_per_seq * paging.page_size
         L = len(layers)
         self.layers = list(layers)
         q0, kv0 = layers[0]["q"], layers[0]["kv"]
         Hq, Dqk = q0.shape[2], q0.shape[3]
         _layout("q_idx", q_idx, torch.uint8, (B, T, H, D))
         _layout("w", w, torch.float32, (B, T, H))
-        _layout("k_idx", k_idx, torch.uint8, (B, S, D))
+        if paging is None:
+            _layout("k_idx", k_idx, torch.uint8, (B, S, D))
+        else:
+            _layout("k_idx", k_idx, torch.uint8, (paging.num_pages, paging.page_size, D))
+            _layout("block_table", paging._table, torch.int32, (B, -1))
         _layout("ctx_len", ctx_len, torch.int32, (B,))
         _layout("idx", idx, torch.int32, (B, T, topk * pool))
         v0 = layers[0].get("v")
         for l, lay in enumerate(self.layers):
             # one set of K/V strides describes every layer's caches
             _attn_layouts(lay["q"], lay["kv"], lay.get("v"), torch.empty((B, T, 0), dtype=torch.int32), d_v,
-                          lay.get("out"), lay.get("lse"))
+                          lay.get("out"), lay.get("lse"), paging)
             if lay["q"].shape != q0.shape or lay["kv"].stride() != kv0.stride():
                 raise ValueError(f"layer {l}: q shape or kv strides differ from layer 0's")
             vl = lay.get("v")
@@ -308,7 +371,9 @@ class Group:
             kv_row_stride=kv0.stride(1), kv_batch_stride=kv0.stride(0),
             v_row_stride=v_any.stride(1) if v_any is not None else 0,
             v_batch_stride=v_any.stride(0) if v_any is not None else 0,
-            Hq=Hq, d_qk=Dqk, d_v=d_v, sm_scale=float(sm_scale), idx=_ptr(self.idx))
+            Hq=Hq, d_qk=Dqk, d_v=d_v, sm_scale=float(sm_scale), idx=_ptr(self.idx),
+            paging=paging if paging is not None else Paging())
+        self._paging = paging
         self.device = q0.device
 
     def workspace_size(self, t_chunk: int) -> int:
@@ -322,10 +387,11 @@ class Group:
 
 def dsa_group_forward(q_idx, w, k_idx, ctx_len, topk: int, layers: Sequence[dict], sm_scale: float, d_v: int,
                       pool: int = 1, t_chunk: Optional[int] = None, ws: Optional[torch.Tensor] = None,
-                      want_lse: bool = False, stream=None):
+                      want_lse: bool = False, paging: Optional[Paging] = None, stream=None):
     """One IndexShare group: indexer + top-k once, then attention for each layer dict
-    {"q", "kv", optional "v", "out", "lse"}.  Returns (idx, [(out, lse) per layer])."""
-    g = Group(q_idx, w, k_idx, ctx_len, topk, layers, sm_scale, d_v, pool, want_lse=want_lse)
+    {"q", "kv", optional "v", "out", "lse"}; with `paging`, k_idx and every layer's kv (and v)
+    are page pools sharing its block table.  Returns (idx, [(out, lse) per layer])."""
+    g = Group(q_idx, w, k_idx, ctx_len, topk, layers, sm_scale, d_v, pool, want_lse=want_lse, paging=paging)
     if ws is None:
         ws = torch.empty(g.workspace_size(t_chunk or q_idx.shape[1]), dtype=torch.uint8, device=g.device)
     return g.forward(ws, stream)

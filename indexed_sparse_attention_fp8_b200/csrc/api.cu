@@ -27,20 +27,55 @@ int num_sms() {
   return cache[dev];
 }
 
+// A dsa_paging (NULL or a NULL table: contiguous caches) whose sequences can hold S rows.
+int check_paging(const dsa_paging* p, int S) {
+  if (p == nullptr || p->block_table == nullptr) return DSA_OK;
+  const int ps = p->page_size;
+  if (ps < 128 || (ps & (ps - 1))) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (p->pages_per_seq < 1 || p->num_pages < 1) return DSA_ERR_INVALID_ARG;
+  if ((int64_t)p->num_pages * ps > (int64_t)INT32_MAX / 2) return DSA_ERR_INVALID_ARG;   // rows fit in int32
+  if ((int64_t)p->pages_per_seq * ps < S) return DSA_ERR_INVALID_ARG;                  // logical capacity
+  return DSA_OK;
+}
+
+// Argument and shape checks of one attention call at `splits` key splits (0 = the default
+// count); nothing is launched.
+int check_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t kv_rs, int64_t kv_bs,
+                      int64_t v_rs, int64_t v_bs, int S_kv, const int32_t* idx, int B, int T, int Hq, int d_qk,
+                      int d_v, int k, const uint16_t* out, const void* ws, size_t ws_bytes, const dsa_paging* paging,
+                      int splits) {
+  if (B < 0 || T < 0 || k < 1 || k > 8192 || S_kv < 1 || splits < 0) return DSA_ERR_INVALID_ARG;
+  if (const int st = check_paging(paging, S_kv)) return st;
+  if (!(Hq == 128 && d_qk == 576 && d_v == 512) && !(Hq == 16 && d_qk == 128 && d_v == 128))
+    return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (Hq == 128 && v != nullptr) return DSA_ERR_UNSUPPORTED_SHAPE;  // MLA: V is part of the K row
+  if (kv_rs < d_qk || kv_bs < 0 || (v && (v_rs < d_v || v_bs < 0))) return DSA_ERR_INVALID_ARG;
+  if (B == 0 || T == 0) return DSA_OK;
+  if (!q || !kv || !idx || !out) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || (v && !aligned16(v)))
+    return DSA_ERR_MISALIGNED;
+  if ((kv_rs & 7) || (kv_bs & 7) || (v && ((v_rs & 7) || (v_bs & 7)))) return DSA_ERR_MISALIGNED;
+  const size_t need = attn_workspace_bytes(B, T, Hq, d_v, k, splits);
+  if (ws_bytes < need) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  if (need > 0 && (!ws || !aligned16(ws))) return ws ? DSA_ERR_MISALIGNED : DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
 namespace {
 
 bool indexer_shape_ok(int H_I, int d_I) { return (H_I == 64 && d_I == 128) || (H_I == 4 && d_I == 64); }
-bool attn_shape_ok(int Hq, int d_qk, int d_v) {
-  return (Hq == 128 && d_qk == 576 && d_v == 512) || (Hq == 16 && d_qk == 128 && d_v == 128);
-}
+// IndexPool factors: 1 (off), the pages' 4, and 2 and 8.
+bool pool_ok(int pool) { return pool == 1 || pool == 2 || pool == 4 || pool == 8; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int check_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                        const int32_t* ctx_len, int B, int T, int S_max, int H_I, int d_I, int pool,
-                       int t_begin, int t_count, const float* scores, int64_t ld) {
+                       int t_begin, int t_count, const float* scores, int64_t ld, const dsa_paging* paging) {
   if (B < 0 || T < 1 || S_max < 1 || t_begin < 0 || t_count < 0 || t_begin + t_count > T)
     return DSA_ERR_INVALID_ARG;
-  if (pool != 1 && pool != 4) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!pool_ok(pool)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (const int st = check_paging(paging, S_max)) return st;
+  if (paging && paging->block_table && pool > 1) return DSA_ERR_UNSUPPORTED_SHAPE;   // pooled keys are contiguous
   if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (ld < S_max || (ld & 3)) return DSA_ERR_INVALID_ARG;
   if (B == 0 || t_count == 0) return DSA_OK;
@@ -53,30 +88,12 @@ int check_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, i
                int pool, int t_begin, int t_count, int k, const int32_t* idx) {
   if (B < 0 || T < 1 || S_max < 1 || t_begin < 0 || t_count < 0 || t_begin + t_count > T)
     return DSA_ERR_INVALID_ARG;
-  if (pool != 1 && pool != 4) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!pool_ok(pool)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (k < 1 || k > 2048) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (ld < S_max || (ld & 3)) return DSA_ERR_INVALID_ARG;
   if (B == 0 || t_count == 0) return DSA_OK;
   if (!scores || !ctx_len || !idx) return DSA_ERR_INVALID_ARG;
   if (!aligned16(scores)) return DSA_ERR_MISALIGNED;
-  return DSA_OK;
-}
-
-int check_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t kv_rs,
-               int64_t kv_bs, int64_t v_rs, int64_t v_bs, const int32_t* idx, int B, int T, int Hq,
-               int d_qk, int d_v, int k, const uint16_t* out, const void* ws, size_t ws_bytes) {
-  if (B < 0 || T < 0 || k < 1 || k > 8192) return DSA_ERR_INVALID_ARG;
-  if (!attn_shape_ok(Hq, d_qk, d_v)) return DSA_ERR_UNSUPPORTED_SHAPE;
-  if (Hq == 128 && v != nullptr) return DSA_ERR_UNSUPPORTED_SHAPE;  // MLA: V is part of the K row
-  if (kv_rs < d_qk || kv_bs < 0 || (v && (v_rs < d_v || v_bs < 0))) return DSA_ERR_INVALID_ARG;
-  if (B == 0 || T == 0) return DSA_OK;
-  if (!q || !kv || !idx || !out) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || (v && !aligned16(v)))
-    return DSA_ERR_MISALIGNED;
-  if ((kv_rs & 7) || (kv_bs & 7) || (v && ((v_rs & 7) || (v_bs & 7)))) return DSA_ERR_MISALIGNED;
-  const size_t need = attn_workspace_bytes(B, T, Hq, d_v, k);
-  if (ws_bytes < need) return DSA_ERR_WORKSPACE_TOO_SMALL;
-  if (need > 0 && (!ws || !aligned16(ws))) return ws ? DSA_ERR_MISALIGNED : DSA_ERR_INVALID_ARG;
   return DSA_OK;
 }
 
@@ -101,21 +118,23 @@ int check_group(const dsa_group_args* a) {
   if (!a) return DSA_ERR_INVALID_ARG;
   if (a->group_size < 1 || a->group_size > 16 || !a->q || !a->kv || !a->out || !a->idx)
     return DSA_ERR_INVALID_ARG;
-  if (a->pool != 1 && a->pool != 4) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!pool_ok(a->pool)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (a->pool > 1 && (a->S_max % a->pool)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (a->topk < 1 || a->topk > 2048) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (a->topk * a->pool > 8192) return DSA_ERR_UNSUPPORTED_SHAPE;
   const int S_eff = a->pool > 1 ? a->S_max / a->pool : a->S_max;
   const int64_t ld = (int64_t)round_up((size_t)S_eff, 4);
   int st = check_index_scores(a->q_idx, a->w, a->k_idx, a->ctx_len, a->B, a->T, S_eff, a->H_I,
-                              a->d_I, a->pool, 0, a->T, reinterpret_cast<const float*>(16), ld);
+                              a->d_I, a->pool, 0, a->T, reinterpret_cast<const float*>(16), ld, nullptr);
   if (st != DSA_OK) return st;
+  if ((st = check_paging(&a->paging, a->S_max)) != DSA_OK) return st;
   // the attention workspace is carved from the group workspace: only shapes are checked here
   for (int l = 0; l < a->group_size; ++l) {
     const uint16_t* v = a->v ? a->v[l] : nullptr;
-    st = check_attn(a->q[l], a->kv[l], v, a->kv_row_stride, a->kv_batch_stride, a->v_row_stride,
-                    a->v_batch_stride, a->idx, a->B, a->T, a->Hq, a->d_qk, a->d_v,
-                    a->topk * a->pool, a->out[l], reinterpret_cast<const void*>(256), (size_t)-1);
+    st = check_sparse_attn(a->q[l], a->kv[l], v, a->kv_row_stride, a->kv_batch_stride, a->v_row_stride,
+                           a->v_batch_stride, a->S_max, a->idx, a->B, a->T, a->Hq, a->d_qk, a->d_v,
+                           a->topk * a->pool, a->out[l], reinterpret_cast<const void*>(256), (size_t)-1,
+                           &a->paging);
     if (st != DSA_OK) return st;
   }
   return DSA_OK;
@@ -137,6 +156,7 @@ const char* dsa_status_string(int status) {
     case DSA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
     case DSA_ERR_CUDA: return "CUDA launch failed";
     case DSA_ERR_TIMEOUT: return "bounded device wait timed out";
+    case DSA_ERR_INDEX_RANGE: return "a selected id was at or beyond the cache length (skipped)";
     default: return "unknown status";
   }
 }
@@ -149,9 +169,11 @@ int dsa_device_status(void* stream) {
     set_cuda_error(e);
     return DSA_ERR_CUDA;
   }
-  const unsigned int a = indexer_take_status();
-  const unsigned int b = attn_tc_take_status();
-  return (a | b) ? DSA_ERR_TIMEOUT : DSA_OK;
+  const unsigned int st =
+      indexer_take_status() | attn_tc_take_status() | attn_mma_take_status() | pool_take_status();
+  if (st & 1u) return DSA_ERR_TIMEOUT;
+  if (st & 2u) return DSA_ERR_INDEX_RANGE;
+  return DSA_OK;
 }
 uint64_t dsa_launch_count(void) { return g_launches; }
 
@@ -162,12 +184,13 @@ int dsa_debug_wait_timeout(uint64_t limit_ns, void* stream) {
 
 int dsa_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                      const int32_t* ctx_len, int B, int T, int S_max, int H_I, int d_I, int pool,
-                     int t_begin, int t_count, float* scores, int64_t ld, void* stream) {
+                     int t_begin, int t_count, float* scores, int64_t ld, const dsa_paging* paging,
+                     void* stream) {
   const int st = check_index_scores(q_idx, w, k_idx, ctx_len, B, T, S_max, H_I, d_I, pool,
-                                    t_begin, t_count, scores, ld);
+                                    t_begin, t_count, scores, ld, paging);
   if (st != DSA_OK || B == 0 || t_count == 0) return st;
   return launch_index_scores(q_idx, w, k_idx, ctx_len, B, T, S_max, H_I, d_I, pool, t_begin,
-                             t_count, scores, ld, static_cast<cudaStream_t>(stream));
+                             t_count, scores, ld, page_map(paging), static_cast<cudaStream_t>(stream));
 }
 
 int dsa_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, int T, int S_max,
@@ -184,26 +207,27 @@ size_t dsa_sparse_attn_workspace_size(int B, int T, int Hq, int d_v, int k) {
 }
 
 int dsa_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t kv_row_stride,
-                    int64_t kv_batch_stride, int64_t v_row_stride, int64_t v_batch_stride,
+                    int64_t kv_batch_stride, int64_t v_row_stride, int64_t v_batch_stride, int S_kv,
                     const int32_t* idx, int B, int T, int Hq, int d_qk, int d_v, int k,
                     float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
-                    void* stream) {
-  const int st = check_attn(q, kv, v, kv_row_stride, kv_batch_stride, v_row_stride,
-                            v_batch_stride, idx, B, T, Hq, d_qk, d_v, k, out, ws, ws_bytes);
+                    const dsa_paging* paging, void* stream) {
+  const int st = check_sparse_attn(q, kv, v, kv_row_stride, kv_batch_stride, v_row_stride,
+                                   v_batch_stride, S_kv, idx, B, T, Hq, d_qk, d_v, k, out, ws, ws_bytes, paging);
   if (st != DSA_OK || B == 0 || T == 0) return st;
   return launch_sparse_attn(q, kv, v, kv_row_stride, kv_batch_stride, v_row_stride, v_batch_stride,
-                            idx, B, T, Hq, d_qk, d_v, k, sm_scale, out, lse, ws,
+                            S_kv, idx, B, T, Hq, d_qk, d_v, k, sm_scale, out, lse, ws, page_map(paging),
                             static_cast<cudaStream_t>(stream));
 }
 
 int dsa_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool, uint8_t* k_pool,
-                   void* stream) {
+                   const dsa_paging* paging, void* stream) {
   if (B < 0 || S_max < 0 || d_I <= 0) return DSA_ERR_INVALID_ARG;
-  if (pool != 4 || (S_max % 4) || (d_I % 16)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (pool == 1 || !pool_ok(pool) || (S_max % pool) || (d_I % 16)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (const int st = check_paging(paging, S_max)) return st;
   if (B == 0 || S_max == 0) return DSA_OK;
   if (!k_idx || !k_pool) return DSA_ERR_INVALID_ARG;
   if (!aligned16(k_idx) || !aligned16(k_pool)) return DSA_ERR_MISALIGNED;
-  return launch_index_pool(k_idx, B, S_max, d_I, k_pool, static_cast<cudaStream_t>(stream));
+  return launch_index_pool(k_idx, B, S_max, d_I, pool, k_pool, page_map(paging), static_cast<cudaStream_t>(stream));
 }
 
 size_t dsa_group_workspace_size(const dsa_group_args* a, int t_chunk) {
@@ -229,17 +253,20 @@ int dsa_group_forward(const dsa_group_args* a, void* ws, size_t ws_bytes, void* 
   void* attn_ws = base + g.pool_bytes;
   float* scores = reinterpret_cast<float*>(base + g.fixed_bytes);
 
+  const PageMap pm = page_map(&a->paging);
   const uint8_t* keys = a->k_idx;
+  PageMap key_pm = pm;   // the indexer reads the paged keys, or the (contiguous) pooled ones
   if (a->pool > 1) {
-    st = launch_index_pool(a->k_idx, a->B, a->S_max, a->d_I, k_pool, s);
+    st = launch_index_pool(a->k_idx, a->B, a->S_max, a->d_I, a->pool, k_pool, pm, s);
     if (st != DSA_OK) return st;
     keys = k_pool;
+    key_pm = PageMap{nullptr, 0, 0, 0};
   }
   // IndexShare: one indexer + one top-k over every query, in chunks that fit the workspace
   for (int t0 = 0; t0 < a->T; t0 += t_chunk) {
     const int tc = std::min(t_chunk, a->T - t0);
     st = launch_index_scores(a->q_idx, a->w, keys, a->ctx_len, a->B, a->T, g.S_eff, a->H_I, a->d_I,
-                             a->pool, t0, tc, scores, g.ld, s);
+                             a->pool, t0, tc, scores, g.ld, key_pm, s);
     if (st != DSA_OK) return st;
     st = launch_topk(scores, g.ld, a->ctx_len, a->B, a->T, g.S_eff, a->pool, t0, tc, a->topk,
                      a->idx, s);
@@ -250,8 +277,8 @@ int dsa_group_forward(const dsa_group_args* a, void* ws, size_t ws_bytes, void* 
     const uint16_t* v = a->v ? a->v[l] : nullptr;
     float* lse = a->lse ? a->lse[l] : nullptr;
     st = launch_sparse_attn(a->q[l], a->kv[l], v, a->kv_row_stride, a->kv_batch_stride,
-                            a->v_row_stride, a->v_batch_stride, a->idx, a->B, a->T, a->Hq, a->d_qk,
-                            a->d_v, a->topk * a->pool, a->sm_scale, a->out[l], lse, attn_ws, s);
+                            a->v_row_stride, a->v_batch_stride, a->S_max, a->idx, a->B, a->T, a->Hq, a->d_qk,
+                            a->d_v, a->topk * a->pool, a->sm_scale, a->out[l], lse, attn_ws, pm, s);
     if (st != DSA_OK) return st;
   }
   return DSA_OK;

@@ -19,6 +19,20 @@ namespace {
 
 constexpr int kTargetCtas = 296;  // 2 x 148 SMs
 
+// Status word of this kernel (bit 1: a selected id at or beyond the cache length was skipped);
+// read and cleared by the host through dsa_device_status().
+__device__ unsigned int g_attn_mma_status;
+
+// A selected id as the gathers use it: ids at or beyond the cache's S_kv rows are skipped like
+// a -1 (nothing outside the cache is read) and flagged in the status word.
+__device__ __forceinline__ int checked_id(int key, int S_kv) {
+  if (key >= S_kv) {
+    atomicOr(&g_attn_mma_status, 2u);
+    return -1;
+  }
+  return key;
+}
+
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
@@ -75,10 +89,10 @@ template <int D_QK, int D_V, int HG, bool LATENT>
 __global__ void __launch_bounds__(Cfg<D_QK, D_V, HG, LATENT>::THREADS, 1)
 sparse_attn_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv,
                        const __nv_bfloat16* __restrict__ vv, int64_t kv_rs, int64_t kv_bs,
-                       int64_t v_rs, int64_t v_bs, const int32_t* __restrict__ idx, int T, int Hq,
+                       int64_t v_rs, int64_t v_bs, int S_kv, const int32_t* __restrict__ idx, int T, int Hq,
                        int k, int keys_per_split, float scale_log2, __nv_bfloat16* __restrict__ out,
                        float* __restrict__ lse, float* __restrict__ part_o,
-                       float* __restrict__ part_lse) {
+                       float* __restrict__ part_lse, PageMap pm) {
   using C = Cfg<D_QK, D_V, HG, LATENT>;
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -97,8 +111,17 @@ sparse_attn_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16*
   const int ntiles = kend > kbeg ? (kend - kbeg + C::KT - 1) / C::KT : 0;
 
   const __nv_bfloat16* qrow = q + ((int64_t)bt * Hq + hg * HG) * D_QK;
-  const __nv_bfloat16* kvb = kv + (int64_t)b * kv_bs;
-  const __nv_bfloat16* vb = LATENT ? kvb : vv + (int64_t)b * v_bs;
+  // contiguous: this sequence's cache rows; paged: rows of the shared page pools
+  const __nv_bfloat16* kvb = pm.bt != nullptr ? kv : kv + (int64_t)b * kv_bs;
+  const __nv_bfloat16* vb = LATENT ? kvb : (pm.bt != nullptr ? vv : vv + (int64_t)b * v_bs);
+  // cache row of a (checked) selected id: itself, or its page's row; -1 stays -1, and an id
+  // whose page id is out of range becomes -1 and is flagged
+  auto cache_row = [&](int key) -> int {
+    if (key < 0 || pm.bt == nullptr) return key;
+    const int r = paged_row(pm, b, key);
+    if (r < 0) atomicOr(&g_attn_mma_status, 2u);
+    return r;
+  };
   const int32_t* irow = idx + (int64_t)bt * k;
 
   // ---- async loads: q once, then one tile of gathered rows per stage
@@ -111,7 +134,7 @@ sparse_attn_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16*
     for (int i = tid; i < C::KT * C::QCH; i += C::THREADS) {
       const int r = i / C::QCH, c = i % C::QCH;
       const int p = p0 + r;
-      const int key = p < kend ? __ldg(irow + p) : -1;
+      const int key = cache_row(p < kend ? checked_id(__ldg(irow + p), S_kv) : -1);
       const __nv_bfloat16* src = kvb + (int64_t)(key < 0 ? 0 : key) * kv_rs + c * 8;
       cp_async16(sbase + C::OFF_K + stage * C::K_TILE + swz(r, c, C::QCH), src, key < 0 ? 0 : 16);
       if (c == 0) idx_s[stage * C::KT + r] = key;
@@ -120,7 +143,7 @@ sparse_attn_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16*
       for (int i = tid; i < C::KT * C::VCH; i += C::THREADS) {
         const int r = i / C::VCH, c = i % C::VCH;
         const int p = p0 + r;
-        const int key = p < kend ? __ldg(irow + p) : -1;
+        const int key = cache_row(p < kend ? checked_id(__ldg(irow + p), S_kv) : -1);
         const __nv_bfloat16* src = vb + (int64_t)(key < 0 ? 0 : key) * v_rs + c * 8;
         cp_async16(sbase + C::OFF_V + stage * C::V_TILE + swz(r, c, C::VCH), src, key < 0 ? 0 : 16);
       }
@@ -324,8 +347,9 @@ namespace {
 
 template <int D_QK, int D_V, int HG, bool LATENT>
 int launch_cfg(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t kv_rs, int64_t kv_bs,
-               int64_t v_rs, int64_t v_bs, const int32_t* idx, int B, int T, int Hq, int k,
-               float sm_scale, uint16_t* out, float* lse, void* ws, cudaStream_t stream) {
+               int64_t v_rs, int64_t v_bs, int S_kv, const int32_t* idx, int B, int T, int Hq, int k,
+               float sm_scale, uint16_t* out, float* lse, void* ws, int splits, const PageMap& pm,
+               cudaStream_t stream) {
   using C = Cfg<D_QK, D_V, HG, LATENT>;
   auto kern = sparse_attn_mma_kernel<D_QK, D_V, HG, LATENT>;
   static bool attr_set[64] = {};  // per device; the attribute is idempotent
@@ -335,7 +359,7 @@ int launch_cfg(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  const int splits = attn_num_splits(B, T, Hq, k);
+  if (splits <= 0) splits = attn_num_splits(B, T, Hq, k);
   int kps = (k + splits - 1) / splits;
   kps = (kps + C::KT - 1) / C::KT * C::KT;
   const int64_t rows = (int64_t)B * T * Hq;
@@ -349,8 +373,8 @@ int launch_cfg(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t
   const float scale_log2 = sm_scale * 1.4426950408889634f;
   kern<<<grid, C::THREADS, C::SMEM, stream>>>(
       reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(kv),
-      reinterpret_cast<const __nv_bfloat16*>(v), kv_rs, kv_bs, v_rs, v_bs, idx, T, Hq, k, kps,
-      scale_log2, reinterpret_cast<__nv_bfloat16*>(out), lse, part_o, part_lse);
+      reinterpret_cast<const __nv_bfloat16*>(v), kv_rs, kv_bs, v_rs, v_bs, S_kv, idx, T, Hq, k, kps,
+      scale_log2, reinterpret_cast<__nv_bfloat16*>(out), lse, part_o, part_lse, pm);
   int st = check_launch();
   if (st != DSA_OK || splits == 1) return st;
   return launch_attn_combine(part_o, part_lse, splits, rows, D_V, out, lse, stream);
@@ -374,31 +398,38 @@ int attn_num_splits(int B, int T, int Hq, int k) {
   return splits;
 }
 
-size_t attn_workspace_bytes(int B, int T, int Hq, int d_v, int k) {
-  const int splits = attn_num_splits(B, T, Hq, k);
+size_t attn_workspace_bytes(int B, int T, int Hq, int d_v, int k, int splits) {
+  if (splits <= 0) splits = attn_num_splits(B, T, Hq, k);
   if (splits == 1) return 0;
   const size_t rows = (size_t)B * T * Hq;
   return (size_t)splits * rows * (size_t)(d_v + 1) * sizeof(float);
 }
 
 int launch_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t kv_rs,
-                       int64_t kv_bs, int64_t v_rs, int64_t v_bs, const int32_t* idx, int B, int T,
+                       int64_t kv_bs, int64_t v_rs, int64_t v_bs, int S_kv, const int32_t* idx, int B, int T,
                        int Hq, int d_qk, int d_v, int k, float sm_scale, uint16_t* out, float* lse,
-                       void* ws, cudaStream_t stream) {
+                       void* ws, const PageMap& pm, cudaStream_t stream, int splits) {
   if (B == 0 || T == 0) return DSA_OK;
   if (Hq == 128 && d_qk == 576 && d_v == 512) {
     // MLA latent form only: V must be the first d_v columns of the K row (tensor-core kernel)
     if (v != nullptr) return DSA_ERR_UNSUPPORTED_SHAPE;
-    return launch_sparse_mla_tc(q, kv, kv_rs, kv_bs, idx, B, T, k, sm_scale, out, lse, ws, stream);
+    return launch_sparse_mla_tc(q, kv, kv_rs, kv_bs, S_kv, idx, B, T, k, sm_scale, out, lse, ws, splits, pm, stream);
   }
   if (Hq == 16 && d_qk == 128 && d_v == 128) {
     if (v == nullptr)
-      return launch_cfg<128, 128, 16, true>(q, kv, v, kv_rs, kv_bs, v_rs, v_bs, idx, B, T, Hq, k,
-                                            sm_scale, out, lse, ws, stream);
-    return launch_cfg<128, 128, 16, false>(q, kv, v, kv_rs, kv_bs, v_rs, v_bs, idx, B, T, Hq, k,
-                                           sm_scale, out, lse, ws, stream);
+      return launch_cfg<128, 128, 16, true>(q, kv, v, kv_rs, kv_bs, v_rs, v_bs, S_kv, idx, B, T, Hq, k,
+                                            sm_scale, out, lse, ws, splits, pm, stream);
+    return launch_cfg<128, 128, 16, false>(q, kv, v, kv_rs, kv_bs, v_rs, v_bs, S_kv, idx, B, T, Hq, k,
+                                           sm_scale, out, lse, ws, splits, pm, stream);
   }
   return DSA_ERR_UNSUPPORTED_SHAPE;
+}
+
+unsigned int attn_mma_take_status() {
+  unsigned int v = 0, zero = 0;
+  cudaMemcpyFromSymbol(&v, g_attn_mma_status, sizeof(v));
+  if (v) cudaMemcpyToSymbol(g_attn_mma_status, &zero, sizeof(zero));
+  return v;
 }
 
 }  // namespace dsa

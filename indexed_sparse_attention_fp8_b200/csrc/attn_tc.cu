@@ -285,9 +285,9 @@ struct Item {
 
 __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(THREADS, 1)
 sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv, int64_t kv_rs,
-                     int64_t kv_bs, const int32_t* __restrict__ idx, int T, int nbt, int items, int k,
+                     int64_t kv_bs, int S_kv, const int32_t* __restrict__ idx, int T, int nbt, int items, int k,
                      int keys_per_split, float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-                     float* __restrict__ part_o, float* __restrict__ part_lse) {
+                     float* __restrict__ part_o, float* __restrict__ part_lse, PageMap pm) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
   const uint32_t sbase = (sraw + 1023u) & ~1023u;
@@ -367,19 +367,38 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     uint32_t g = 0;   // tiles gathered so far
     for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
     const Item I = geom(it);
-    const __nv_bfloat16* kvb = kv + (int64_t)I.b * kv_bs;
+    // contiguous: rows of this sequence's cache; paged: rows of the shared page pool
+    const __nv_bfloat16* kvb = pm.bt != nullptr ? kv : kv + (int64_t)I.b * kv_bs;
     const int32_t* irow = idx + (int64_t)I.bt * k;
-    auto load_id = [&](int j, int r) -> int {
+    // Selected id of slot r of tile j (-1 when empty), and through `row` the cache row to read.
+    // Ids at or beyond the cache's S_kv rows, and ids whose page id is out of range, are
+    // skipped like a -1 (nothing outside the cache is read) and flagged in the status word.
+    auto load_id = [&](int j, int r, int& row) -> int {
       const int p = I.kbeg + j * NK + r;
-      return (j < I.ntiles && p < I.kend) ? __ldg(irow + p) : -1;
+      int id = (j < I.ntiles && p < I.kend) ? __ldg(irow + p) : -1;
+      if (id >= S_kv) {
+        atomicOr(&g_status, 2u);
+        id = -1;
+      }
+      row = id;
+      if (id >= 0 && pm.bt != nullptr) {
+        row = paged_row(pm, I.b, id);
+        if (row < 0) {
+          atomicOr(&g_status, 2u);
+          id = -1;
+        }
+      }
+      return id;
     };
-    int id_next0 = load_id(0, lane), id_next1 = load_id(0, lane + 32);
+    int row_next0, row_next1;
+    int id_next0 = load_id(0, lane, row_next0), id_next1 = load_id(0, lane + 32, row_next1);
     for (int j = 0; j < I.ntiles; ++j, ++g) {
       const int st = g % NS;
       const int id0 = id_next0, id1 = id_next1;
-      id_next0 = load_id(j + 1, lane);
-      id_next1 = load_id(j + 1, lane + 32);
-      if (!(ok = mbar_wait(kv_empty(st), ((g / NS) & 1) ^ 1, abort, kWaitLimitNs))) break;
+      const int row0 = row_next0, row1 = row_next1;
+      id_next0 = load_id(j + 1, lane, row_next0);
+      id_next1 = load_id(j + 1, lane + 32, row_next1);
+      if (!(ok = mbar_wait_warp(kv_empty(st), ((g / NS) & 1) ^ 1, abort, kWaitLimitNs))) break;
       if (gw == 0) {
         ids_s[st * NK + lane] = id0;
         ids_s[st * NK + 32 + lane] = id1;
@@ -392,7 +411,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
 #pragma unroll 4
       for (int r = gw; r < NK; r += 3) {
         const int key = __shfl_sync(0xffffffffu, r < 32 ? id0 : id1, r & 31);
-        const __nv_bfloat16* src = kvb + (int64_t)(key < 0 ? 0 : key) * kv_rs;
+        const int crow = __shfl_sync(0xffffffffu, r < 32 ? row0 : row1, r & 31);
+        const __nv_bfloat16* src = kvb + (int64_t)(key < 0 ? 0 : crow) * kv_rs;
         const int nbytes = key < 0 ? 0 : 16;
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
@@ -416,8 +436,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     const int ks0 = half * KSTEPS;
     auto issue_s = [&](uint32_t gg) -> bool {
       const int st = gg % NS;
-      if (!mbar_wait(kv_full(st), (gg / NS) & 1, abort, kWaitLimitNs)) return false;
-      if (!mbar_wait(s_empty, (gg & 1) ^ 1, abort, kWaitLimitNs)) return false;
+      if (!mbar_wait_warp(kv_full(st), (gg / NS) & 1, abort, kWaitLimitNs)) return false;
+      if (!mbar_wait_warp(s_empty, (gg & 1) ^ 1, abort, kWaitLimitNs)) return false;
       tc_fence_after();
       fence_proxy_async();
       if (lane == 0) {
@@ -436,7 +456,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       return true;
     };
     auto issue_pv = [&](uint32_t gg, bool first) -> bool {
-      if (!mbar_wait(p_full, gg & 1, abort, kWaitLimitNs)) return false;
+      if (!mbar_wait_warp(p_full, gg & 1, abort, kWaitLimitNs)) return false;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t stage = sbase + OFF_KV + (gg % NS) * KV_STAGE;
@@ -456,7 +476,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
       const Item I = geom(it);
       if (I.ntiles == 0) continue;
-      if (!(ok = mbar_wait(q_ready, nq & 1, abort, kWaitLimitNs))) break;   // this item's q is in TMEM
+      if (!(ok = mbar_wait_warp(q_ready, nq & 1, abort, kWaitLimitNs))) break;   // this item's q is in TMEM
       ++nq;
       ok = issue_s(g);
       if (ok && I.ntiles > 1) ok = issue_s(g + 1);
@@ -477,7 +497,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     // jj&1: staged locally, one 8 KB bulk copy that completes the partner's per-warp barrier.
     // Sent one tile ahead, so the copy is in flight while the current tile is finished.
     auto load_send = [&](uint32_t jj, float (&sv)[NK]) -> bool {
-      if (!mbar_wait(s_full, jj & 1, abort, kWaitLimitNs)) return false;
+      if (!mbar_wait_warp(s_full, jj & 1, abort, kWaitLimitNs)) return false;
       tc_fence_after();
       tmem_ld32(tmem + lane_off + COL_S, *reinterpret_cast<float(*)[32]>(sv));
       tmem_ld32(tmem + lane_off + COL_S + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
@@ -514,7 +534,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     // Tile jj, first half: the partner's partial + ours -> masked scores and their max.
     auto part1 = [&](uint32_t jj, float (&sv)[NK], float& mt) -> bool {
       const int st = jj % NS;
-      if (!mbar_wait_cluster(x_full(warp), jj & 1, abort)) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait_cluster(x_full(warp), jj & 1, abort))) return false;
       {
         // both CTAs add the partials in column order (0..287 first): the same scores in both
         const uint32_t xrow = sbase + OFF_X + row * 256;
@@ -532,7 +552,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_expect_tx(x_full(warp), X_BYTES / 4);   // arm the next exchange
-      if (!mbar_wait(ids_ready(st), (jj / NS) & 1, abort, kWaitLimitNs)) return false;
+      if (!mbar_wait_warp(ids_ready(st), (jj / NS) & 1, abort, kWaitLimitNs)) return false;
       {   // tile max in the log2 domain (scaled)
         const bool all_valid = ids_s[NS * NK + 4 * st] != 0;
         if (!all_valid) {
@@ -565,7 +585,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     auto part2 = [&](uint32_t jj, int j, float (&sv)[NK], float mt) -> bool {
       // P.V of tile jj-1 has finished: the P columns are free and O holds the item's tiles < j
       if (jj >= 1) {
-        if (!mbar_wait(pv_done, (jj - 1) & 1, abort, kWaitLimitNs)) return false;
+        if (!mbar_wait_warp(pv_done, (jj - 1) & 1, abort, kWaitLimitNs)) return false;
         tc_fence_after();
       }
       // Lazy rescale, decided for the whole warp: the O round trip through TMEM is a
@@ -671,9 +691,9 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
 
 }  // namespace
 
-int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, int64_t kv_bs, const int32_t* idx,
-                         int B, int T, int k, float sm_scale, uint16_t* out, float* lse, void* ws,
-                         cudaStream_t stream) {
+int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, int64_t kv_bs, int S_kv,
+                         const int32_t* idx, int B, int T, int k, float sm_scale, uint16_t* out, float* lse,
+                         void* ws, int splits, const PageMap& pm, cudaStream_t stream) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -681,7 +701,7 @@ int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, i
     cudaFuncSetAttribute(sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  const int splits = attn_num_splits(B, T, HQ, k);
+  if (splits <= 0) splits = attn_num_splits(B, T, HQ, k);
   int kps = (k + splits - 1) / splits;
   kps = (kps + NK - 1) / NK * NK;
   const int64_t rows = (int64_t)B * T * HQ;
@@ -697,8 +717,8 @@ int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, i
   const int nclu = std::max(1, std::min(items, num_sms() / 2));
   dim3 grid((unsigned)nclu, 2, 1);
   sparse_mla_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(
-      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(kv), kv_rs, kv_bs, idx, T, nbt,
-      items, k, kps, sm_scale * 1.4426950408889634f, reinterpret_cast<__nv_bfloat16*>(out), lse, part_o, part_lse);
+      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(kv), kv_rs, kv_bs, S_kv, idx, T, nbt,
+      items, k, kps, sm_scale * 1.4426950408889634f, reinterpret_cast<__nv_bfloat16*>(out), lse, part_o, part_lse, pm);
   int st = check_launch();
   if (st != DSA_OK || splits == 1) return st;
   return launch_attn_combine(part_o, part_lse, splits, rows, DV, out, lse, stream);

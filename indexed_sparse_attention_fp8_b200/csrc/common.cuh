@@ -30,6 +30,33 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 int num_sms();  // SM count of the current device (cached per device)
 
+// Page map of a paged cache (dsa_paging in dsa.h); bt == nullptr means the cache is contiguous
+// per sequence.  Passed to kernels by value.
+struct PageMap {
+  const int32_t* bt;   // device [B, pps] page ids
+  int shift;           // log2(page_size)
+  int pps;             // pages per sequence
+  int num_pages;       // pages in the pool
+};
+
+inline PageMap page_map(const dsa_paging* p) {
+  PageMap m{nullptr, 0, 0, 0};
+  if (p != nullptr && p->block_table != nullptr) {
+    m.bt = p->block_table;
+    while ((1 << m.shift) < p->page_size) ++m.shift;
+    m.pps = p->pages_per_seq;
+    m.num_pages = p->num_pages;
+  }
+  return m;
+}
+
+// Physical row of logical row s of sequence b in a paged pool, or -1 when the page id in the
+// block table lies outside [0, num_pages).
+__device__ __forceinline__ int paged_row(const PageMap& m, int b, int s) {
+  const int page = __ldg(m.bt + (int64_t)b * m.pps + (s >> m.shift));
+  return (page >= 0 && page < m.num_pages) ? (page << m.shift) | (s & ((1 << m.shift) - 1)) : -1;
+}
+
 // ---------------------------------------------------------------- device helpers
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -91,7 +91,7 @@ template <int H, int D, int QB>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                        const float* __restrict__ w, const int32_t* __restrict__ ctx_len, int B, int T, int S_max,
-                       int pool, int t_begin, int t_count, float* __restrict__ scores, int64_t ld) {
+                       int pool, int t_begin, int t_count, float* __restrict__ scores, int64_t ld, PageMap pm) {
   using C = IdxCfg<H, D, QB>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
@@ -147,7 +147,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       ItemGeom g;
       if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g)) continue;
       const int bs = b_cnt & 1;
-      if (!(ok = mbar_wait(b_empty(bs), ((b_cnt >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
+      if (!(ok = mbar_wait_warp(b_empty(bs), ((b_cnt >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
       if (lane == 0) {
         const uint32_t wbytes = (uint32_t)(g.nq * H * 4);
         mbar_arrive_expect_tx(b_full(bs), C::B_BYTES + wbytes);
@@ -157,10 +157,20 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       ++b_cnt;
       for (int kt = g.kt0; kt < g.kt1; ++kt) {
         const int as = a_cnt % NA;
-        if (!(ok = mbar_wait(a_empty(as), ((a_cnt / NA) & 1) ^ 1, abort, kWaitLimitNs))) break;
+        if (!(ok = mbar_wait_warp(a_empty(as), ((a_cnt / NA) & 1) ^ 1, abort, kWaitLimitNs))) break;
         if (lane == 0) {
+          // contiguous: row b*S_max + s of the cache; paged: the tile's page (a tile never
+          // straddles one); a bad page id loads past the map's extent, which reads zeros
+          int y = g.b * S_max + kt * KTILE;
+          if (pm.bt != nullptr) {
+            y = paged_row(pm, g.b, kt * KTILE);
+            if (y < 0) {
+              atomicOr(&g_status, 2u);
+              y = pm.num_pages << pm.shift;
+            }
+          }
           mbar_arrive_expect_tx(a_full(as), C::A_BYTES);
-          tma_load_2d(sbase + C::OFF_A + as * C::A_BYTES, &tmap_k, a_full(as), 0, g.b * S_max + kt * KTILE);
+          tma_load_2d(sbase + C::OFF_A + as * C::A_BYTES, &tmap_k, a_full(as), 0, y);
         }
         ++a_cnt;
       }
@@ -180,13 +190,13 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       ItemGeom g;
       if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g)) continue;
       const int bs = b_cnt & 1;
-      if (!(ok = mbar_wait(b_full(bs), (b_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
+      if (!(ok = mbar_wait_warp(b_full(bs), (b_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
       const uint32_t b_addr = sbase + C::OFF_B + bs * C::B_BYTES;
       for (int kt = g.kt0; kt < g.kt1; ++kt) {
         const int as = a_cnt % NA;
         const int ab = acc_cnt & 1;
-        if (!(ok = mbar_wait(a_full(as), (a_cnt / NA) & 1, abort, kWaitLimitNs))) break;
-        if (!(ok = mbar_wait(acc_empty(ab), ((acc_cnt >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
+        if (!(ok = mbar_wait_warp(a_full(as), (a_cnt / NA) & 1, abort, kWaitLimitNs))) break;
+        if (!(ok = mbar_wait_warp(acc_empty(ab), ((acc_cnt >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
         tc_fence_after();
         if (lane == 0) {
           const uint32_t a_addr = sbase + C::OFF_A + as * C::A_BYTES;
@@ -221,7 +231,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       ItemGeom g;
       if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g)) continue;
       const int bs = b_cnt & 1;
-      if (!(ok = mbar_wait(b_full(bs), (b_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
+      if (!(ok = mbar_wait_warp(b_full(bs), (b_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
       const float* wsm = reinterpret_cast<const float*>(sgen + C::OFF_W + bs * C::W_BYTES) + half * C::COLS;
       const int ctx_b = __ldg(ctx_len + g.b);
       // H == 64: the 16x256b TMEM shape gives each thread 2 keys x 2 heads per 8-column group,
@@ -266,7 +276,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
           if (qok[ql] && s < S_max) qrow[ql][s] = (s <= lim[ql]) ? val : -INFINITY;
         };
         if (g.kt0 < g.kt1) {
-          if (!(ok = mbar_wait(acc_full(acc_cnt & 1), (acc_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
+          if (!(ok = mbar_wait_warp(acc_full(acc_cnt & 1), (acc_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
           tc_fence_after();
           issue(acc_cnt & 1, 0, v[0]);
           tmem_ld_wait();
@@ -286,7 +296,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
               __syncwarp();
               if (lane == 0) mbar_arrive(acc_empty(ab));
               if (more) {
-                if (!(ok = mbar_wait(acc_full(ab ^ 1), ((acc_cnt + 1) >> 1) & 1, abort, kWaitLimitNs))) break;
+                if (!(ok = mbar_wait_warp(acc_full(ab ^ 1), ((acc_cnt + 1) >> 1) & 1, abort, kWaitLimitNs))) break;
                 tc_fence_after();
                 issue(ab ^ 1, 0, v[0]);
               }
@@ -338,7 +348,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       } else {
       for (int kt = g.kt0; kt < g.kt1; ++kt) {
         const int ab = acc_cnt & 1;
-        if (!(ok = mbar_wait(acc_full(ab), (acc_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
+        if (!(ok = mbar_wait_warp(acc_full(ab), (acc_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
         tc_fence_after();
         // finished sum of query ql (local to this warp) for key s -> masked store
         auto store = [&](int ql, int s, float val) {
@@ -434,10 +444,12 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t row_byte
 
 template <int H, int D, int QB>
 int launch_tc(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* ctx_len, int B, int T,
-              int S_max, int pool, int t_begin, int t_count, float* scores, int64_t ld, cudaStream_t stream) {
+              int S_max, int pool, int t_begin, int t_count, float* scores, int64_t ld, const PageMap& pm,
+              cudaStream_t stream) {
   using C = IdxCfg<H, D, QB>;
   CUtensorMap mk, mq;
-  if (!make_map(&mk, k_idx, (uint64_t)B * S_max, D, KTILE)) return DSA_ERR_CUDA;
+  const uint64_t key_rows = pm.bt != nullptr ? ((uint64_t)pm.num_pages << pm.shift) : (uint64_t)B * S_max;
+  if (!make_map(&mk, k_idx, key_rows, D, KTILE)) return DSA_ERR_CUDA;
   if (!make_map(&mq, q_idx, (uint64_t)B * T * H, D, C::N)) return DSA_ERR_CUDA;
   auto kern = index_scores_tc_kernel<H, D, QB>;
   static bool attr_set[64] = {};
@@ -451,7 +463,8 @@ int launch_tc(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const 
   const int nkc = ((S_max + KTILE - 1) / KTILE + KC - 1) / KC;
   const int64_t items = (int64_t)B * nqb * nkc;
   const int grid = (int)std::min<int64_t>(items, num_sms());
-  kern<<<grid, NUM_THREADS, C::SMEM, stream>>>(mk, mq, w, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld);
+  kern<<<grid, NUM_THREADS, C::SMEM, stream>>>(mk, mq, w, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld,
+                                               pm);
   return check_launch();
 }
 
@@ -459,15 +472,17 @@ int launch_tc(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const 
 
 int launch_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* ctx_len, int B,
                         int T, int S_max, int H_I, int d_I, int pool, int t_begin, int t_count, float* scores,
-                        int64_t ld, cudaStream_t stream) {
+                        int64_t ld, const PageMap& pm, cudaStream_t stream) {
   if (B == 0 || t_count == 0 || S_max == 0) return DSA_OK;
   if (H_I == 64 && d_I == 128) {
     if (t_count < 4)  // decode-like: one query per block keeps the MMA N at the head count
-      return launch_tc<64, 128, 1>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, stream);
-    return launch_tc<64, 128, 4>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, stream);
+      return launch_tc<64, 128, 1>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, pm,
+                                   stream);
+    return launch_tc<64, 128, 4>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, pm,
+                                 stream);
   }
   if (H_I == 4 && d_I == 64)
-    return launch_tc<4, 64, 64>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, stream);
+    return launch_tc<4, 64, 64>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, pm, stream);
   return DSA_ERR_UNSUPPORTED_SHAPE;
 }
 

@@ -4,23 +4,40 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "common.cuh"
+
 namespace dsa {
 
 int launch_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                         const int32_t* ctx_len, int B, int T, int S_max, int H_I, int d_I, int pool,
-                        int t_begin, int t_count, float* scores, int64_t ld, cudaStream_t stream);
+                        int t_begin, int t_count, float* scores, int64_t ld, const PageMap& pm,
+                        cudaStream_t stream);
 
 int launch_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, int T, int S_max,
                 int pool, int t_begin, int t_count, int k, int32_t* idx, cudaStream_t stream);
 
-// Split count the attention uses for a problem (1 = no split, no workspace).
+// Split count the attention uses for a problem by default (1 = no split, no workspace).
 int attn_num_splits(int B, int T, int Hq, int k);
-size_t attn_workspace_bytes(int B, int T, int Hq, int d_v, int k);
+// Workspace of the attention at `splits` key splits (0 = the default count).
+size_t attn_workspace_bytes(int B, int T, int Hq, int d_v, int k, int splits = 0);
+// Argument and shape checks of dsa_sparse_attn at `splits` key splits (0 = default), without
+// launching anything; the same status dsa_sparse_attn would return before its first launch.
+int check_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t kv_rs,
+                      int64_t kv_bs, int64_t v_rs, int64_t v_bs, int S_kv, const int32_t* idx, int B,
+                      int T, int Hq, int d_qk, int d_v, int k, const uint16_t* out, const void* ws,
+                      size_t ws_bytes, const dsa_paging* paging, int splits = 0);
+// Checks of a dsa_paging (NULL is valid); S is the logical rows the call needs per sequence.
+int check_paging(const dsa_paging* paging, int S);
+// Selected ids >= S_kv are skipped on the device (and flagged in the status word).
 int launch_sparse_attn(const uint16_t* q, const uint16_t* kv, const uint16_t* v,
                        int64_t kv_row_stride, int64_t kv_batch_stride, int64_t v_row_stride,
-                       int64_t v_batch_stride, const int32_t* idx, int B, int T, int Hq, int d_qk,
-                       int d_v, int k, float sm_scale, uint16_t* out, float* lse, void* ws,
-                       cudaStream_t stream);
+                       int64_t v_batch_stride, int S_kv, const int32_t* idx, int B, int T, int Hq,
+                       int d_qk, int d_v, int k, float sm_scale, uint16_t* out, float* lse, void* ws,
+                       const PageMap& pm, cudaStream_t stream, int splits = 0);
+// Reads and clears the status word of the mma.sync attention (bit 1: an id >= S_kv).
+unsigned int attn_mma_take_status();
+// Reads and clears the status word of the pool kernel (bit 1: a page id out of range).
+unsigned int pool_take_status();
 
 // Reads and clears the device status word of the tensor-core indexer.
 unsigned int indexer_take_status();
@@ -28,15 +45,16 @@ unsigned int indexer_take_status();
 int launch_wait_timeout_probe(uint64_t limit_ns, cudaStream_t stream);
 
 // Tensor-core sparse MLA attention (128 heads, latent 576 / V 512); same split rule.
-int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, int64_t kv_bs, const int32_t* idx,
-                         int B, int T, int k, float sm_scale, uint16_t* out, float* lse, void* ws,
-                         cudaStream_t stream);
+int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, int64_t kv_bs, int S_kv,
+                         const int32_t* idx, int B, int T, int k, float sm_scale, uint16_t* out, float* lse,
+                         void* ws, int splits, const PageMap& pm, cudaStream_t stream);
 unsigned int attn_tc_take_status();
 // Merges split-key attention partials (normalised fp32 O and log-sum-exp per split).
 int launch_attn_combine(const float* part_o, const float* part_lse, int splits, int64_t rows, int d_v,
                         uint16_t* out, float* lse, cudaStream_t stream);
 
-int launch_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, uint8_t* k_pool,
-                      cudaStream_t stream);
+// IndexPool over `pool` (2, 4 or 8) consecutive keys.
+int launch_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool, uint8_t* k_pool,
+                      const PageMap& pm, cudaStream_t stream);
 
 }  // namespace dsa

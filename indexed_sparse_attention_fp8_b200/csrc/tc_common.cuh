@@ -13,8 +13,9 @@ namespace dsa {
 namespace tc {
 
 // ---------------------------------------------------------------- device status word
-// Set (bit 0) by any kernel whose bounded wait gave up; read and cleared by the host
-// through dsa_device_status().  One word per translation unit that includes this header.
+// Set by the kernels and read and cleared by the host through dsa_device_status(): bit 0 when
+// a bounded wait gave up, bit 1 when an attention gather met an id at or beyond the cache
+// length.  One word per translation unit that includes this header.
 static __device__ unsigned int g_status;
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -80,6 +81,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       }
     }
   }
+}
+
+// mbar_wait taken by every lane of a warp, with the result made warp-uniform: if any lane gave
+// up, the whole warp treats the wait as failed, so no lane goes on alone into the warp-collective
+// tcgen05, shuffle or .sync.aligned operations that follow a successful wait.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               uint64_t limit_ns) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, limit_ns));
 }
 
 // Bounded wait used while draining after an abort: gives up silently after limit_ns.

@@ -16,6 +16,7 @@ Workloads (all on one GPU, synthetic data, no trained weights):
   decode256k  : 32 seqs x 1 new token, each with a 262144-token cache; shapes as prefill32k.
   chunk1m : 8192 new queries at the end of a 1,048,576-token cache; shapes as prefill32k;
             plus the IndexPool variant (pool 4 keys, top-512 blocks -> 2048 tokens).
+  decode256k_pool : decode256k with IndexPool (pool 4 keys, top-512 blocks -> 2048 tokens).
 
 Value distributions: indexer q/k = e4m3(N(0,1)*0.5) (round-to-nearest-even, no scale),
 w = N(0,1)/2 (tiny) or N(0,1)/8 (others) in fp32, attention q/K/V = bf16(N(0,1)).
@@ -81,6 +82,9 @@ WORKLOADS: Dict[str, Workload] = {
 }
 # IndexPool variant of the 1M chunked prefill: 4 keys pooled into one, top-512 blocks.
 WORKLOADS["chunk1m_pool"] = WORKLOADS["chunk1m"].replace(name="chunk1m_pool", pool=4, topk=512)
+# IndexPool at decode: the 32 x 256K decode batch with 4 keys pooled into one, top-512 blocks
+# (2048 tokens), so the decode indexer reads a quarter of the keys.
+WORKLOADS["decode256k_pool"] = WORKLOADS["decode256k"].replace(name="decode256k_pool", pool=4, topk=512)
 
 # Tensor ids for the per-tensor generators.
 _TID = {"q_idx": 1, "w": 2, "k_idx": 3, "q": 4, "kv": 5, "v": 6, "plant": 7}

@@ -53,15 +53,16 @@ def test_status_strings(lib):
 
 def test_index_scores_validation(lib):
     f = lib.dsa_index_scores
-    good = dict(q=A, w=A, k=A, c=A, B=1, T=8, S=8, H=64, D=128, pool=1, tb=0, tc=8, sc=A, ld=8)
+    good = dict(q=A, w=A, k=A, c=A, B=1, T=8, S=8, H=64, D=128, pool=1, tb=0, tc=8, sc=A, ld=8, pg=None)
 
     def call(**kw):
         a = {**good, **kw}
         return f(a["q"], a["w"], a["k"], a["c"], a["B"], a["T"], a["S"], a["H"], a["D"], a["pool"], a["tb"], a["tc"],
-                 a["sc"], a["ld"], None)
+                 a["sc"], a["ld"], a["pg"], None)
     assert call(H=8) == UNSUPPORTED
     assert call(H=64, D=64) == UNSUPPORTED
-    assert call(pool=2) == UNSUPPORTED
+    assert call(pool=3) == UNSUPPORTED
+    assert call(pool=16) == UNSUPPORTED
     assert call(tb=4, tc=5) == INVALID
     assert call(ld=6) == INVALID            # ld not a multiple of 4
     assert call(ld=4) == INVALID            # ld < S_max
@@ -83,8 +84,8 @@ def test_topk_validation(lib):
 def test_sparse_attn_validation(lib):
     f = lib.dsa_sparse_attn
 
-    def call(Hq=128, dqk=576, dv=512, v=None, kv_rs=576, k=2048, B=1, T=4, ws=None, wsb=0, q=A):
-        return f(q, A, v, kv_rs, 576 * 64, 0, 0, A, B, T, Hq, dqk, dv, k, 0.04, A, None, ws, wsb, None)
+    def call(Hq=128, dqk=576, dv=512, v=None, kv_rs=576, k=2048, B=1, T=4, ws=None, wsb=0, q=A, S_kv=64, pg=None):
+        return f(q, A, v, kv_rs, 576 * 64, 0, 0, S_kv, A, B, T, Hq, dqk, dv, k, 0.04, A, None, ws, wsb, pg, None)
     assert call(Hq=64) == UNSUPPORTED
     assert call(dqk=512) == UNSUPPORTED
     assert call(v=A) == UNSUPPORTED         # MLA shapes read V from the latent row
@@ -92,6 +93,7 @@ def test_sparse_attn_validation(lib):
     assert call(kv_rs=580) == MISALIGNED    # row stride not a multiple of 16 bytes
     assert call(q=A + 2) == MISALIGNED
     assert call(k=0) == INVALID
+    assert call(S_kv=0) == INVALID           # the cache length bounds every selected id
     # decode-shaped problems split the keys and need a workspace
     need = lib.dsa_sparse_attn_workspace_size(32, 1, 128, 512, 2048)
     assert need > 0
@@ -100,13 +102,31 @@ def test_sparse_attn_validation(lib):
     assert lib.dsa_sparse_attn_workspace_size(1, 32768, 128, 512, 2048) == 0
 
 
+def test_noalloc_validation_matches_workspace_entry(lib):
+    """The workspace-free entry point checks arguments exactly as dsa_sparse_attn does, before
+    looking at its scratch: a bad shape or pointer reports the same status there."""
+    f, g = lib.dsa_sparse_attn_noalloc, lib.dsa_sparse_attn
+
+    def both(Hq=128, dqk=576, dv=512, v=None, kv_rs=576, k=2048, B=32, T=1, q=A, S_kv=64):
+        a = f(q, A, v, kv_rs, 576 * 64, 0, 0, S_kv, A, B, T, Hq, dqk, dv, k, 0.04, A, None, None, None)
+        ws_need = lib.dsa_sparse_attn_workspace_size(max(B, 1), max(T, 1), Hq, dv, k) if Hq in (16, 128) else 0
+        b = g(q, A, v, kv_rs, 576 * 64, 0, 0, S_kv, A, B, T, Hq, dqk, dv, k, 0.04, A, None, A, ws_need, None, None)
+        return a, b
+    for kw, want in [({"v": A}, UNSUPPORTED), ({"Hq": 64}, UNSUPPORTED), ({"kv_rs": 500}, INVALID),
+                     ({"kv_rs": 580}, MISALIGNED), ({"q": A + 2}, MISALIGNED), ({"k": 0}, INVALID),
+                     ({"S_kv": 0}, INVALID), ({"B": -1}, INVALID), ({"B": 0}, OK)]:
+        assert both(**kw) == (want, want), kw
+
+
 def test_index_pool_validation(lib):
     f = lib.dsa_index_pool
-    assert f(A, 1, 10, 128, 4, A, None) == UNSUPPORTED    # S not a multiple of 4
-    assert f(A, 1, 16, 128, 2, A, None) == UNSUPPORTED
-    assert f(A, 1, 16, 24, 4, A, None) == UNSUPPORTED     # d_I not a multiple of 16
-    assert f(A + 1, 1, 16, 128, 4, A, None) == MISALIGNED
-    assert f(A, 0, 16, 128, 4, A, None) == OK
+    assert f(A, 1, 10, 128, 4, A, None, None) == UNSUPPORTED    # S not a multiple of 4
+    assert f(A, 1, 16, 128, 3, A, None, None) == UNSUPPORTED    # pool factors are 2, 4 and 8
+    assert f(A, 1, 16, 128, 1, A, None, None) == UNSUPPORTED
+    assert f(A, 1, 12, 128, 8, A, None, None) == UNSUPPORTED    # S not a multiple of 8
+    assert f(A, 1, 16, 24, 4, A, None, None) == UNSUPPORTED     # d_I not a multiple of 16
+    assert f(A + 1, 1, 16, 128, 4, A, None, None) == MISALIGNED
+    assert f(A, 0, 16, 128, 4, A, None, None) == OK
 
 
 def _group_args(pool=1, topk=2048, S=32768, T=32768, B=1, group=4, d_I=128, H_I=64):
@@ -116,6 +136,32 @@ def _group_args(pool=1, topk=2048, S=32768, T=32768, B=1, group=4, d_I=128, H_I=
                          pool=pool, group_size=group, q=arr, kv=arr, v=None, out=arr, lse=None,
                          kv_row_stride=576, kv_batch_stride=576 * S, v_row_stride=0, v_batch_stride=0,
                          Hq=128, d_qk=576, d_v=512, sm_scale=0.04, idx=A), arr
+
+
+def test_paging_validation(lib):
+    """A page map is checked before anything is launched: page sizes are powers of two >= 128,
+    the table covers the rows the call needs, and pooled indexer keys are never paged."""
+    def pg(page_size=256, pps=4, num_pages=16, table=A):
+        return ctypes.byref(dsa.Paging(block_table=table, page_size=page_size, pages_per_seq=pps, num_pages=num_pages))
+    f = lib.dsa_sparse_attn
+
+    def attn(p, S_kv=1024):
+        return f(A, A, None, 576, 0, 0, 0, S_kv, A, 1, 4, 128, 576, 512, 2048, 0.04, A, None, None, 0, p, None)
+    assert attn(pg(page_size=192)) == UNSUPPORTED            # not a power of two
+    assert attn(pg(page_size=64)) == UNSUPPORTED             # below one indexer tile
+    assert attn(pg(pps=0)) == INVALID
+    assert attn(pg(num_pages=0)) == INVALID
+    assert attn(pg(pps=3)) == INVALID                        # 3 x 256 rows < S_kv = 1024
+    assert attn(pg(num_pages=1 << 30)) == INVALID            # pool rows beyond int32
+    assert attn(pg(), S_kv=0) == INVALID
+    g = lib.dsa_index_scores
+    assert g(A, A, A, A, 1, 8, 1024, 64, 128, 4, 0, 8, A, 1024, pg(), None) == UNSUPPORTED   # pooled keys
+    assert g(A, A, A, A, 1, 8, 2048, 64, 128, 1, 0, 8, A, 2048, pg(), None) == INVALID      # table too short
+    assert lib.dsa_index_pool(A, 1, 2048, 128, 4, A, pg(), None) == INVALID
+    assert lib.dsa_index_pool(A, 1, 1024, 128, 4, A, pg(page_size=100), None) == UNSUPPORTED
+    bad, keep = _group_args(S=4096, T=4096)
+    bad.paging = dsa.Paging(block_table=A, page_size=256, pages_per_seq=8, num_pages=64)   # 2048 < 4096 rows
+    assert lib.dsa_group_forward(ctypes.byref(bad), A, 1 << 40, None) == INVALID
 
 
 def test_group_workspace_and_validation(lib):

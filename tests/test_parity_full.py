@@ -41,7 +41,7 @@ def _sample_rows(wl, n_random=3):
 
 def _check(wl, ind, lays, idx, outs, rows):
     kdec = P.Decoded(ind["k_idx"])
-    kp = dsa.dsa_index_pool(ind["k_idx"]) if wl.pool > 1 else None
+    kp = dsa.dsa_index_pool(ind["k_idx"], pool=wl.pool) if wl.pool > 1 else None
     kpdec = P.Decoded(kp) if kp is not None else None
     idx_h = P.to_np(idx)
     for (b, t) in rows:
@@ -79,7 +79,7 @@ def _run(name):
     _check(wl, ind, lays, idx, outs, _sample_rows(wl))
 
 
-@pytest.mark.parametrize("name", ["prefill32k", "prefill128k", "decode256k", "chunk1m", "chunk1m_pool"])
+@pytest.mark.parametrize("name", ["prefill32k", "prefill128k", "decode256k", "decode256k_pool", "chunk1m", "chunk1m_pool"])
 def test_full_size_group_sampled_rows(name):
     _run(name)
 

@@ -48,7 +48,7 @@ def _check_rows(wl, ind, lays, idx, outs, rows, ctx_len=None, check_scores=True)
     kdec = P.Decoded(ind["k_idx"])
     kpool_dec = None
     if wl.pool > 1:
-        kpool_dec = P.Decoded(dsa.dsa_index_pool(ind["k_idx"]))
+        kpool_dec = P.Decoded(dsa.dsa_index_pool(ind["k_idx"], pool=wl.pool))
     idx_h = P.to_np(idx)
     nfloor_total = 0
     by_b = {}
@@ -58,7 +58,7 @@ def _check_rows(wl, ind, lays, idx, outs, rows, ctx_len=None, check_scores=True)
         kd = kdec[b]
         kpd = kpool_dec[b] if kpool_dec is not None else None
         if check_scores:
-            keys = ind["k_idx"] if wl.pool == 1 else dsa.dsa_index_pool(ind["k_idx"])
+            keys = ind["k_idx"] if wl.pool == 1 else dsa.dsa_index_pool(ind["k_idx"], pool=wl.pool)
             sc = dsa.dsa_index_scores(q_idx, w, keys, ctx, pool=wl.pool)
             sc_h = P.to_np(sc[b])
         lay_np = [(P.bf16_np(L["kv"][b]), None if wl.kv_latent else P.bf16_np(L["v"][b])) for L in lays]
@@ -150,15 +150,16 @@ def test_indexpool_small():
     _check_rows(wl, ind, lays, idx, outs, [(0, t) for t in (0, 1, 2, 3, 100, 255, 256, 511)])
 
 
-def test_indexpool_every_code_bit_exact():
+@pytest.mark.parametrize("factor", [2, 4, 8])
+def test_indexpool_every_code_bit_exact(factor):
     """Pooling of keys drawn uniformly over all 254 finite e4m3 codes (so sums cancel,
     saturate and land on ties of every binade): the pooled codes equal the oracle's bit for
-    bit."""
+    bit, for the pages' factor 4 and for 2 and 8."""
     g = torch.Generator(device="cpu").manual_seed(17)
     codes = torch.randint(0, 254, (2, 1 << 17, 128), generator=g, dtype=torch.int32)
     codes = torch.where(codes >= 0x7F, codes + 1, codes).to(torch.uint8)   # skip 0x7F (NaN); 0xFF is never drawn
-    kp = dsa.dsa_index_pool(codes.to(DEV))
-    assert np.array_equal(P.to_np(kp), O.index_pool(codes.numpy()))
+    kp = dsa.dsa_index_pool(codes.to(DEV), pool=factor)
+    assert np.array_equal(P.to_np(kp), O.index_pool(codes.numpy(), pool=factor))
 
 
 def test_mla_shapes_small_prefill():
@@ -245,3 +246,173 @@ def test_topk_long_rows_exact_with_ties(reps):
         valid = got[got >= 0]
         assert np.array_equal(np.sort(valid), np.sort(ref[ref >= 0])), f"row {b}"
         assert (np.diff(valid) > 0).all() and (got[valid.size:] == -1).all(), f"row {b}"
+
+
+@pytest.mark.parametrize("name", ["tiny", "prefill32k"])
+def test_attention_ids_beyond_the_cache_are_skipped_and_flagged(name):
+    """Selected ids at or beyond the cache length S_kv are skipped on the device like a -1 and
+    reported by dsa_device_status() as DSA_ERR_INDEX_RANGE.  The cache passed is a view of the
+    first S_kv rows of a larger allocation, so the rows the bad ids name are real memory and a
+    missing check would show up as wrong outputs, not as a read outside any allocation."""
+    wl = W.WORKLOADS[name].replace(T=48, ctx=300)
+    S = wl.ctx
+    big = W.make_attn_inputs(wl.replace(ctx=S + 128), 0, device=DEV)
+    q = big["q"][:, :wl.T].contiguous()
+    kv = big["kv"][:, :S]                                   # S_kv = S rows; 128 more rows follow in memory
+    v = None if big["v"] is None else big["v"][:, :S]
+    g = torch.Generator(device="cpu").manual_seed(23)
+    k = min(wl.topk, 128)
+    idx = torch.randint(0, S, (1, wl.T, k), generator=g).to(torch.int32)
+    bad = torch.rand((1, wl.T, k), generator=g) < 0.1
+    idx[bad] = (S + torch.randint(0, 128, (int(bad.sum()),), generator=g)).to(torch.int32)
+    idx[0, 5] = S + 3                                       # a row where every id is out of range
+    assert dsa.dsa_device_status() == 0
+    out, lse = dsa.dsa_sparse_attn(q, kv, idx.to(DEV), wl.sm_scale, wl.d_v, v=v, want_lse=True)
+    assert dsa.dsa_device_status() == 7                     # DSA_ERR_INDEX_RANGE, then cleared
+    assert dsa.dsa_device_status() == 0
+    K = P.bf16_np(kv[0])
+    V = K[:, : wl.d_v] if wl.kv_latent else P.bf16_np(v[0])
+    skipped = idx[0].numpy().copy()
+    skipped[skipped >= S] = -1                              # what the oracle must see
+    for t in (0, 1, 5, 17, wl.T - 1):
+        msg = P.check_attn_row(P.bf16_np(out[0, t]), P.bf16_np(q[0, t]), K, V, skipped[t], wl.sm_scale,
+                               P.to_np(lse[0, t]).astype(np.float64))
+        assert msg is None, f"row {t}: {msg}"
+    assert (P.bf16_np(out[0, 5]) == 0).all() and np.isneginf(P.to_np(lse[0, 5])).all()
+
+
+@pytest.mark.parametrize("factor,topk", [(2, 96), (8, 24)])
+def test_indexpool_factors_2_and_8(factor, topk):
+    """IndexPool over 2 and 8 keys: pooled keys bit-exact against the oracle, then the pooled
+    indexer, block top-k and expansion to P tokens per block, and the attention over them."""
+    wl = W.WORKLOADS["tiny"].replace(T=512, ctx=2048, topk=topk, pool=factor)
+    ind, lays = _inputs(wl, layers=2)
+    kp = dsa.dsa_index_pool(ind["k_idx"], pool=factor)
+    kp_h = P.to_np(kp)
+    assert kp_h.shape[1] == 2048 // factor
+    assert np.array_equal(kp_h, O.index_pool(P.to_np(ind["k_idx"]), pool=factor))
+    idx, outs = _run_group(wl, ind, lays)
+    _check_rows(wl, ind, lays, idx, outs, [(0, t) for t in (0, 1, factor - 1, factor, 100, 255, 256, 511)])
+
+
+def test_pooled_decode_small():
+    """The decode-shaped pooled path (one query per sequence, QB=1 indexer over pooled keys,
+    top-512 blocks, split-key MLA attention), at a cache size the oracle checks in seconds."""
+    wl = W.WORKLOADS["decode256k_pool"].replace(B=3, ctx=9000)
+    ind, lays = _inputs(wl, layers=2)
+    ctx = torch.tensor([9000, 4097, 2051], dtype=torch.int32, device=DEV)
+    idx, outs = _run_group(wl, ind, lays, ctx_len=ctx)
+    _check_rows(wl, ind, lays, idx, outs, [(b, 0) for b in range(3)], ctx_len=ctx)
+
+
+def _run_box(wl, ind, lays, box):
+    """One shard box (b0, b1, t0, t1) as its own group call: rows t0..t1-1 of sequences
+    b0..b1-1, with ctx_len moved to the chunk's end so every row keeps its position."""
+    b0, b1, t0, t1 = box
+    sl = lambda x: x[b0:b1, t0:t1].contiguous()      # noqa: E731
+    ctx = ind["ctx_len"][b0:b1] - (wl.T - t1)
+    layers = [{"q": sl(L["q"]), "kv": L["kv"][b0:b1], "v": None if L["v"] is None else L["v"][b0:b1]} for L in lays]
+    return dsa.dsa_group_forward(sl(ind["q_idx"]), sl(ind["w"]), ind["k_idx"][b0:b1], ctx, wl.topk, layers,
+                                 wl.sm_scale, wl.d_v, pool=wl.pool, want_lse=True)
+
+
+@pytest.mark.parametrize("name,over", [("tiny", {}), ("decode256k", {"B": 5, "ctx": 3000})])
+def test_sharded_plan_reproduces_the_single_call_bitwise(name, over):
+    """The 2-rank sharding plan (zig-zag row chunks for prefill, batch slices for decode), its
+    boxes run one after another on this GPU, gives the single call's ids, outputs and lse bit
+    for bit (both sides use the same key split here, so even the fp32 sums agree)."""
+    from indexed_sparse_attention_fp8_b200 import shard
+    wl = W.WORKLOADS[name].replace(**over)
+    ind, lays = _inputs(wl, layers=2)
+    idx, outs = _run_group(wl, ind, lays)
+    seen = 0
+    for rank in range(2):
+        for box in shard.plan(wl, 2, rank):
+            b0, b1, t0, t1 = box
+            idx_c, outs_c = _run_box(wl, ind, lays, box)
+            assert torch.equal(idx_c, idx[b0:b1, t0:t1]), box
+            for (o, l), (oc, lc) in zip(outs, outs_c):
+                assert torch.equal(oc, o[b0:b1, t0:t1]) and torch.equal(lc, l[b0:b1, t0:t1]), box
+            seen += (b1 - b0) * (t1 - t0)
+    assert seen == wl.B * wl.T
+
+
+def _to_pages(x, page_size, table, num_pages):
+    """A per-sequence cache [B, S, W] copied into a page pool [num_pages, page_size, W] along
+    the block table [B, pages_per_seq]; pages not in the table hold noise."""
+    B, S, W = x.shape
+    if x.dtype == torch.uint8:                              # e4m3 codes: any byte but NaN (0x7F, 0xFF)
+        pool = torch.randint(0, 0x7F, (num_pages, page_size, W), dtype=torch.uint8, device=x.device)
+    else:
+        pool = torch.randn((num_pages, page_size, W), device=x.device).to(x.dtype)
+    for b in range(B):
+        for j in range(table.shape[1]):
+            rows = x[b, j * page_size:(j + 1) * page_size]
+            pool[int(table[b, j]), : rows.shape[0]] = rows
+    return pool
+
+
+def _page_table(B, S, page_size, spare, seed):
+    pps = (S + page_size - 1) // page_size
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    perm = torch.randperm(B * pps + spare, generator=g)[: B * pps].to(torch.int32)
+    return perm.view(B, pps).to(DEV), B * pps + spare
+
+
+@pytest.mark.parametrize("name,over,page_size", [
+    ("tiny", {"B": 2, "T": 300, "ctx": 1000}, 128),
+    ("decode256k", {"B": 3, "ctx": 3000}, 256),
+    ("decode256k_pool", {"B": 2, "ctx": 5000}, 128),
+])
+def test_paged_caches_reproduce_the_contiguous_call_bitwise(name, over, page_size):
+    """Paged KV (the serving form of decode and chunked prefill): the indexer keys and every
+    layer's latent (or K and V) rows live in shuffled pages of shared pools, addressed through
+    a block table; the group call gives the contiguous call's ids, outputs and lse bit for bit
+    (the indexer, the pool kernel and both attention kernels read through the table)."""
+    wl = W.WORKLOADS[name].replace(**over)
+    ind, lays = _inputs(wl, layers=2)
+    ctx = torch.tensor([wl.ctx - 37 * b for b in range(wl.B)], dtype=torch.int32, device=DEV)
+    idx, outs = _run_group(wl, ind, lays, ctx_len=ctx)
+    table, num_pages = _page_table(wl.B, wl.S, page_size, spare=3, seed=7)
+    pg = dsa.paging(table, page_size, num_pages)
+    kp = _to_pages(ind["k_idx"], page_size, table.cpu(), num_pages)
+    layers = [{"q": L["q"], "kv": _to_pages(L["kv"], page_size, table.cpu(), num_pages),
+               "v": None if L["v"] is None else _to_pages(L["v"], page_size, table.cpu(), num_pages)} for L in lays]
+    idx_p, outs_p = dsa.dsa_group_forward(ind["q_idx"], ind["w"], kp, ctx, wl.topk, layers, wl.sm_scale, wl.d_v,
+                                          pool=wl.pool, want_lse=True, paging=pg)
+    assert dsa.dsa_device_status() == 0
+    assert torch.equal(idx_p, idx)
+    for (o, l), (op, lp) in zip(outs, outs_p):
+        assert torch.equal(op, o) and torch.equal(lp, l)
+
+
+def test_paged_bad_page_ids_are_skipped_and_flagged():
+    """A block-table entry outside [0, num_pages) is never followed: the attention skips the
+    rows on that page (like -1 ids), the indexer reads zeros for them, and the status reports
+    DSA_ERR_INDEX_RANGE.  The bad entries here point just past the pool and at -1."""
+    wl = W.WORKLOADS["decode256k"].replace(B=2, ctx=1024)
+    ind, lays = _inputs(wl, layers=1)
+    table, num_pages = _page_table(wl.B, wl.S, 256, spare=0, seed=9)
+    bad = table.clone()
+    bad[0, 1] = num_pages                                   # rows 256..511 of sequence 0
+    bad[1, 3] = -1                                          # rows 768..1023 of sequence 1
+    pg = dsa.paging(bad, 256, num_pages)
+    kv_pool = _to_pages(lays[0]["kv"], 256, table.cpu(), num_pages)
+    g = torch.Generator(device="cpu").manual_seed(4)
+    sel = torch.randint(0, 1024, (wl.B, 1, 300), generator=g).to(torch.int32).to(DEV)
+    out, lse = dsa.dsa_sparse_attn(lays[0]["q"], kv_pool, sel, wl.sm_scale, wl.d_v, want_lse=True, paging=pg)
+    assert dsa.dsa_device_status() == 7
+    K = [P.bf16_np(lays[0]["kv"][b]) for b in range(wl.B)]
+    sel_h = P.to_np(sel).copy()
+    sel_h[0][(sel_h[0] >= 256) & (sel_h[0] < 512)] = -1     # what the oracle must see
+    sel_h[1][sel_h[1] >= 768] = -1
+    for b in range(wl.B):
+        msg = P.check_attn_row(P.bf16_np(out[b, 0]), P.bf16_np(lays[0]["q"][b, 0]), K[b], K[b][:, : wl.d_v],
+                               sel_h[b, 0], wl.sm_scale, P.to_np(lse[b, 0]).astype(np.float64))
+        assert msg is None, f"sequence {b}: {msg}"
+    kp = _to_pages(ind["k_idx"], 256, table.cpu(), num_pages)
+    sc = dsa.dsa_index_scores(ind["q_idx"], ind["w"], kp, ind["ctx_len"], paging=pg)
+    assert dsa.dsa_device_status() == 7
+    assert (P.to_np(sc[0, 0, 256:512]) == 0).all()          # zero keys score exactly 0
+    ref = dsa.dsa_index_scores(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"])
+    assert torch.equal(sc[0, 0, :256], ref[0, 0, :256]) and torch.equal(sc[1, 0, :768], ref[1, 0, :768])

@@ -1,8 +1,11 @@
 """The workspace-free attention entry point (dsa_sparse_attn_noalloc), for callers that can
 neither allocate device memory nor pass a workspace.  It must give the same results as
 dsa_sparse_attn on split-key (decode-shaped) problems, on two calls in a row with different
-inputs (the shared scratch keeps the previous call's contents), and reject problems larger
-than its fixed scratch.  Called through the C ABI."""
+inputs (the shared scratch keeps the previous call's contents), with and without the lse
+output, at both split counts the MLA kernel picks for decode batches (4 splits up to 18
+queries, 2 from 19 to 37), and for a 32-query decode batch whose default split needs more
+partials than the scratch holds (the call then runs at fewer splits instead of failing).
+Called through the C ABI.  This file is collected last."""
 import numpy as np
 import pytest
 import torch
@@ -23,6 +26,20 @@ def _decode_case(seed_layer, B, ctx, wl_name="decode256k"):
     return wl, lay, idx.cuda()
 
 
+def _compare(wl, lay, idx, want_lse):
+    ref, ref_lse = dsa.dsa_sparse_attn(lay["q"], lay["kv"], idx, wl.sm_scale, wl.d_v, v=lay["v"], want_lse=want_lse)
+    got, got_lse = dsa.dsa_sparse_attn_noalloc(lay["q"], lay["kv"], idx, wl.sm_scale, wl.d_v, v=lay["v"],
+                                               want_lse=want_lse)
+    torch.cuda.synchronize()
+    d = np.abs(P.bf16_np(got) - P.bf16_np(ref))
+    assert d.max() <= P.ATTN_MAX and d.mean() <= P.ATTN_MEAN
+    if want_lse:
+        np.testing.assert_allclose(P.to_np(got_lse), P.to_np(ref_lse), rtol=1e-5, atol=1e-5)
+    else:
+        assert got_lse is None
+    assert dsa.dsa_device_status() == 0
+
+
 @pytest.mark.parametrize("wl_name,B,ctx", [("decode256k", 3, 5000), ("tiny", 4, 700)])
 def test_noalloc_matches_workspace_entry_on_two_calls(wl_name, B, ctx):
     lib = dsa._lib()
@@ -30,23 +47,23 @@ def test_noalloc_matches_workspace_entry_on_two_calls(wl_name, B, ctx):
     for call in range(2):                                  # second call sees the first call's scratch
         wl, lay, idx = _decode_case(call, B, ctx, wl_name)
         assert dsa.dsa_sparse_attn_workspace_size(B, 1, wl.Hq, wl.d_v, wl.topk) > 0   # split-key path
-        ref, ref_lse = dsa.dsa_sparse_attn(lay["q"], lay["kv"], idx, wl.sm_scale, wl.d_v, v=lay["v"], want_lse=True)
-        got, got_lse = dsa.dsa_sparse_attn_noalloc(lay["q"], lay["kv"], idx, wl.sm_scale, wl.d_v, v=lay["v"],
-                                                   want_lse=True)
-        torch.cuda.synchronize()
-        d = np.abs(P.bf16_np(got) - P.bf16_np(ref))
-        assert d.max() <= P.ATTN_MAX and d.mean() <= P.ATTN_MEAN
-        np.testing.assert_allclose(P.to_np(got_lse), P.to_np(ref_lse), rtol=1e-5, atol=1e-5)
-        assert dsa.dsa_device_status() == 0
+        _compare(wl, lay, idx, want_lse=True)
 
 
-def test_noalloc_rejects_problems_beyond_its_scratch():
-    wl = W.WORKLOADS["decode256k"].replace(B=32, T=1, ctx=4096)   # two splits: 16.8 MB of partials
+@pytest.mark.parametrize("B,want_lse", [(3, False), (24, True), (24, False)])
+def test_noalloc_both_mla_split_counts_with_and_without_lse(B, want_lse):
+    """B=3 takes 4 key splits, B=24 takes 2; the lse output is optional."""
+    wl, lay, idx = _decode_case(2, B, 4100)
+    need = dsa.dsa_sparse_attn_workspace_size(B, 1, wl.Hq, wl.d_v, wl.topk)
+    assert 0 < need <= dsa._lib().dsa_noalloc_scratch_bytes()
+    _compare(wl, lay, idx, want_lse)
+
+
+def test_noalloc_decode_batch_beyond_its_scratch_runs_at_fewer_splits():
+    """32 decode queries: the default split's partials exceed the fixed scratch, so the call
+    runs at fewer splits and still matches the workspace entry point."""
+    wl, lay, idx = _decode_case(3, 32, 4096)
     need = dsa.dsa_sparse_attn_workspace_size(wl.B, 1, wl.Hq, wl.d_v, wl.topk)
     assert need > dsa._lib().dsa_noalloc_scratch_bytes()
-    q = torch.zeros((wl.B, 1, wl.Hq, wl.d_qk), dtype=torch.bfloat16, device="cuda")
-    kv = torch.zeros((wl.B, 64, wl.d_qk), dtype=torch.bfloat16, device="cuda")
-    idx = torch.zeros((wl.B, 1, wl.topk), dtype=torch.int32, device="cuda")
-    with pytest.raises(dsa.DSAError) as ei:
-        dsa.dsa_sparse_attn_noalloc(q, kv, idx, wl.sm_scale, wl.d_v)
-    assert ei.value.status == 4                            # DSA_ERR_WORKSPACE_TOO_SMALL, nothing enqueued
+    for want_lse in (True, False):
+        _compare(wl, lay, idx, want_lse)
