@@ -140,6 +140,32 @@ int dsa_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, int
              int pool, int t_begin, int t_count, int k, int32_t* idx, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * dsa_index_select - Stage 1 and Stage 2 together: the selection dsa_index_scores followed by
+ * dsa_topk would give for rows t_begin .. t_begin+t_count-1 (same arguments, same ids bit for
+ * bit), without writing the full score rows when the keys allow it ("fused": contiguous keys,
+ * S_max a multiple of 16):
+ *   1. the indexer scores every 16th key row; per query row the r-th largest of those samples
+ *      (r = k/8 clamped to [32, 512]) becomes the row's threshold tau;
+ *   2. the indexer scores every visible key and appends only the keys scoring >= tau, as
+ *      (score, key id), to a candidate row of up to 8192 entries;
+ *   3. the exact top-k (ties toward lower key index, ids ascending) runs on the candidates:
+ *      with at least k candidates, every key that the full row's top-k keeps is among them.
+ *   Rows left with fewer than k candidates, or more than 8192, are redone from full score rows
+ *   by a repair pass that runs only their work items.
+ * Otherwise (paged keys, or S_max not a multiple of 16) the full score rows go through the
+ * workspace.  k_idx: keys, or pooled blocks when pool > 1, as for dsa_index_scores.
+ *   idx  [B, T, k*pool] int32 out (rows t_begin .. t_begin+t_count-1 written)
+ *   ws   at least dsa_index_select_workspace_size(B, 1, S_max, pool) bytes; the call works in
+ *        query chunks of the largest size that fits.
+ * Supported: as dsa_index_scores, and 1 <= k <= 2048.
+ * ------------------------------------------------------------------------------------ */
+size_t dsa_index_select_workspace_size(int B, int t_chunk, int S_max, int pool);
+int dsa_index_select(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                     const int32_t* ctx_len, int B, int T, int S_max, int H_I, int d_I, int pool,
+                     int t_begin, int t_count, int k, int32_t* idx, void* ws, size_t ws_bytes,
+                     const dsa_paging* paging, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * dsa_sparse_attn - attention of every query over its selected keys only (Stage 2; the
  * "China's First Frontier Model?" page, section "The Time has Come": attend only to the
  * indexer's candidates).  All Hq query heads share one KV head (MQA; MLA latent form when
@@ -215,8 +241,9 @@ int dsa_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool, ui
 /* ------------------------------------------------------------------------------------
  * dsa_group_forward - one IndexShare group ("IndexShare: Amortizing the Indexer"): the
  * indexer and the top-k run ONCE, and each of the group_size attention layers reads the
- * same index buffer.  Equivalent to dsa_index_scores + dsa_topk over all queries
- * (processed in query chunks sized to the workspace), then group_size x dsa_sparse_attn.
+ * same index buffer.  Equivalent to dsa_index_select over all queries (in query chunks sized
+ * to the workspace; full score rows instead when full_scores = 1), then group_size x
+ * dsa_sparse_attn.
  * With pool > 1 the indexer runs on dsa_index_pool's blocks and `topk` counts blocks
  * (idx then holds pool*topk token ids per row).  The comparator without IndexShare is
  * group_size calls with group_size = 1 and per-layer indexer tensors.
@@ -244,6 +271,8 @@ typedef struct dsa_group_args {
   int32_t* idx;            /* [B, T, topk*pool] int32 out: the shared selection */
   dsa_paging paging;       /* block_table NULL: contiguous caches; else k_idx and every
                               layer's kv (and v) are page pools sharing this table */
+  int32_t full_scores;     /* 0 (default): fused selection where the keys allow it (see
+                              dsa_index_select); 1: always full score rows + dsa_topk */
 } dsa_group_args;
 
 /* Workspace for dsa_group_forward when the indexer is run over chunks of t_chunk queries

@@ -65,7 +65,7 @@ class GroupArgs(ctypes.Structure):
         ("kv_row_stride", _c_i64), ("kv_batch_stride", _c_i64), ("v_row_stride", _c_i64),
         ("v_batch_stride", _c_i64),
         ("Hq", ctypes.c_int32), ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32), ("sm_scale", _c_f),
-        ("idx", _c_p), ("paging", Paging),
+        ("idx", _c_p), ("paging", Paging), ("full_scores", ctypes.c_int32),
     ]
 
 
@@ -81,6 +81,9 @@ _SIGS = {
     "dsa_index_scores": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                   _c_int, _c_int, _c_p, _c_i64, ctypes.POINTER(Paging), _c_p]),
     "dsa_topk": (_c_int, [_c_p, _c_i64, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p]),
+    "dsa_index_select_workspace_size": (_c_sz, [_c_int, _c_int, _c_int, _c_int]),
+    "dsa_index_select": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                  _c_int, _c_int, _c_p, _c_p, _c_sz, ctypes.POINTER(Paging), _c_p]),
     "dsa_sparse_attn_workspace_size": (_c_sz, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "dsa_sparse_attn": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_p, _c_int, _c_int,
                                  _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_sz, ctypes.POINTER(Paging),
@@ -233,6 +236,38 @@ def _cache_rows(kv: torch.Tensor, v: Optional[torch.Tensor], pg: Optional[Paging
     return int(kv.shape[1] if v is None else min(kv.shape[1], v.shape[1]))
 
 
+def dsa_index_select_workspace_size(B: int, t_chunk: int, S_max: int, pool: int = 1) -> int:
+    return int(_lib().dsa_index_select_workspace_size(B, t_chunk, S_max, pool))
+
+
+def dsa_index_select(q_idx: torch.Tensor, w: torch.Tensor, k_idx: torch.Tensor, ctx_len: torch.Tensor, k: int,
+                     pool: int = 1, t_begin: int = 0, t_count: Optional[int] = None, idx: Optional[torch.Tensor] = None,
+                     ws: Optional[torch.Tensor] = None, t_chunk: Optional[int] = None, paging: Optional[Paging] = None,
+                     stream=None) -> torch.Tensor:
+    """Indexer + top-k of rows t_begin.. in one call (fused: no full score rows where the keys
+    allow it).  Same ids as dsa_index_scores followed by dsa_topk.  Returns idx [B, T, k*pool]."""
+    B, T, H, D = q_idx.shape
+    S = k_idx.shape[1] if paging is None else paging.pages_per_seq * paging.page_size
+    tc = T - t_begin if t_count is None else t_count
+    _layout("q_idx", q_idx, torch.uint8, (B, T, H, D))
+    _layout("w", w, torch.float32, (B, T, H))
+    if paging is None:
+        _layout("k_idx", k_idx, torch.uint8, (B, S, D))
+    else:
+        _layout("k_idx", k_idx, torch.uint8, (paging.num_pages, paging.page_size, D))
+    _layout("ctx_len", ctx_len, torch.int32, (B,))
+    if idx is None:
+        idx = torch.full((B, T, k * pool), -1, dtype=torch.int32, device=q_idx.device)
+    _layout("idx", idx, torch.int32, (B, T, k * pool))
+    if ws is None:
+        ws = torch.empty(dsa_index_select_workspace_size(B, t_chunk or tc, S, pool), dtype=torch.uint8,
+                         device=q_idx.device)
+    _check("dsa_index_select", _lib().dsa_index_select(
+        _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(ctx_len), B, T, S, H, D, pool, t_begin, tc, k, _ptr(idx), _ptr(ws),
+        ws.numel() * ws.element_size(), _paging_ref(paging), _stream(stream)))
+    return idx
+
+
 def _attn_layouts(q, kv, v, idx, d_v, out, lse, pg: Optional[Paging] = None) -> None:
     B, T, Hq, Dqk = q.shape
     _layout("q", q, torch.bfloat16, (B, T, Hq, Dqk))
@@ -323,7 +358,7 @@ class Group:
 
     def __init__(self, q_idx, w, k_idx, ctx_len, topk: int, layers: Sequence[dict], sm_scale: float,
                  d_v: int, pool: int = 1, idx: Optional[torch.Tensor] = None, want_lse: bool = False,
-                 paging: Optional[Paging] = None):
+                 paging: Optional[Paging] = None, full_scores: bool = False):
         B, T, H, D = q_idx.shape
         S = k_idx.shape[1] if paging is None else paging.pages_per_seq * paging.page_size
         L = len(layers)
@@ -372,7 +407,7 @@ class Group:
             v_row_stride=v_any.stride(1) if v_any is not None else 0,
             v_batch_stride=v_any.stride(0) if v_any is not None else 0,
             Hq=Hq, d_qk=Dqk, d_v=d_v, sm_scale=float(sm_scale), idx=_ptr(self.idx),
-            paging=paging if paging is not None else Paging())
+            paging=paging if paging is not None else Paging(), full_scores=1 if full_scores else 0)
         self._paging = paging
         self.device = q0.device
 
@@ -387,11 +422,13 @@ class Group:
 
 def dsa_group_forward(q_idx, w, k_idx, ctx_len, topk: int, layers: Sequence[dict], sm_scale: float, d_v: int,
                       pool: int = 1, t_chunk: Optional[int] = None, ws: Optional[torch.Tensor] = None,
-                      want_lse: bool = False, paging: Optional[Paging] = None, stream=None):
+                      want_lse: bool = False, paging: Optional[Paging] = None, full_scores: bool = False,
+                      stream=None):
     """One IndexShare group: indexer + top-k once, then attention for each layer dict
     {"q", "kv", optional "v", "out", "lse"}; with `paging`, k_idx and every layer's kv (and v)
     are page pools sharing its block table.  Returns (idx, [(out, lse) per layer])."""
-    g = Group(q_idx, w, k_idx, ctx_len, topk, layers, sm_scale, d_v, pool, want_lse=want_lse, paging=paging)
+    g = Group(q_idx, w, k_idx, ctx_len, topk, layers, sm_scale, d_v, pool, want_lse=want_lse, paging=paging,
+              full_scores=full_scores)
     if ws is None:
         ws = torch.empty(g.workspace_size(t_chunk or q_idx.shape[1]), dtype=torch.uint8, device=g.device)
     return g.forward(ws, stream)

@@ -97,20 +97,113 @@ int check_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, i
   return DSA_OK;
 }
 
-// Workspace pieces of a group call: pooled keys, attention partials, a scores chunk.
+// ---- selection (indexer + top-k) of a chunk of queries
+// Fused where the keys allow it: a sampling pass scores every kSampleStride-th key row, the
+// r-th largest sample of a row is its threshold, the indexer appends only the keys scoring at
+// least the threshold, and the exact top-k runs on those candidates; rows left with fewer
+// than k candidates (or more than kCandCap) are redone from full score rows by a repair pass
+// that runs only their work items.  Otherwise the full score rows go through the workspace.
+constexpr int kSampleStride = 16;
+constexpr int kCandCap = 8192;   // candidates per row (the top-k's shared-memory buffer)
+
+// Workspace of one chunk of `rows` = B * t_chunk query rows, carved in this order.
+struct SelectWs {
+  bool fused;
+  int64_t ld, lds;
+  size_t scores, samples, cand, small;   // bytes of each piece (small: tau, cnt, fail)
+  size_t total() const { return scores + samples + cand + 3 * small; }
+};
+
+SelectWs select_ws(int64_t rows, int S_eff, bool fused) {
+  SelectWs w;
+  w.fused = fused;
+  w.ld = (int64_t)round_up((size_t)S_eff, 4);
+  w.lds = (int64_t)round_up((size_t)(S_eff / kSampleStride), 4);
+  w.scores = round_up((size_t)rows * w.ld * sizeof(float), 256);
+  w.samples = fused ? round_up((size_t)rows * w.lds * sizeof(float), 256) : 0;
+  w.cand = fused ? round_up((size_t)rows * kCandCap * sizeof(float2), 256) : 0;
+  w.small = fused ? round_up((size_t)rows * sizeof(int), 256) : 0;
+  return w;
+}
+
+// The fused path needs contiguous keys whose sequences hold whole sampled rows.
+bool select_fused_ok(int S_eff, const PageMap& key_pm, int full_scores) {
+  return full_scores == 0 && key_pm.bt == nullptr && S_eff >= kSampleStride && S_eff % kSampleStride == 0;
+}
+
+// Largest chunk of queries (<= T) whose selection workspace fits `bytes`; 0 if none does.
+int select_chunk(size_t bytes, int B, int T, int S_eff, bool fused) {
+  int lo = 0, hi = T;
+  while (lo < hi) {
+    const int mid = lo + (hi - lo + 1) / 2;
+    if (select_ws((int64_t)B * mid, S_eff, fused).total() <= bytes) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Selection of rows t0 .. t0+tc-1 of every sequence into idx, using the chunk workspace `ws`.
+int run_select(const uint8_t* q_idx, const float* w, const uint8_t* keys, const int32_t* ctx_len, int B, int T,
+               int S_eff, int H_I, int d_I, int pool, int t0, int tc, int k, int32_t* idx, uint8_t* ws, bool fused,
+               const PageMap& key_pm, cudaStream_t s) {
+  const int64_t rows = (int64_t)B * tc;
+  const SelectWs L = select_ws(rows, S_eff, fused);
+  float* scores = reinterpret_cast<float*>(ws);
+  if (!fused) {
+    int st = launch_index_scores(q_idx, w, keys, ctx_len, B, T, S_eff, H_I, d_I, pool, t0, tc, scores, L.ld, key_pm, s);
+    if (st != DSA_OK) return st;
+    return launch_topk(scores, L.ld, ctx_len, B, T, S_eff, pool, t0, tc, k, idx, s);
+  }
+  float* samples = reinterpret_cast<float*>(ws + L.scores);
+  float2* cand = reinterpret_cast<float2*>(ws + L.scores + L.samples);
+  float* tau = reinterpret_cast<float*>(ws + L.scores + L.samples + L.cand);
+  int* cnt = reinterpret_cast<int*>(ws + L.scores + L.samples + L.cand + L.small);
+  int* fail = reinterpret_cast<int*>(ws + L.scores + L.samples + L.cand + 2 * L.small);
+  // about 2k candidates expected per row (every kSampleStride-th key scored, r = k/8 of them
+  // above the threshold), so falling below k is a rare event even for small k
+  const int r = std::min(std::max(k / 8, 32), kCandCap / kSampleStride);
+  IndexerMode sample;
+  sample.kstride = kSampleStride;
+  int st = launch_index_scores(q_idx, w, keys, ctx_len, B, T, S_eff / kSampleStride, H_I, d_I, pool * kSampleStride,
+                               t0, tc, samples, L.lds, key_pm, s, sample);
+  if (st != DSA_OK) return st;
+  if ((st = launch_sample_threshold(samples, L.lds, ctx_len, B, T, S_eff, pool, kSampleStride, t0, tc, r, kCandCap,
+                                    tau, s)) != DSA_OK)
+    return st;
+  if (cudaMemsetAsync(cnt, 0, (size_t)rows * sizeof(int), s) != cudaSuccess) return check_launch();
+  IndexerMode cm;
+  cm.tau = tau;
+  cm.cand = cand;
+  cm.cnt = cnt;
+  cm.cap = kCandCap;
+  if ((st = launch_index_scores(q_idx, w, keys, ctx_len, B, T, S_eff, H_I, d_I, pool, t0, tc, nullptr, L.ld, key_pm, s,
+                                cm)) != DSA_OK)
+    return st;
+  if ((st = launch_topk_cand(cand, cnt, kCandCap, ctx_len, B, T, S_eff, pool, t0, tc, k, idx, fail, s)) != DSA_OK)
+    return st;
+  // repair: full score rows and the row top-k, for the flagged rows only
+  IndexerMode rep;
+  rep.row_flag = fail;
+  if ((st = launch_index_scores(q_idx, w, keys, ctx_len, B, T, S_eff, H_I, d_I, pool, t0, tc, scores, L.ld, key_pm, s,
+                                rep)) != DSA_OK)
+    return st;
+  return launch_topk(scores, L.ld, ctx_len, B, T, S_eff, pool, t0, tc, k, idx, s, fail);
+}
+
+// Workspace pieces of a group call: pooled keys, attention partials, then a selection chunk.
 struct GroupWs {
   size_t pool_bytes, attn_bytes, fixed_bytes;
   int S_eff;
-  int64_t ld;
+  bool fused;
 };
 
 GroupWs group_ws(const dsa_group_args* a) {
   GroupWs g;
   g.S_eff = a->pool > 1 ? a->S_max / a->pool : a->S_max;
-  g.ld = (int64_t)round_up((size_t)g.S_eff, 4);
   g.pool_bytes = a->pool > 1 ? round_up((size_t)a->B * g.S_eff * a->d_I, 256) : 0;
   g.attn_bytes = round_up(attn_workspace_bytes(a->B, a->T, a->Hq, a->d_v, a->topk * a->pool), 256);
   g.fixed_bytes = g.pool_bytes + g.attn_bytes;
+  const PageMap key_pm = a->pool > 1 ? PageMap{nullptr, 0, 0, 0} : page_map(&a->paging);
+  g.fused = select_fused_ok(g.S_eff, key_pm, a->full_scores);
   return g;
 }
 
@@ -234,7 +327,37 @@ size_t dsa_group_workspace_size(const dsa_group_args* a, int t_chunk) {
   if (!a || t_chunk < 1) return 0;
   const GroupWs g = group_ws(a);
   const int tc = std::min(t_chunk, a->T);
-  return g.fixed_bytes + (size_t)a->B * tc * (size_t)g.ld * sizeof(float);
+  return g.fixed_bytes + select_ws((int64_t)a->B * tc, g.S_eff, g.fused).total();
+}
+
+size_t dsa_index_select_workspace_size(int B, int t_chunk, int S_max, int pool) {
+  if (B <= 0 || t_chunk < 1 || S_max < 1 || pool < 1) return 0;
+  return select_ws((int64_t)B * t_chunk, S_max, select_fused_ok(S_max, PageMap{nullptr, 0, 0, 0}, 0)).total();
+}
+
+int dsa_index_select(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* ctx_len, int B,
+                     int T, int S_max, int H_I, int d_I, int pool, int t_begin, int t_count, int k, int32_t* idx,
+                     void* ws, size_t ws_bytes, const dsa_paging* paging, void* stream) {
+  int st = check_index_scores(q_idx, w, k_idx, ctx_len, B, T, S_max, H_I, d_I, pool, t_begin, t_count,
+                              reinterpret_cast<const float*>(16), (int64_t)round_up((size_t)S_max, 4), paging);
+  if (st != DSA_OK) return st;
+  if (k < 1 || k > 2048) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || t_count == 0) return DSA_OK;
+  if (!idx) return DSA_ERR_INVALID_ARG;
+  const PageMap key_pm = page_map(paging);
+  const bool fused = select_fused_ok(S_max, key_pm, 0);
+  const int t_chunk = select_chunk(ws_bytes, B, t_count, S_max, fused);
+  if (t_chunk < 1) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  if (!ws) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return DSA_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int t0 = t_begin; t0 < t_begin + t_count; t0 += t_chunk) {
+    const int tc = std::min(t_chunk, t_begin + t_count - t0);
+    st = run_select(q_idx, w, k_idx, ctx_len, B, T, S_max, H_I, d_I, pool, t0, tc, k, idx, static_cast<uint8_t*>(ws),
+                    fused, key_pm, s);
+    if (st != DSA_OK) return st;
+  }
+  return DSA_OK;
 }
 
 int dsa_group_forward(const dsa_group_args* a, void* ws, size_t ws_bytes, void* stream) {
@@ -242,16 +365,15 @@ int dsa_group_forward(const dsa_group_args* a, void* ws, size_t ws_bytes, void* 
   if (st != DSA_OK) return st;
   if (a->B == 0) return DSA_OK;
   const GroupWs g = group_ws(a);
-  const size_t row_bytes = (size_t)a->B * g.ld * sizeof(float);
-  if (ws_bytes < g.fixed_bytes + row_bytes) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  const int t_chunk = ws_bytes < g.fixed_bytes ? 0 : select_chunk(ws_bytes - g.fixed_bytes, a->B, a->T, g.S_eff, g.fused);
+  if (t_chunk < 1) return DSA_ERR_WORKSPACE_TOO_SMALL;
   if (!ws) return DSA_ERR_INVALID_ARG;
   if (!aligned16(ws)) return DSA_ERR_MISALIGNED;
-  const int t_chunk = (int)std::min<size_t>((size_t)a->T, (ws_bytes - g.fixed_bytes) / row_bytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint8_t* k_pool = base;
   void* attn_ws = base + g.pool_bytes;
-  float* scores = reinterpret_cast<float*>(base + g.fixed_bytes);
+  uint8_t* sel_ws = base + g.fixed_bytes;
 
   const PageMap pm = page_map(&a->paging);
   const uint8_t* keys = a->k_idx;
@@ -265,11 +387,8 @@ int dsa_group_forward(const dsa_group_args* a, void* ws, size_t ws_bytes, void* 
   // IndexShare: one indexer + one top-k over every query, in chunks that fit the workspace
   for (int t0 = 0; t0 < a->T; t0 += t_chunk) {
     const int tc = std::min(t_chunk, a->T - t0);
-    st = launch_index_scores(a->q_idx, a->w, keys, a->ctx_len, a->B, a->T, g.S_eff, a->H_I, a->d_I,
-                             a->pool, t0, tc, scores, g.ld, key_pm, s);
-    if (st != DSA_OK) return st;
-    st = launch_topk(scores, g.ld, a->ctx_len, a->B, a->T, g.S_eff, a->pool, t0, tc, a->topk,
-                     a->idx, s);
+    st = run_select(a->q_idx, a->w, keys, a->ctx_len, a->B, a->T, g.S_eff, a->H_I, a->d_I, a->pool, t0, tc, a->topk,
+                    a->idx, sel_ws, g.fused, key_pm, s);
     if (st != DSA_OK) return st;
   }
   // every layer of the group reads the same selection

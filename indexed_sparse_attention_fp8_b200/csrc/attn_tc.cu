@@ -57,7 +57,7 @@ constexpr int OFF_XS = OFF_KV + NS * KV_STAGE;         // own partial, staged fo
 constexpr int OFF_X = OFF_XS + X_BYTES;                // partner's partial, copied in
 constexpr int OFF_IDS = OFF_X + X_BYTES;
 constexpr int OFF_BAR = OFF_IDS + NS * NK * 4 + 16 * NS;   // ids + an all-valid flag per stage
-constexpr int NBARS = 3 * NS + 13;
+constexpr int NBARS = 3 * NS + 14;   // + the MMA drain barrier
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;       // + alignment slack
 constexpr int THREADS = 256;            // 8 warps: 2 per SM sub-partition, so up to 255 registers
@@ -304,6 +304,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   // per softmax warp w (rows 32w..32w+31): the partner's rows landed / the partner read ours
   auto x_full = [&](int w) { return bar0 + 8u * (3 * NS + 5 + w); };
   auto x_free = [&](int w) { return bar0 + 8u * (3 * NS + 9 + w); };
+  const uint32_t mma_drain = bar0 + 8u * (3 * NS + 13);   // completes when every issued MMA has
   volatile int* ids_s = reinterpret_cast<volatile int*>(sgen + OFF_IDS);
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(sgen + OFF_MISC + 4);
@@ -343,6 +344,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     mbar_init(p_full, 4);
     mbar_init(pv_done, 1);
     mbar_init(q_ready, 4);
+    mbar_init(mma_drain, 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -486,6 +488,12 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       }
       g += I.ntiles;
     }
+    // every MMA this warp issued must have finished before the TMEM is freed: after a normal
+    // run the consumers have waited for all of them already, but after any role gave up (here or
+    // elsewhere, now or later) some may still run
+    if (lane == 0) mma_commit(mma_drain);
+    __syncwarp();
+    mbar_wait_bounded(mma_drain, 0, 100000000ull);
   } else {
     // ------------------------------------------------------------ softmax + epilogue (warps 0-3)
     const int row = warp * 32 + lane;  // head

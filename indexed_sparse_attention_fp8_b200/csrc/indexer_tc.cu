@@ -55,7 +55,7 @@ struct IdxCfg {
   static constexpr int OFF_B = OFF_A + NA * A_BYTES;
   static constexpr int OFF_W = OFF_B + 2 * B_BYTES;
   static constexpr int OFF_BAR = OFF_W + 2 * W_BYTES;
-  static constexpr int NBAR = 2 * NA + 8;
+  static constexpr int NBAR = 2 * NA + 9;           // + the MMA drain barrier
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(D == 128 || D == 64, "row = one swizzle atom");
@@ -69,15 +69,22 @@ struct ItemGeom {
   int b, t0, nq, kt0, kt1;
 };
 
-// Decodes work item `it` and returns false when it holds no visible key tile.
+// Decodes work item `it` and returns false when it holds no visible key tile, or (with a row
+// filter) none of its queries is flagged.
 __device__ __forceinline__ bool item_geom(int it, int QB, int nqb, int nkc, int T, int t_begin, int t_count,
-                                          int S_max, int pool, const int32_t* __restrict__ ctx_len, ItemGeom& g) {
+                                          int S_max, int pool, const int32_t* __restrict__ ctx_len, ItemGeom& g,
+                                          const int* __restrict__ row_flag) {
   const int kc = it % nkc;
   const int r = it / nkc;
   const int qb = r % nqb;
   g.b = r / nqb;
   g.t0 = t_begin + qb * QB;
   g.nq = min(QB, t_begin + t_count - g.t0);
+  if (row_flag != nullptr) {
+    bool any = false;
+    for (int q = 0; q < g.nq; ++q) any |= __ldg(row_flag + (int64_t)g.b * t_count + (g.t0 - t_begin) + q) != 0;
+    if (!any) return false;
+  }
   const int pos_last = __ldg(ctx_len + g.b) - T + g.t0 + g.nq - 1;
   if (pos_last < 0) return false;
   const int n_valid = min(S_max, pos_last / pool + 1);
@@ -87,11 +94,36 @@ __device__ __forceinline__ bool item_geom(int it, int QB, int nqb, int nkc, int 
   return g.kt0 < g.kt1;
 }
 
-template <int H, int D, int QB>
+// Candidate append of the fused selection: every lane of the warp calls it for the same query
+// (the lanes hold different keys); the keys that pass (visible, score >= the query's threshold)
+// take consecutive slots of the query's candidate row with one atomic per warp.  Slots past the
+// buffer are not written; the count keeps growing, so the top-k sees the overflow.
+__device__ __forceinline__ void cand_append(bool pass, float val, int s, int* __restrict__ cnt_row,
+                                            float2* __restrict__ cand_row, int cap) {
+  const unsigned m = __ballot_sync(0xffffffffu, pass);
+  if (m == 0u) return;
+  const int lane = threadIdx.x & 31;
+  const int leader = __ffs(m) - 1;
+  int base = 0;
+  if (lane == leader) base = atomicAdd(cnt_row, __popc(m));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  if (pass) {
+    const int slot = base + __popc(m & ((1u << lane) - 1u));
+    if (slot < cap) cand_row[slot] = make_float2(val, __int_as_float(s));
+  }
+}
+
+// CAND = false: the score rows are stored (masked entries -inf).  CAND = true (fused
+// selection): nothing is stored but the candidates of each query, the visible keys whose score
+// reaches tau[row]; `cnt` counts them per row.  row_flag (optional): only the work items
+// holding a flagged query run.
+template <int H, int D, int QB, bool CAND>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                        const float* __restrict__ w, const int32_t* __restrict__ ctx_len, int B, int T, int S_max,
-                       int pool, int t_begin, int t_count, float* __restrict__ scores, int64_t ld, PageMap pm) {
+                       int pool, int t_begin, int t_count, float* __restrict__ scores, int64_t ld, PageMap pm,
+                       const float* __restrict__ tau, float2* __restrict__ cand, int* __restrict__ cnt, int cap,
+                       const int* __restrict__ row_flag) {
   using C = IdxCfg<H, D, QB>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
@@ -104,6 +136,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
   auto b_empty = [&](int s) { return bar0 + 8u * (2 * NA + 2 + s); };
   auto acc_full = [&](int s) { return bar0 + 8u * (2 * NA + 4 + s); };
   auto acc_empty = [&](int s) { return bar0 + 8u * (2 * NA + 6 + s); };
+  const uint32_t mma_drain = bar0 + 8u * (2 * NA + 8);   // completes when every issued MMA has
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + C::OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(sgen + C::OFF_MISC + 4);
 
@@ -123,6 +156,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       mbar_init(acc_full(i), 1);
       mbar_init(acc_empty(i), 4 * C::HALVES);
     }
+    mbar_init(mma_drain, 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -145,7 +179,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
     bool ok = true;
     for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
       ItemGeom g;
-      if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g)) continue;
+      if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g, row_flag)) continue;
       const int bs = b_cnt & 1;
       if (!(ok = mbar_wait_warp(b_empty(bs), ((b_cnt >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
       if (lane == 0) {
@@ -176,19 +210,19 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       }
       __syncwarp();
     }
-    if (!ok) {  // drain the copies this warp issued before giving up (bounded waits)
-      for (uint32_t i = (a_cnt > NA ? a_cnt - NA : 0); i < a_cnt; ++i)
-        mbar_wait_bounded(a_full(i % NA), (i / NA) & 1, 100000000ull);
-      for (uint32_t i = (b_cnt > 2 ? b_cnt - 2 : 0); i < b_cnt; ++i)
-        mbar_wait_bounded(b_full(i & 1), (i >> 1) & 1, 100000000ull);
-    }
+    // drain, whether this warp gave up or not: the copies it issued land before the CTA can leave
+    // (after a normal run they landed long ago; after any role gave up some may be in flight)
+    for (uint32_t i = (a_cnt > NA ? a_cnt - NA : 0); i < a_cnt; ++i)
+      mbar_wait_bounded(a_full(i % NA), (i / NA) & 1, 100000000ull);
+    for (uint32_t i = (b_cnt > 2 ? b_cnt - 2 : 0); i < b_cnt; ++i)
+      mbar_wait_bounded(b_full(i & 1), (i >> 1) & 1, 100000000ull);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     uint32_t a_cnt = 0, b_cnt = 0, acc_cnt = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
       ItemGeom g;
-      if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g)) continue;
+      if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g, row_flag)) continue;
       const int bs = b_cnt & 1;
       if (!(ok = mbar_wait_warp(b_full(bs), (b_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
       const uint32_t b_addr = sbase + C::OFF_B + bs * C::B_BYTES;
@@ -218,6 +252,12 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       __syncwarp();
       ++b_cnt;
     }
+    // every MMA this warp issued must have finished before the TMEM is freed: after a normal
+    // run the consumers have waited for all of them already, but after any role gave up (here or
+    // elsewhere, now or later) some may still run
+    if (lane == 0) mma_commit(mma_drain);
+    __syncwarp();
+    mbar_wait_bounded(mma_drain, 0, 100000000ull);
   } else {
     // ------------------------------------------------------------ epilogue (8 warps)
     const int quad = warp & 3;          // TMEM lanes 32*quad .. +31
@@ -229,7 +269,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
     // the active ones)
     for (int it = blockIdx.x; half < C::HALVES && it < items && ok; it += gridDim.x) {
       ItemGeom g;
-      if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g)) continue;
+      if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g, row_flag)) continue;
       const int bs = b_cnt & 1;
       if (!(ok = mbar_wait_warp(b_full(bs), (b_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
       const float* wsm = reinterpret_cast<const float*>(sgen + C::OFF_W + bs * C::W_BYTES) + half * C::COLS;
@@ -263,17 +303,26 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
         float* qrow[C::QPH];
         int lim[C::QPH];
         bool qok[C::QPH];
+        float qtau[C::QPH];
+        int64_t qr[C::QPH];
 #pragma unroll
         for (int ql = 0; ql < C::QPH; ++ql) {
           const int qq = half * C::QPH + ql;
           const int t = g.t0 + qq;
           qok[ql] = qq < g.nq;
-          qrow[ql] = scores + ((int64_t)g.b * t_count + (t - t_begin)) * ld;
+          qr[ql] = (int64_t)g.b * t_count + (t - t_begin);
+          qrow[ql] = scores + qr[ql] * ld;
           const int pos = ctx_b - T + t;
           lim[ql] = pos < 0 ? -1 : pos / pool;   // s * pool <= pos  <=>  s <= pos / pool
+          if constexpr (CAND) qtau[ql] = qok[ql] ? __ldg(tau + qr[ql]) : INFINITY;
         }
         auto store = [&](int ql, int s, float val) {
-          if (qok[ql] && s < S_max) qrow[ql][s] = (s <= lim[ql]) ? val : -INFINITY;
+          if constexpr (CAND) {
+            cand_append(qok[ql] && s < S_max && s <= lim[ql] && val >= qtau[ql], val, s, cnt + qr[ql],
+                        cand + qr[ql] * cap, cap);
+          } else {
+            if (qok[ql] && s < S_max) qrow[ql][s] = (s <= lim[ql]) ? val : -INFINITY;
+          }
         };
         if (g.kt0 < g.kt1) {
           if (!(ok = mbar_wait_warp(acc_full(acc_cnt & 1), (acc_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
@@ -353,10 +402,15 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
         // finished sum of query ql (local to this warp) for key s -> masked store
         auto store = [&](int ql, int s, float val) {
           const int qq = half * C::QPH + ql;
-          if (qq < g.nq && s < S_max) {
-            const int t = g.t0 + qq;
-            const int pos = ctx_b - T + t;
-            scores[((int64_t)g.b * t_count + (t - t_begin)) * ld + s] = (s * pool <= pos) ? val : -INFINITY;
+          const int t = g.t0 + qq;
+          const int pos = ctx_b - T + t;
+          const int64_t qrow_id = (int64_t)g.b * t_count + (t - t_begin);
+          if constexpr (CAND) {
+            const bool live = qq < g.nq && s < S_max && s * pool <= pos;
+            cand_append(live && val >= __ldg(tau + (live ? qrow_id : 0)), val, s, cnt + (live ? qrow_id : 0),
+                        cand + (live ? qrow_id : 0) * cap, cap);
+          } else {
+            if (qq < g.nq && s < S_max) scores[qrow_id * ld + s] = (s * pool <= pos) ? val : -INFINITY;
           }
         };
         const uint32_t tcol = tmem_base + (uint32_t)(ab * C::N + half * C::COLS);
@@ -428,12 +482,14 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
 
 // ---------------------------------------------------------------- host side
 
-// 2-D uint8 tensor map: `rows` rows of `row_bytes`, boxes of box_rows x row_bytes.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t row_bytes, uint32_t box_rows) {
+// 2-D uint8 tensor map: `rows` rows of `row_bytes` spaced `row_stride` bytes apart (0 = dense),
+// boxes of box_rows x row_bytes.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t row_bytes, uint32_t box_rows,
+              uint64_t row_stride = 0) {
   auto enc = tmap_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {row_bytes, rows};
-  cuuint64_t strides[1] = {row_bytes};
+  cuuint64_t strides[1] = {row_stride ? row_stride : row_bytes};
   cuuint32_t box[2] = {row_bytes, box_rows};
   cuuint32_t estr[2] = {1, 1};
   const CUtensorMapSwizzle sw = row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -442,16 +498,17 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t row_byte
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int H, int D, int QB>
+template <int H, int D, int QB, bool CAND>
 int launch_tc(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* ctx_len, int B, int T,
               int S_max, int pool, int t_begin, int t_count, float* scores, int64_t ld, const PageMap& pm,
-              cudaStream_t stream) {
+              const IndexerMode& md, cudaStream_t stream) {
   using C = IdxCfg<H, D, QB>;
   CUtensorMap mk, mq;
+  // key rows: contiguous (every md.kstride-th row of the cache when sampling), or the page pool
   const uint64_t key_rows = pm.bt != nullptr ? ((uint64_t)pm.num_pages << pm.shift) : (uint64_t)B * S_max;
-  if (!make_map(&mk, k_idx, key_rows, D, KTILE)) return DSA_ERR_CUDA;
+  if (!make_map(&mk, k_idx, key_rows, D, KTILE, (uint64_t)md.kstride * D)) return DSA_ERR_CUDA;
   if (!make_map(&mq, q_idx, (uint64_t)B * T * H, D, C::N)) return DSA_ERR_CUDA;
-  auto kern = index_scores_tc_kernel<H, D, QB>;
+  auto kern = index_scores_tc_kernel<H, D, QB, CAND>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -464,26 +521,38 @@ int launch_tc(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const 
   const int64_t items = (int64_t)B * nqb * nkc;
   const int grid = (int)std::min<int64_t>(items, num_sms());
   kern<<<grid, NUM_THREADS, C::SMEM, stream>>>(mk, mq, w, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld,
-                                               pm);
+                                               pm, md.tau, md.cand, md.cnt, md.cap, md.row_flag);
   return check_launch();
+}
+
+template <bool CAND>
+int launch_shape(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* ctx_len, int B, int T,
+                 int S_max, int H_I, int d_I, int pool, int t_begin, int t_count, float* scores, int64_t ld,
+                 const PageMap& pm, const IndexerMode& md, cudaStream_t stream) {
+  if (H_I == 64 && d_I == 128) {
+    if (t_count < 4)  // decode-like: one query per block keeps the MMA N at the head count
+      return launch_tc<64, 128, 1, CAND>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld,
+                                         pm, md, stream);
+    return launch_tc<64, 128, 4, CAND>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, pm,
+                                       md, stream);
+  }
+  if (H_I == 4 && d_I == 64)
+    return launch_tc<4, 64, 64, CAND>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, pm,
+                                      md, stream);
+  return DSA_ERR_UNSUPPORTED_SHAPE;
 }
 
 }  // namespace
 
 int launch_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* ctx_len, int B,
                         int T, int S_max, int H_I, int d_I, int pool, int t_begin, int t_count, float* scores,
-                        int64_t ld, const PageMap& pm, cudaStream_t stream) {
+                        int64_t ld, const PageMap& pm, cudaStream_t stream, const IndexerMode& md) {
   if (B == 0 || t_count == 0 || S_max == 0) return DSA_OK;
-  if (H_I == 64 && d_I == 128) {
-    if (t_count < 4)  // decode-like: one query per block keeps the MMA N at the head count
-      return launch_tc<64, 128, 1>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, pm,
-                                   stream);
-    return launch_tc<64, 128, 4>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, pm,
-                                 stream);
-  }
-  if (H_I == 4 && d_I == 64)
-    return launch_tc<4, 64, 64>(q_idx, w, k_idx, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld, pm, stream);
-  return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (md.cand != nullptr)
+    return launch_shape<true>(q_idx, w, k_idx, ctx_len, B, T, S_max, H_I, d_I, pool, t_begin, t_count, scores, ld, pm,
+                              md, stream);
+  return launch_shape<false>(q_idx, w, k_idx, ctx_len, B, T, S_max, H_I, d_I, pool, t_begin, t_count, scores, ld, pm,
+                             md, stream);
 }
 
 namespace {

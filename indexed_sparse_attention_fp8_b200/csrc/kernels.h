@@ -8,13 +8,37 @@
 
 namespace dsa {
 
+// Options of the indexer launch beyond storing every score row (the defaults do that).
+struct IndexerMode {
+  int kstride = 1;               // read every kstride-th key row (the sampling pass of the fused
+                                 // selection; S_max and pool are then given in sampled rows)
+  const float* tau = nullptr;    // fused selection: per-row thresholds [B * t_count] ...
+  float2* cand = nullptr;        // ... candidate rows [B * t_count, cap] (score, key id as bits)
+  int* cnt = nullptr;            // ... candidates per row, zeroed before the launch
+  int cap = 0;
+  const int* row_flag = nullptr; // only work items holding a flagged row run (repair pass)
+};
+
 int launch_index_scores(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
                         const int32_t* ctx_len, int B, int T, int S_max, int H_I, int d_I, int pool,
                         int t_begin, int t_count, float* scores, int64_t ld, const PageMap& pm,
-                        cudaStream_t stream);
+                        cudaStream_t stream, const IndexerMode& md = IndexerMode());
 
+// row_flag (optional, [B * t_count]): only the rows whose flag is non-zero are selected.
 int launch_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, int T, int S_max,
-                int pool, int t_begin, int t_count, int k, int32_t* idx, cudaStream_t stream);
+                int pool, int t_begin, int t_count, int k, int32_t* idx, cudaStream_t stream,
+                const int* row_flag = nullptr);
+
+// Fused selection (indexer scores never written in full):
+//  * per row, the r-th largest of the scores of every `stride`-th key row, or -inf when all
+//    visible keys fit the candidate buffer of `cap` entries;
+int launch_sample_threshold(const float* samples, int64_t lds, const int32_t* ctx_len, int B, int T, int S_eff,
+                            int pool, int stride, int t_begin, int t_count, int r, int cap, float* tau,
+                            cudaStream_t stream);
+//  * per row, the exact top-k of its candidates (score, key id); rows with fewer than k
+//    candidates, or more than cap, get fail = 1 and are left for the repair pass.
+int launch_topk_cand(const float2* cand, const int* cnt, int cap, const int32_t* ctx_len, int B, int T, int S_max,
+                     int pool, int t_begin, int t_count, int k, int32_t* idx, int* fail, cudaStream_t stream);
 
 // Split count the attention uses for a problem by default (1 = no split, no workspace).
 int attn_num_splits(int B, int T, int Hq, int k);

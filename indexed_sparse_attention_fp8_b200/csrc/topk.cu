@@ -123,7 +123,7 @@ __device__ __forceinline__ void sort_ascending(int* sel, int n) {
 __global__ void __launch_bounds__(TK_THREADS, 1)
 topk_rows_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ ctx_len,
                  int T, int S_max, int pool, int t_begin, int t_count, int k,
-                 int32_t* __restrict__ idx_out) {
+                 int32_t* __restrict__ idx_out, const int* __restrict__ row_flag) {
   __shared__ uint32_t hist[TK_BINS];
   __shared__ int sel[TK_KMAX];
   __shared__ int warp_buf[32];
@@ -131,6 +131,7 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __
 
   const int tid = threadIdx.x;
   const int row_id = blockIdx.x;
+  if (row_flag != nullptr && row_flag[row_id] == 0) return;   // only the flagged rows (repair pass)
   const int b = row_id / t_count;
   const int t = t_begin + row_id % t_count;
   const int pos = ctx_len[b] - T + t;
@@ -262,10 +263,159 @@ topk_rows_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __
   for (int i = tid; i < k; i += TK_THREADS) write_expanded(out, i, sel[i], pool, pos);
 }
 
+
+__device__ __forceinline__ float from_order_key(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Threshold of the fused selection (one CTA per query row): the r-th largest of the row's
+// visible sampled scores -- the scores of every `stride`-th key row -- by three digit passes
+// over the samples; -inf when every visible key fits the candidate buffer (cap) anyway.
+__global__ void __launch_bounds__(TK_THREADS, 1)
+sample_threshold_kernel(const float* __restrict__ samples, int64_t lds, const int32_t* __restrict__ ctx_len, int T,
+                        int S_eff, int pool, int stride, int t_begin, int t_count, int r, int cap,
+                        float* __restrict__ tau) {
+  __shared__ uint32_t hist[TK_BINS];
+  __shared__ int warp_buf[32];
+  __shared__ int sh_bin, sh_above;
+  const int tid = threadIdx.x;
+  const int row_id = blockIdx.x;
+  const int b = row_id / t_count;
+  const int t = t_begin + row_id % t_count;
+  const int pos = ctx_len[b] - T + t;
+  const int n_valid = pos < 0 ? 0 : min(S_eff, pos / pool + 1);
+  if (n_valid <= cap) {
+    if (tid == 0) tau[row_id] = -INFINITY;
+    return;
+  }
+  const int n_s = min((S_eff + stride - 1) / stride, pos / (pool * stride) + 1);   // >= cap / stride >= r
+  const float* srow = samples + (int64_t)row_id * lds;
+  uint32_t prefix = 0, mask = 0;
+  int kk = r;
+  const int shifts[3] = {21, 10, 0};
+  for (int p = 0; p < 3; ++p) {
+    const int shift = shifts[p];
+    for (int i = tid; i < TK_BINS; i += TK_THREADS) hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n_s; i += TK_THREADS) {
+      const uint32_t key = order_key(__ldg(srow + i));
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (TK_BINS - 1)], 1u);
+    }
+    __syncthreads();
+    const int hb = TK_BINS - 1 - 2 * tid;
+    const int h0 = (int)hist[hb], h1 = (int)hist[hb - 1];
+    int total;
+    const int excl = block_excl_scan(h0 + h1, warp_buf, &total);
+    if (excl < kk && kk <= excl + h0) {
+      sh_bin = hb; sh_above = excl;
+    } else if (excl + h0 < kk && kk <= excl + h0 + h1) {
+      sh_bin = hb - 1; sh_above = excl + h0;
+    }
+    __syncthreads();
+    kk -= sh_above;
+    prefix |= (uint32_t)sh_bin << shift;
+    mask |= (uint32_t)(TK_BINS - 1) << shift;
+    __syncthreads();
+  }
+  if (tid == 0) tau[row_id] = from_order_key(prefix);   // the r-th largest sample exactly
+}
+
+// Exact top-k of one row from its candidates (score, key id): the fused indexer appended every
+// visible key scoring at least the row's threshold.  When there are at least k candidates the
+// k best keys of the row are all among them (ties at the k-th score included), so the result is
+// the full row's selection; otherwise, or when the buffer overflowed, the row is flagged for
+// the repair pass (full score row + topk_rows_kernel).
+__global__ void __launch_bounds__(TK_THREADS, 1)
+topk_cand_kernel(const float2* __restrict__ cand, const int* __restrict__ cnt, int cap,
+                 const int32_t* __restrict__ ctx_len, int T, int S_max, int pool, int t_begin, int t_count, int k,
+                 int32_t* __restrict__ idx_out, int* __restrict__ fail) {
+  __shared__ uint32_t hist[TK_BINS];
+  __shared__ int sel[TK_KMAX];
+  __shared__ int warp_buf[32];
+  __shared__ int sh_bin, sh_above, sh_cnt, sh_ngt, sh_neq;
+  const int tid = threadIdx.x;
+  const int row_id = blockIdx.x;
+  const int b = row_id / t_count;
+  const int t = t_begin + row_id % t_count;
+  const int pos = ctx_len[b] - T + t;
+  const int n_valid = pos < 0 ? 0 : min(S_max, pos / pool + 1);
+  int32_t* out = idx_out + ((int64_t)b * T + t) * (int64_t)k * pool;
+  if (n_valid <= k) {  // every visible key is selected
+    if (tid == 0) fail[row_id] = 0;
+    for (int i = tid; i < k; i += TK_THREADS) write_expanded(out, i, i < n_valid ? i : -1, pool, pos);
+    return;
+  }
+  const int ncand = cnt[row_id];
+  if (ncand < k || ncand > cap) {
+    if (tid == 0) fail[row_id] = 1;
+    return;
+  }
+  if (tid == 0) fail[row_id] = 0;
+  extern __shared__ uint32_t cand_smem[];
+  uint32_t* ck = cand_smem;
+  int* ci = reinterpret_cast<int*>(cand_smem + TK_CAP);
+  int* tie = reinterpret_cast<int*>(cand_smem + 2 * TK_CAP);
+  const float2* crow = cand + (int64_t)row_id * cap;
+  for (int j = tid; j < ncand; j += TK_THREADS) {
+    const float2 c = __ldcs(crow + j);
+    ck[j] = order_key(c.x);
+    ci[j] = __float_as_int(c.y);
+  }
+  __syncthreads();
+  uint32_t prefix = 0, mask = 0;
+  int kk = k, eq_count = ncand;
+  const int shifts[3] = {21, 10, 0};
+  for (int p = 0; p < 3 && eq_count != kk; ++p) {
+    const int shift = shifts[p];
+    for (int i = tid; i < TK_BINS; i += TK_THREADS) hist[i] = 0u;
+    __syncthreads();
+    for (int j = tid; j < ncand; j += TK_THREADS) {
+      const uint32_t key = ck[j];
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (TK_BINS - 1)], 1u);
+    }
+    __syncthreads();
+    const int hb = TK_BINS - 1 - 2 * tid;
+    const int h0 = (int)hist[hb], h1 = (int)hist[hb - 1];
+    int total;
+    const int excl = block_excl_scan(h0 + h1, warp_buf, &total);
+    if (excl < kk && kk <= excl + h0) {
+      sh_bin = hb; sh_above = excl; sh_cnt = h0;
+    } else if (excl + h0 < kk && kk <= excl + h0 + h1) {
+      sh_bin = hb - 1; sh_above = excl + h0; sh_cnt = h1;
+    }
+    __syncthreads();
+    kk -= sh_above;
+    prefix |= (uint32_t)sh_bin << shift;
+    mask |= (uint32_t)(TK_BINS - 1) << shift;
+    eq_count = sh_cnt;
+    __syncthreads();
+  }
+  // winners: every candidate above the prefix, then the ties at it (all, or the kk lowest ids)
+  const bool take_all_eq = (eq_count == kk);
+  if (tid == 0) { sh_ngt = 0; sh_neq = 0; }
+  __syncthreads();
+  for (int j = tid; j < ncand; j += TK_THREADS) {
+    const uint32_t m = ck[j] & mask;
+    if (m > prefix) {
+      sel[atomicAdd(&sh_ngt, 1)] = ci[j];
+    } else if (m == prefix) {
+      tie[atomicAdd(&sh_neq, 1)] = ci[j];
+    }
+  }
+  __syncthreads();
+  const int n_gt = sh_ngt, nties = sh_neq;   // n_gt == k - kk
+  if (!take_all_eq) sort_ascending(tie, nties);   // the lowest ids win
+  __syncthreads();
+  for (int j = tid; j < kk; j += TK_THREADS) sel[n_gt + j] = tie[j];
+  __syncthreads();
+  sort_ascending(sel, k);
+  for (int i = tid; i < k; i += TK_THREADS) write_expanded(out, i, sel[i], pool, pos);
+}
+
 }  // namespace
 
 int launch_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, int T, int S_max,
-                int pool, int t_begin, int t_count, int k, int32_t* idx, cudaStream_t stream) {
+                int pool, int t_begin, int t_count, int k, int32_t* idx, cudaStream_t stream, const int* row_flag) {
   if (B * t_count == 0) return DSA_OK;
   const int rows = B * t_count;
   static bool attr_set[64] = {};
@@ -276,7 +426,31 @@ int launch_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, 
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   topk_rows_kernel<<<rows, TK_THREADS, TK_DYN_SMEM, stream>>>(scores, ld, ctx_len, T, S_max, pool, t_begin, t_count,
-                                                               k, idx);
+                                                               k, idx, row_flag);
+  return check_launch();
+}
+
+int launch_sample_threshold(const float* samples, int64_t lds, const int32_t* ctx_len, int B, int T, int S_eff,
+                            int pool, int stride, int t_begin, int t_count, int r, int cap, float* tau,
+                            cudaStream_t stream) {
+  if (B * t_count == 0) return DSA_OK;
+  sample_threshold_kernel<<<B * t_count, TK_THREADS, 0, stream>>>(samples, lds, ctx_len, T, S_eff, pool, stride,
+                                                                  t_begin, t_count, r, cap, tau);
+  return check_launch();
+}
+
+int launch_topk_cand(const float2* cand, const int* cnt, int cap, const int32_t* ctx_len, int B, int T, int S_max,
+                     int pool, int t_begin, int t_count, int k, int32_t* idx, int* fail, cudaStream_t stream) {
+  if (B * t_count == 0) return DSA_OK;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaFuncSetAttribute(topk_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TK_DYN_SMEM);
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  topk_cand_kernel<<<B * t_count, TK_THREADS, TK_DYN_SMEM, stream>>>(cand, cnt, cap, ctx_len, T, S_max, pool,
+                                                                     t_begin, t_count, k, idx, fail);
   return check_launch();
 }
 

@@ -138,6 +138,20 @@ def _group_args(pool=1, topk=2048, S=32768, T=32768, B=1, group=4, d_I=128, H_I=
                          Hq=128, d_qk=576, d_v=512, sm_scale=0.04, idx=A), arr
 
 
+def test_index_select_validation(lib):
+    f = lib.dsa_index_select
+
+    def call(k=2048, pool=1, ws=A, wsb=1 << 30, idx=A, S=4096, tc=8):
+        return f(A, A, A, A, 1, 8, S, 64, 128, pool, 0, tc, k, idx, ws, wsb, None, None)
+    assert call(k=0) == UNSUPPORTED
+    assert call(k=4096) == UNSUPPORTED
+    assert call(pool=3) == UNSUPPORTED
+    assert call(idx=None) == INVALID
+    assert call(wsb=100) == WS_SMALL
+    assert call(ws=A + 4) == MISALIGNED
+    assert call(tc=0) == OK                                  # nothing to select
+
+
 def test_paging_validation(lib):
     """A page map is checked before anything is launched: page sizes are powers of two >= 128,
     the table covers the rows the call needs, and pooled indexer keys are never paged."""
@@ -164,17 +178,31 @@ def test_paging_validation(lib):
     assert lib.dsa_group_forward(ctypes.byref(bad), A, 1 << 40, None) == INVALID
 
 
+def _fused_row_bytes(S):
+    """Selection workspace of one query row on the fused path: a full score row (kept for the
+    repair pass), the 1/16 samples, 8192 (score, id) candidates, and tau, count and flag
+    (each piece rounded to 256 bytes)."""
+    r = lambda x: (x + 255) // 256 * 256                    # noqa: E731
+    return r(S * 4) + r((S // 16 + 3) // 4 * 4 * 4) + r(8192 * 8) + 3 * r(4)
+
+
 def test_group_workspace_and_validation(lib):
     args, keep = _group_args()
+    args.full_scores = 1
     one = lib.dsa_group_workspace_size(ctypes.byref(args), 1)
     big = lib.dsa_group_workspace_size(ctypes.byref(args), 1024)
     assert one == 32768 * 4 and big == 1024 * 32768 * 4     # a chunk of fp32 score rows
+    args.full_scores = 0                                    # the default: fused selection
+    one = lib.dsa_group_workspace_size(ctypes.byref(args), 1)
+    assert one == _fused_row_bytes(32768)
+    assert lib.dsa_index_select_workspace_size(1, 1, 32768, 1) == one
+    assert lib.dsa_index_select_workspace_size(1, 1, 32760, 1) == (32760 * 4 + 255) // 256 * 256   # full rows only
     # too small a workspace is refused before any launch
     assert lib.dsa_group_forward(ctypes.byref(args), A, one - 16, None) == WS_SMALL
     bad, keep2 = _group_args(topk=4096)
     assert lib.dsa_group_forward(ctypes.byref(bad), A, 1 << 40, None) == UNSUPPORTED
     pool_args, keep3 = _group_args(pool=4, topk=512, S=1048576, T=8192)
     need = lib.dsa_group_workspace_size(ctypes.byref(pool_args), 1)
-    assert need == (1048576 // 4) * 128 + (1048576 // 4) * 4   # pooled keys + one score row
+    assert need == (1048576 // 4) * 128 + _fused_row_bytes(1048576 // 4)   # pooled keys + one selection row
     odd, keep4 = _group_args(pool=4, topk=512, S=1048574, T=8192)
     assert lib.dsa_group_forward(ctypes.byref(odd), A, 1 << 40, None) == UNSUPPORTED

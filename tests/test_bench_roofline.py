@@ -28,18 +28,18 @@ def test_work_counts_closed_forms():
 
 def test_roofline_prefill_entries():
     wl = W.WORKLOADS["prefill128k"]
-    brk = {"indexer": 89.3, "topk": 30.7, "attn": 451.4,
-           "per_launch": {"indexer_chunk": 11.16, "topk_chunk": 3.84, "attn_layer": 112.85}}
+    brk = {"select": 70.0, "attn": 451.4, "unfused": {"indexer": 89.3, "topk": 30.7},
+           "per_launch": {"select_chunk": 8.75, "attn_layer": 112.85}}
     r = bench.roofline(wl, brk, PK, 16384)
     assert r["kernel"] == "attn" and r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     flops = 128 * 2 * (576 + 512) * bench.selected_pairs(wl)
-    assert r["achieved"] == pytest.approx(flops / 112.85e-3 / 1e12)
+    assert r["achieved"] == pytest.approx(4 * flops / 451.4e-3 / 1e12)
     assert r["peak"] == 1382.4 and r["frac"] == pytest.approx(r["achieved"] / 1382.4)
     assert r["traffic"] == pytest.approx(bench.TRAFFIC_PER_QUERY[("prefill128k", "attn")] * wl.B * wl.T)
-    ix, tk = r["others"]["indexer"], r["others"]["topk"]
+    sel, ix, tk = r["others"]["select"], r["others"]["indexer_unfused"], r["others"]["topk_unfused"]
+    assert sel["achieved"] == pytest.approx(2 * 64 * 128 * bench.causal_pairs(wl) / 70.0e-3 / 1e12)
+    assert sel["peak"] == pytest.approx(2 * 1382.4)
     assert ix["achieved"] == pytest.approx(2 * 64 * 128 * bench.causal_pairs(wl) / 89.3e-3 / 1e12)
-    assert ix["peak"] == pytest.approx(2 * 1382.4)
-    assert ix["traffic"] is None   # the indexer changed after the traffic capture
     assert tk["bound"] == "hbm"
     assert tk["achieved"] == pytest.approx((4 * bench.causal_pairs(wl) + 4 * wl.T * 2048) / 30.7e-3 / 1e9)
     assert tk["frac"] == pytest.approx(tk["achieved"] / 6535.7)
@@ -47,10 +47,22 @@ def test_roofline_prefill_entries():
 
 def test_roofline_decode_is_hbm_bound():
     wl = W.WORKLOADS["decode256k"]
-    brk = {"indexer": 0.186, "topk": 0.079, "attn": 0.218,
-           "per_launch": {"indexer_chunk": 0.186, "topk_chunk": 0.079, "attn_layer": 0.0545}}
+    brk = {"select": 0.25, "attn": 0.218, "per_launch": {"select_chunk": 0.25, "attn_layer": 0.0545}}
     r = bench.roofline(wl, brk, PK, 1)
-    assert r["kernel"] == "attn" and r["bound"] == "hbm" and r["unit"] == "GB/s"
-    assert r["achieved"] == pytest.approx(bench.attn_bytes(wl) / 0.0545e-3 / 1e9)
-    assert r["traffic"] is None                        # no capture at this context
-    assert r["others"]["indexer"]["bound"] == "hbm"
+    assert r["kernel"] == "select" and r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx((32 * 262144 * 128 + 32 * 64 * 132) / 0.25e-3 / 1e9)
+    a = r["others"]["attn"]
+    assert a["bound"] == "hbm" and a["achieved"] == pytest.approx(4 * bench.attn_bytes(wl) / 0.218e-3 / 1e9)
+    assert r["traffic"] is None and a["traffic"] is None          # no capture at this context
+
+
+def test_roofline_sums_the_work_of_shards():
+    """A rank's shards (zig-zag chunks) add up: two halves give the whole workload's figures."""
+    wl = W.WORKLOADS["prefill32k"]
+    boxes = [(0, 1, 0, wl.T // 2), (0, 1, wl.T // 2, wl.T)]
+    halves = [bench.box_workload(wl, b) for b in boxes]
+    assert sum(bench.causal_pairs(h) for h in halves) == bench.causal_pairs(wl)
+    assert sum(bench.selected_pairs(h) for h in halves) == bench.selected_pairs(wl)
+    brk = {"select": 10.0, "attn": 40.0, "per_launch": {"select_chunk": 5.0, "attn_layer": 5.0}}
+    assert bench.roofline(halves, brk, PK, 16384)["achieved"] == pytest.approx(
+        bench.roofline(wl, brk, PK, 16384)["achieved"])

@@ -68,9 +68,12 @@ class Buf:
 class Cta:
     """One persistent CTA serving `items` (key tiles per item; 0 = nothing visible)."""
 
-    def __init__(self, items, seed, mistakes=()):
+    def __init__(self, items, seed, mistakes=(), abort_at=None):
         self.rng = random.Random(seed)
         self.items, self.mk = items, set(mistakes)
+        # abort_at: the scheduling step at which some bounded wait gives up (None: never); from
+        # then on every wait returns "failed" and each role takes its exit path
+        self.abort_at, self.aborted = abort_at, False
         self.q = {"tma": [], "tc": []}
         acc_empty = E - 1 if "acc_empty_count" in self.mk else E
         b_empty = E if "b_empty_without_mma" in self.mk else E + 1
@@ -83,6 +86,7 @@ class Cta:
             self.bar[f"b_empty{s}"] = Bar(f"b_empty{s}", b_empty)
             self.bar[f"acc_full{s}"] = Bar(f"acc_full{s}", 1)
             self.bar[f"acc_empty{s}"] = Bar(f"acc_empty{s}", acc_empty)
+        self.bar["mma_drain"] = Bar("mma_drain", 1)
         self.buf = {n: Buf(n) for n in [f"A{s}" for s in range(NA)] + ["B0", "B1", "acc0", "acc1"]}
 
     def work(self):
@@ -94,9 +98,12 @@ class Cta:
     def producer(self):
         B, R = self.bar, self.buf
         a_cnt = b_cnt = 0
+        ok = True
         for it, nt in self.work():
             bs = b_cnt & 1
-            yield ("wait", B[f"b_empty{bs}"], self.bpar(b_cnt) ^ 1)
+            ok = yield ("wait", B[f"b_empty{bs}"], self.bpar(b_cnt) ^ 1)
+            if not ok:
+                break
             B[f"b_full{bs}"].expect_tx(2)                     # the query block and its head weights
 
             def load_b(bs=bs, it=it, nt=nt):
@@ -107,7 +114,9 @@ class Cta:
             for _ in range(nt):
                 s = a_cnt % NA
                 if "no_a_empty_wait" not in self.mk:
-                    yield ("wait", B[f"a_empty{s}"], ((a_cnt // NA) & 1) ^ 1)
+                    ok = yield ("wait", B[f"a_empty{s}"], ((a_cnt // NA) & 1) ^ 1)
+                    if not ok:
+                        break
                 B[f"a_full{s}"].expect_tx(1)
 
                 def load_a(s=s, v=a_cnt):
@@ -115,19 +124,33 @@ class Cta:
                     B[f"a_full{s}"].complete_tx(1)
                 yield ("async", "tma", load_a)
                 a_cnt += 1
+            if not ok:
+                break
+        if "no_tma_drain" not in self.mk:
+            # drain, whether this warp gave up or not: the copies it issued land before it
+            # leaves (bounded waits; after a normal run they have landed long ago)
+            for i in range(max(0, a_cnt - NA), a_cnt):
+                yield ("drain", B[f"a_full{i % NA}"], (i // NA) & 1)
+            for i in range(max(0, b_cnt - 2), b_cnt):
+                yield ("drain", B[f"b_full{i & 1}"], self.bpar(i))
         yield ("done",)
 
     def mma(self):
         B, R = self.bar, self.buf
         a_cnt = b_cnt = acc_cnt = 0
+        ok = True
         for it, nt in self.work():
             bs = b_cnt & 1
-            yield ("wait", B[f"b_full{bs}"], self.bpar(b_cnt))
+            ok = yield ("wait", B[f"b_full{bs}"], self.bpar(b_cnt))
+            if not ok:
+                break
             for _ in range(nt):
                 s, ab = a_cnt % NA, acc_cnt & 1
-                yield ("wait", B[f"a_full{s}"], (a_cnt // NA) & 1)
-                if "no_acc_empty_wait" not in self.mk:
-                    yield ("wait", B[f"acc_empty{ab}"], ((acc_cnt >> 1) & 1) ^ 1)
+                ok = yield ("wait", B[f"a_full{s}"], (a_cnt // NA) & 1)
+                if ok and "no_acc_empty_wait" not in self.mk:
+                    ok = yield ("wait", B[f"acc_empty{ab}"], ((acc_cnt >> 1) & 1) ^ 1)
+                if not ok:
+                    break
 
                 def run(s=s, ab=ab, va=a_cnt, vacc=acc_cnt, bs=bs, it=it):
                     R[f"A{s}"].read(va)
@@ -138,9 +161,16 @@ class Cta:
                 yield ("async", "tc", run)
                 a_cnt += 1
                 acc_cnt += 1
+            if not ok:
+                break
             yield ("async", "tc", lambda bs=bs: B[f"b_empty{bs}"].arrive() if "b_empty_without_mma" not in self.mk
                    else None)
             b_cnt += 1
+        if "no_mma_drain" not in self.mk:
+            # drain, whether this warp gave up or not: a commit completes once every MMA issued
+            # before it has finished (another role may have given up and left MMAs unconsumed)
+            yield ("async", "tc", lambda: B["mma_drain"].arrive())
+            yield ("drain", B["mma_drain"], 0)
         yield ("done",)
 
     def epilogue(self, w):
@@ -148,16 +178,22 @@ class Cta:
         b_cnt = acc_cnt = 0
         for it, nt in self.work():
             bs = b_cnt & 1
-            yield ("wait", B[f"b_full{bs}"], self.bpar(b_cnt))
+            if not (yield ("wait", B[f"b_full{bs}"], self.bpar(b_cnt))):
+                break
             R[f"B{bs}"].read(it)                               # head weights into registers
+            ok = True
             for _ in range(nt):
                 ab = acc_cnt & 1
                 if "no_acc_full_wait" not in self.mk:
-                    yield ("wait", B[f"acc_full{ab}"], (acc_cnt >> 1) & 1)
+                    ok = yield ("wait", B[f"acc_full{ab}"], (acc_cnt >> 1) & 1)
+                    if not ok:
+                        break
                 R[f"acc{ab}"].read(acc_cnt)
                 yield ("step",)                                # loads complete, then the hand-back
                 B[f"acc_empty{ab}"].arrive()
                 acc_cnt += 1
+            if not ok:
+                break
             if "no_b_empty_arrive" not in self.mk:
                 B[f"b_empty{bs}"].arrive()
             b_cnt += 1
@@ -167,9 +203,14 @@ class Cta:
         actors = [[self.producer(), None], [self.mma(), None]] + [[self.epilogue(w), None] for w in range(E)]
         for a in actors:
             a[1] = next(a[0])
-        for _ in range(max_steps):
+        for step in range(max_steps):
+            if self.abort_at is not None and step == self.abort_at:
+                self.aborted = True                            # a bounded wait somewhere gave up
+            # a wait is ready once its phase completed, or (after an abort) at once, failing; a
+            # drain is a bounded wait: it may only succeed, the model requires it to complete
             ready = [("actor", i) for i, (_, op) in enumerate(actors)
-                     if op[0] != "done" and not (op[0] == "wait" and not op[1].ready(op[2]))]
+                     if op[0] != "done" and not (op[0] == "wait" and not (self.aborted or op[1].ready(op[2])))
+                     and not (op[0] == "drain" and not op[1].ready(op[2]))]
             if self.q["tc"]:
                 ready.append(("async", "tc", 0))               # the tensor pipe runs in issue order
             ready += [("async", "tma", n) for n in range(len(self.q["tma"]))]
@@ -177,14 +218,26 @@ class Cta:
                 if all(op[0] == "done" for _, op in actors):
                     return
                 raise Deadlock(str([(op[0], getattr(op[1], "name", "")) for _, op in actors if op[0] != "done"]))
+            if all(op[0] == "done" for _, op in actors) and self.aborted:
+                # every role has left after an abort: the CTA frees TMEM and exits now, so no
+                # copy into shared memory and no MMA may still be in flight
+                if self.q["tc"] or self.q["tma"]:
+                    raise AssertionError(f"exit with {len(self.q['tc'])} MMA and {len(self.q['tma'])} copies in flight")
+                return
             ch = self.rng.choice(ready)
             if ch[0] == "async":
                 self.q[ch[1]].pop(ch[2])()
                 continue
             a = actors[ch[1]]
-            if a[1][0] == "async":
-                self.q[a[1][1]].append(a[1][2])
-            a[1] = next(a[0])
+            op = a[1]
+            if op[0] == "async":
+                self.q[op[1]].append(op[2])
+            res = None
+            if op[0] == "wait":
+                res = op[1].ready(op[2]) and not self.aborted
+            elif op[0] == "drain":
+                res = True
+            a[1] = a[0].send(res)
         raise Deadlock("step limit")
 
 
@@ -207,6 +260,26 @@ def test_protocol_completes_without_races():
 # earlier MMA of the item has read the query block.  The model confirms that it stays safe.)
 def test_b_empty_commit_is_redundant_but_harmless():
     _run_all(mistakes=("b_empty_without_mma",), seeds=5)
+
+
+def _run_aborts(mistakes=(), seeds=10):
+    for items in PATTERNS:
+        for s in range(seeds):
+            rng = random.Random(7 * s + len(items))
+            Cta(items, seed=100 * len(items) + s, mistakes=mistakes, abort_at=rng.randrange(0, 400)).run()
+
+
+def test_abort_path_drains_every_copy_and_mma_before_exit():
+    """A bounded wait gives up at a random point: every role leaves through its exit path, the
+    producer's in-flight copies and the MMA warp's in-flight MMAs complete (bounded drain
+    waits), and nothing is still writing shared memory or TMEM when the CTA frees TMEM."""
+    _run_aborts(seeds=60)
+
+
+@pytest.mark.parametrize("mistake", ["no_mma_drain", "no_tma_drain"])
+def test_abort_path_without_a_drain_is_caught(mistake):
+    with pytest.raises(AssertionError):
+        _run_aborts(mistakes=(mistake,), seeds=25)
 
 
 @pytest.mark.parametrize("mistake", ["acc_empty_count", "b_parity", "no_a_empty_wait",

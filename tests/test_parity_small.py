@@ -416,3 +416,72 @@ def test_paged_bad_page_ids_are_skipped_and_flagged():
     assert (P.to_np(sc[0, 0, 256:512]) == 0).all()          # zero keys score exactly 0
     ref = dsa.dsa_index_scores(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"])
     assert torch.equal(sc[0, 0, :256], ref[0, 0, :256]) and torch.equal(sc[1, 0, :768], ref[1, 0, :768])
+
+
+def _unfused_ids(wl, ind, keys, t_begin=0, t_count=None):
+    tc = wl.T - t_begin if t_count is None else t_count
+    sc = dsa.dsa_index_scores(ind["q_idx"], ind["w"], keys, ind["ctx_len"], pool=wl.pool, t_begin=t_begin,
+                              t_count=tc)
+    return dsa.dsa_topk(sc, ind["ctx_len"], wl.T, keys.shape[1], wl.topk, pool=wl.pool, t_begin=t_begin)
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny", {"T": 4096, "ctx": 16384}),                       # rows with n <= k, n <= 8192 and n > 8192
+    ("prefill32k", {"T": 1024, "ctx": 20480}),                 # the 64-head, 4-query-block indexer
+    ("decode256k", {"B": 4, "ctx": 40960}),                    # one query per sequence
+    ("chunk1m_pool", {"T": 256, "ctx": 65536}),                # pooled blocks, top-512
+])
+def test_fused_selection_equals_full_score_rows_bitwise(name, over):
+    """The fused selection (sampled threshold, candidate append, top-k on the candidates) gives
+    exactly the ids of full score rows + the row top-k, in every row regime: all visible keys
+    kept (n <= k), threshold -inf (n <= 8192 candidates), sampled threshold; and the oracle
+    accepts sampled rows of each regime."""
+    wl = W.WORKLOADS[name].replace(**over)
+    ind, lays = _inputs(wl, layers=1)
+    keys = ind["k_idx"] if wl.pool == 1 else dsa.dsa_index_pool(ind["k_idx"], pool=wl.pool)
+    assert keys.shape[1] % 16 == 0                          # the fused path applies
+    got = dsa.dsa_index_select(ind["q_idx"], ind["w"], keys, ind["ctx_len"], wl.topk, pool=wl.pool)
+    ref = _unfused_ids(wl, ind, keys)
+    assert torch.equal(got, ref)
+    # through the group call too, with a workspace small enough for several query chunks
+    idx, outs = dsa.dsa_group_forward(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk,
+                                      [{"q": lays[0]["q"], "kv": lays[0]["kv"], "v": lays[0]["v"]}], wl.sm_scale,
+                                      wl.d_v, pool=wl.pool, t_chunk=max(1, wl.T // 3))
+    assert torch.equal(idx, ref)
+    kdec = P.Decoded(ind["k_idx"])
+    kpd = P.Decoded(keys) if wl.pool > 1 else None
+    idx_h = P.to_np(idx)
+    for b in sorted({0, wl.B - 1}):
+        for t in sorted({0, wl.T // 2, wl.T - 1}):
+            pos = wl.ctx - wl.T + t
+            msg = P.check_topk_row(idx_h[b, t], P.to_np(ind["q_idx"][b, t]), P.to_np(ind["w"][b, t]), kdec[b], pos,
+                                   wl.topk, wl.pool, kpd[b] if kpd else None)
+            assert msg is None, f"row {(b, t)}: {msg}"
+
+
+def test_fused_selection_repair_when_the_sample_misleads():
+    """Keys at multiples of 16 (exactly the sampled ones) score far above all others, so each
+    row's threshold (the r-th largest sample) is met by only r = 32 < k keys and every long row
+    is redone by the repair pass;
+    an all-tied row overflows the candidate buffer and is redone too.  The ids still equal the
+    full-row selection, and the oracle accepts them."""
+    wl = W.WORKLOADS["tiny"].replace(T=64, ctx=16384, topk=256)
+    ind = W.make_indexer_inputs(wl, device=DEV)
+    v = torch.zeros(wl.d_I, device=DEV)
+    v[:8] = 2.0
+    codes = v.to(torch.float8_e4m3fn).view(torch.uint8)
+    ind["q_idx"][:] = codes                                 # every head of every query looks along v
+    ind["w"].abs_()                                         # positive head weights
+    kf = ind["k_idx"][0, ::16].view(torch.float8_e4m3fn).float()
+    kf[:, :8] += 4.0                                        # the sampled keys align with v (distinct scores)
+    ind["k_idx"][0, ::16] = kf.to(torch.float8_e4m3fn).view(torch.uint8)
+    ind["w"][0, 10] = 0.0                                   # row 10: every score is 0 (all tied)
+    got = dsa.dsa_index_select(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk)
+    ref = _unfused_ids(wl, ind, ind["k_idx"])
+    assert torch.equal(got, ref)
+    assert list(P.to_np(got[0, 10])) == list(range(256))   # all tied: the lowest ids
+    kdec = P.Decoded(ind["k_idx"])
+    for t in (0, 10, 63):
+        msg = P.check_topk_row(P.to_np(got[0, t]), P.to_np(ind["q_idx"][0, t]), P.to_np(ind["w"][0, t]), kdec[0],
+                               wl.ctx - wl.T + t, wl.topk)
+        assert msg is None, f"row {t}: {msg}"
