@@ -68,8 +68,11 @@ class Buf:
 class Cta:
     """One persistent CTA serving `items` (key tiles per item; 0 = nothing visible)."""
 
-    def __init__(self, items, seed, mistakes=(), abort_at=None):
+    def __init__(self, items, seed, mistakes=(), abort_at=None, async_p=None):
         self.rng = random.Random(seed)
+        # async_p: when roles and asynchronous completions are both ready, the chance that a
+        # completion goes next (None: uniform); small values keep copies and MMAs in flight longer
+        self.async_p = async_p
         self.items, self.mk = items, set(mistakes)
         # abort_at: the scheduling step at which some bounded wait gives up (None: never); from
         # then on every wait returns "failed" and each role takes its exit path
@@ -203,7 +206,9 @@ class Cta:
         actors = [[self.producer(), None], [self.mma(), None]] + [[self.epilogue(w), None] for w in range(E)]
         for a in actors:
             a[1] = next(a[0])
+        self.steps = 0
         for step in range(max_steps):
+            self.steps = step
             if self.abort_at is not None and step == self.abort_at:
                 self.aborted = True                            # a bounded wait somewhere gave up
             # a wait is ready once its phase completed, or (after an abort) at once, failing; a
@@ -224,7 +229,11 @@ class Cta:
                 if self.q["tc"] or self.q["tma"]:
                     raise AssertionError(f"exit with {len(self.q['tc'])} MMA and {len(self.q['tma'])} copies in flight")
                 return
-            ch = self.rng.choice(ready)
+            acts = [r for r in ready if r[0] == "actor"]
+            if self.async_p is not None and acts and len(acts) < len(ready) and self.rng.random() >= self.async_p:
+                ch = self.rng.choice(acts)
+            else:
+                ch = self.rng.choice(ready)
             if ch[0] == "async":
                 self.q[ch[1]].pop(ch[2])()
                 continue
@@ -265,8 +274,11 @@ def test_b_empty_commit_is_redundant_but_harmless():
 def _run_aborts(mistakes=(), seeds=10):
     for items in PATTERNS:
         for s in range(seeds):
+            full = Cta(items, seed=100 * len(items) + s)
+            full.run()                                 # how long the run takes without a timeout
             rng = random.Random(7 * s + len(items))
-            Cta(items, seed=100 * len(items) + s, mistakes=mistakes, abort_at=rng.randrange(0, 400)).run()
+            Cta(items, seed=100 * len(items) + s, mistakes=mistakes,
+                abort_at=rng.randrange(0, max(1, full.steps)), async_p=0.05).run()
 
 
 def test_abort_path_drains_every_copy_and_mma_before_exit():
