@@ -33,7 +33,8 @@
 //              partial with its lse).
 //   warps 8-10 gather: 16-byte cp.async of the selected rows into the 128-byte-swizzled
 //              K-major layout the tensor core reads (also V's MN-major layout).
-//   warp 11    TMEM owner and MMA issuer: S_0, S_1, then per tile S_{j+2} ahead of P_j.V_j.
+//   warp 11    TMEM owner and MMA issuer: S_0, S_1, then per tile the first K-steps of S_{j+2},
+//              then P_j.V_j interleaved with its other K-steps.
 // Persistent: one cluster per two SMs serves work items (query, key split) in turn, and every
 // barrier phase counts tiles over all its items.  At an item boundary the next query's q
 // (prefetched to L2 an item earlier) goes into TMEM before the previous query's O is read out,
@@ -56,6 +57,7 @@ constexpr int NS = 4;                   // key-tile stages
 constexpr int BLKS = 5;                 // 64-column blocks of a key row held per CTA
 constexpr int K_BLK = NK * 128;         // 64 rows x 128 B
 constexpr int KSTEPS = 18;              // 288 score columns / 16 per MMA
+constexpr int S_EARLY = 9;              // K-steps of S_{j+2} issued before P_j.V_j is interleaved
 constexpr int KV_STAGE = BLKS * K_BLK;                 // 40960
 constexpr int OFF_KV = 0;
 constexpr int SMW = 8;                  // softmax warps: 2 per SM sub-partition, 16 heads each
@@ -456,27 +458,43 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     cp_async_wait<0>();
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
-    // Order: S_0, S_1, then for each tile j: S_{j+2} (as soon as the softmax has read S_{j+1})
-    // ahead of P_j.V_j (once P_j is in TMEM), so the next tile's scores are always ready when
-    // the softmax asks for them.  The key ring holds tiles j .. j+2 meanwhile.
+    // Order: S_0, S_1, then for each tile j: the first S_EARLY K-steps of S_{j+2} (as soon as the
+    // softmax has read S_{j+1}), then -- once P_j is in TMEM -- P_j.V_j interleaved with the other
+    // K-steps of S_{j+2}.  The tensor pipe runs the 64-key score MMAs and the MN-major P.V MMAs
+    // side by side when they alternate, and the early K-steps cover the softmax's second half, so
+    // the next tile's scores are ready when the softmax asks for them.  The key ring holds tiles
+    // j .. j+2 meanwhile.
     bool ok = true;
     const int ks0 = half * KSTEPS;
-    auto issue_s = [&](uint32_t gg) -> bool {
-      const int st = gg % NS;
-      if (!mbar_wait_warp(kv_full(st), (gg / NS) & 1, abort, kWaitLimitNs)) return false;
+    // K-steps i0 .. i1-1 of S_gg (lane 0)
+    auto s_steps = [&](uint32_t gg, int i0, int i1) {
+      const uint32_t stage = sbase + OFF_KV + (gg % NS) * KV_STAGE;
+      for (int i = i0; i < i1; ++i) {
+        const int ks = ks0 + i;                      // global 16-column step 0..35
+        const uint32_t blk = (uint32_t)((ks >> 2) - blk0);
+        const uint32_t off = (uint32_t)(ks & 3) * 32u;   // 16 columns = 32 bytes inside the atom
+        const uint64_t bd = smem_desc(stage + blk * K_BLK + off, 1024, kLayoutSw128);
+        mma_bf16_ts(tmem + COL_S, tmem + COL_Q + 8u * i, bd, IDESC_S, i > 0 ? 1u : 0u);
+      }
+    };
+    // keys 16kk .. 16kk+15 of P_gg.V_gg (lane 0); V columns 256*half .. +255 are the stage's
+    // blocks 0..3 for both CTAs
+    auto pv_step = [&](uint32_t gg, bool first, int kk) {
+      const uint32_t stage = sbase + OFF_KV + (gg % NS) * KV_STAGE;
+      const uint64_t bd = smem_desc_lbo(stage + kk * 2048, K_BLK, 1024, kLayoutSw128);
+      mma_bf16_ts(tmem + COL_O, tmem + COL_P + 8u * kk, bd, IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+    };
+    auto wait_s = [&](uint32_t gg) -> bool {
+      if (!mbar_wait_warp(kv_full(gg % NS), (gg / NS) & 1, abort, kWaitLimitNs)) return false;
       if (!mbar_wait_warp(s_empty, (gg & 1) ^ 1, abort, kWaitLimitNs)) return false;
       tc_fence_after();
       fence_proxy_async();
+      return true;
+    };
+    auto issue_s = [&](uint32_t gg) -> bool {
+      if (!wait_s(gg)) return false;
       if (lane == 0) {
-        const uint32_t stage = sbase + OFF_KV + st * KV_STAGE;
-#pragma unroll 2
-        for (int i = 0; i < KSTEPS; ++i) {
-          const int ks = ks0 + i;                      // global 16-column step 0..35
-          const uint32_t blk = (uint32_t)((ks >> 2) - blk0);
-          const uint32_t off = (uint32_t)(ks & 3) * 32u;   // 16 columns = 32 bytes inside the atom
-          const uint64_t bd = smem_desc(stage + blk * K_BLK + off, 1024, kLayoutSw128);
-          mma_bf16_ts(tmem + COL_S, tmem + COL_Q + 8u * i, bd, IDESC_S, i > 0 ? 1u : 0u);
-        }
+        s_steps(gg, 0, KSTEPS);
         mma_commit(s_full);
       }
       __syncwarp();
@@ -486,15 +504,30 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       if (!mbar_wait_warp(p_full, gg & 1, abort, kWaitLimitNs)) return false;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t stage = sbase + OFF_KV + (gg % NS) * KV_STAGE;
 #pragma unroll
-        for (int kk = 0; kk < NK / 16; ++kk) {
-          // V columns 256*half .. +255 are the stage's blocks 0..3 for both CTAs; keys 16kk..
-          const uint64_t bd = smem_desc_lbo(stage + kk * 2048, K_BLK, 1024, kLayoutSw128);
-          mma_bf16_ts(tmem + COL_O, tmem + COL_P + 8u * kk, bd, IDESC_PV, (!first || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < NK / 16; ++kk) pv_step(gg, first, kk);
         mma_commit(kv_empty(gg % NS));
         mma_commit(pv_done);
+      }
+      __syncwarp();
+      return true;
+    };
+    auto issue_s_pv = [&](uint32_t gs, uint32_t gpv, bool first) -> bool {
+      if (!wait_s(gs)) return false;
+      if (lane == 0) s_steps(gs, 0, S_EARLY);
+      __syncwarp();
+      if (!mbar_wait_warp(p_full, gpv & 1, abort, kWaitLimitNs)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+#pragma unroll
+        for (int kk = 0; kk < NK / 16; ++kk) {
+          s_steps(gs, S_EARLY + kk, S_EARLY + kk + 1);
+          pv_step(gpv, first, kk);
+        }
+        mma_commit(kv_empty(gpv % NS));   // both complete once every MMA issued so far has
+        mma_commit(pv_done);
+        s_steps(gs, S_EARLY + NK / 16, KSTEPS);
+        mma_commit(s_full);
       }
       __syncwarp();
       return true;
@@ -507,10 +540,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       ++nq;
       ok = issue_s(g);
       if (ok && I.ntiles > 1) ok = issue_s(g + 1);
-      for (int j = 0; j < I.ntiles && ok; ++j) {
-        if (j + 2 < I.ntiles && !(ok = issue_s(g + j + 2))) break;
-        ok = issue_pv(g + j, j == 0);
-      }
+      for (int j = 0; j < I.ntiles && ok; ++j)
+        ok = j + 2 < I.ntiles ? issue_s_pv(g + j + 2, g + j, j == 0) : issue_pv(g + j, j == 0);
       g += I.ntiles;
     }
     // every MMA this warp issued must have finished before the TMEM is freed: after a normal
