@@ -78,6 +78,7 @@ _SIGS = {
     "dsa_launch_count": (ctypes.c_uint64, []),
     "dsa_device_status": (_c_int, [_c_p]),
     "dsa_debug_wait_timeout": (_c_int, [ctypes.c_uint64, _c_p]),
+    "dsa_debug_set_wait_limit": (_c_int, [ctypes.c_uint64]),
     "dsa_index_scores": (_c_int, [_c_p, _c_p, _c_p, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                   _c_int, _c_int, _c_p, _c_i64, ctypes.POINTER(Paging), _c_p]),
     "dsa_topk": (_c_int, [_c_p, _c_i64, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p]),
@@ -175,6 +176,11 @@ def dsa_device_status(stream=None) -> int:
     (DSA_ERR_TIMEOUT) when a bounded device wait gave up, or 7 (DSA_ERR_INDEX_RANGE) when an
     attention call met a selected id beyond its cache and skipped it."""
     return int(_lib().dsa_device_status(_stream(stream)))
+
+
+def dsa_debug_set_wait_limit(limit_ns: int) -> None:
+    """Time limit of the real kernels' bounded waits (1 us .. 2 s; 0 = the default 2 s)."""
+    _check("dsa_debug_set_wait_limit", _lib().dsa_debug_set_wait_limit(int(limit_ns)))
 
 
 def dsa_debug_wait_timeout(limit_ns: int, stream=None) -> None:

@@ -270,6 +270,19 @@ int dsa_device_status(void* stream) {
 }
 uint64_t dsa_launch_count(void) { return g_launches; }
 
+int dsa_debug_set_wait_limit(uint64_t limit_ns) {
+  if (limit_ns != 0 && (limit_ns < 1000ull || limit_ns > 2000000000ull)) return DSA_ERR_INVALID_ARG;
+  const uint64_t v = limit_ns == 0 ? 2000000000ull : limit_ns;
+  indexer_set_wait_limit(v);
+  attn_tc_set_wait_limit(v);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_cuda_error(e);
+    return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
+}
+
 int dsa_debug_wait_timeout(uint64_t limit_ns, void* stream) {
   if (limit_ns == 0 || limit_ns > 1000000000ull) return DSA_ERR_INVALID_ARG;
   return launch_wait_timeout_probe(limit_ns, static_cast<cudaStream_t>(stream));

@@ -80,7 +80,6 @@ constexpr uint32_t COL_S = 0;      // partial scores, NK columns
 constexpr uint32_t COL_Q = 64;     // this CTA's 288 q columns as packed bf16 pairs: 144 columns
 constexpr uint32_t COL_P = 224;    // P of one tile as packed bf16 pairs (the P.V MMA's A operand): 32 columns
 constexpr uint32_t COL_O = 256;    // DVH output columns
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;
 
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -190,12 +189,13 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 // Bounded wait on a local barrier that the partner CTA completes (cluster-scope acquire).
 __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t limit = *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((it & 31u) == 0u) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit) {
         *abort = 1;
         atomicOr(&g_status, 1u);
         return false;
@@ -808,6 +808,11 @@ int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, i
   int st = check_launch();
   if (st != DSA_OK || splits == 1) return st;
   return launch_attn_combine(part_o, part_lse, splits, rows, DV, out, lse, stream);
+}
+
+void attn_tc_set_wait_limit(uint64_t ns) {
+  const unsigned long long v = ns;
+  cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v));
 }
 
 unsigned int attn_tc_take_status() {

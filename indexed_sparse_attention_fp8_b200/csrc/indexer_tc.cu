@@ -34,7 +34,6 @@ constexpr int KTILE = 128;        // keys per tile (MMA M)
 constexpr int KC = 32;            // key tiles per work item
 constexpr int NA = 6;             // key-tile stages
 constexpr int NUM_THREADS = 320;  // 10 warps
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: no legal wait comes close
 
 template <int H, int D, int QB>
 struct IdxCfg {
@@ -573,6 +572,11 @@ __global__ void wait_timeout_probe_kernel(uint64_t limit_ns) {
 int launch_wait_timeout_probe(uint64_t limit_ns, cudaStream_t stream) {
   wait_timeout_probe_kernel<<<1, 1, 0, stream>>>(limit_ns);
   return check_launch();
+}
+
+void indexer_set_wait_limit(uint64_t ns) {
+  const unsigned long long v = ns;
+  cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v));
 }
 
 // Reads and clears the indexer's device status word (bit 0: a bounded wait gave up).

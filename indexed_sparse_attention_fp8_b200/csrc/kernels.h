@@ -65,6 +65,9 @@ unsigned int pool_take_status();
 
 // Reads and clears the device status word of the tensor-core indexer.
 unsigned int indexer_take_status();
+// Time limit of the bounded waits in the tensor-core indexer / attention (test hook).
+void indexer_set_wait_limit(uint64_t ns);
+void attn_tc_set_wait_limit(uint64_t ns);
 // Launches the bounded-wait probe (see dsa_debug_wait_timeout).
 int launch_wait_timeout_probe(uint64_t limit_ns, cudaStream_t stream);
 

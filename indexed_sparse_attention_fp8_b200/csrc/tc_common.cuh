@@ -18,6 +18,14 @@ namespace tc {
 // length.  One word per translation unit that includes this header.
 static __device__ unsigned int g_status;
 
+// Time limit of the kernels' bounded waits (2 s: no legal wait comes close).  A test hook may
+// shorten it (dsa_debug_set_wait_limit) to make the real kernels' waits run out; waits read it
+// only once their first try has failed.  One copy per translation unit.
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+static __device__ unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
+// The limit a wait passes to mbar_wait to use g_wait_limit_ns.
+constexpr uint64_t kWaitLimitNs = 0;
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -64,11 +72,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after limit_ns of
-// waiting, or as soon as another role of the CTA raised *abort: then sets *abort and the
+// waiting (0: the kernels' wait limit g_wait_limit_ns), or as soon as another role of the CTA raised *abort: then sets *abort and the
 // device status word and returns false.  Never spins without bound.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
+  if (limit_ns == 0) limit_ns = *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;

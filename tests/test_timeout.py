@@ -27,3 +27,39 @@ def test_timeout_probe_rejects_bad_limits():
         dsa.dsa_debug_wait_timeout(0)
     with pytest.raises(dsa.DSAError):
         dsa.dsa_debug_wait_timeout(5_000_000_000)
+
+
+def test_real_kernels_give_up_their_waits_drain_and_recover():
+    """With the wait limit of the real kernels cut to 2 us, the tensor-core indexer's and the MLA
+    attention's waits run out: each launch sets the status word, drains its copies and MMAs,
+    frees TMEM and returns, and dsa_device_status() reports DSA_ERR_TIMEOUT.  With the default
+    limit restored, the same calls give exactly the results they gave before."""
+    wl = W.WORKLOADS["prefill32k"].replace(T=256, ctx=4096)
+    ind = W.make_indexer_inputs(wl, device="cuda")
+    lay = W.make_attn_inputs(wl, 0, device="cuda")
+    g = torch.Generator(device="cpu").manual_seed(3)
+    idx = torch.stack([torch.randperm(4096 - 256, generator=g)[: wl.topk] for _ in range(wl.T)]).to(torch.int32)
+    idx = idx.view(1, wl.T, wl.topk).cuda()
+    ref_sc = dsa.dsa_index_scores(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"])
+    ref_o, ref_l = dsa.dsa_sparse_attn(lay["q"], lay["kv"], idx, wl.sm_scale, wl.d_v, want_lse=True)
+    assert dsa.dsa_device_status() == 0
+    dsa.dsa_debug_set_wait_limit(2000)
+    try:
+        dsa.dsa_index_scores(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"])
+        st_indexer = dsa.dsa_device_status()
+        dsa.dsa_sparse_attn(lay["q"], lay["kv"], idx, wl.sm_scale, wl.d_v, want_lse=True)
+        st_attn = dsa.dsa_device_status()
+    finally:
+        dsa.dsa_debug_set_wait_limit(0)
+    assert st_indexer == 6 and st_attn == 6                  # DSA_ERR_TIMEOUT from each kernel
+    sc = dsa.dsa_index_scores(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"])
+    o, l = dsa.dsa_sparse_attn(lay["q"], lay["kv"], idx, wl.sm_scale, wl.d_v, want_lse=True)
+    assert dsa.dsa_device_status() == 0
+    assert torch.equal(sc, ref_sc) and torch.equal(o, ref_o) and torch.equal(l, ref_l)
+
+
+def test_wait_limit_hook_rejects_bad_limits():
+    with pytest.raises(dsa.DSAError):
+        dsa.dsa_debug_set_wait_limit(10)                     # below 1 us
+    with pytest.raises(dsa.DSAError):
+        dsa.dsa_debug_set_wait_limit(5_000_000_000)          # above 2 s
