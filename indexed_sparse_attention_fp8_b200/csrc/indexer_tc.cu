@@ -56,7 +56,12 @@ struct IdxCfg {
   static constexpr int OFF_BAR = OFF_W + 2 * W_BYTES;
   static constexpr int NBAR = 2 * NA + 9;           // + the MMA drain barrier
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
+  // fused selection (64-head shape): per epilogue warp and query, a staging buffer of CB
+  // candidates, so the global slots are reserved with one atomic per flush, not per tile
+  static constexpr int CB = 64;
+  static constexpr int OFF_CBUF = (OFF_MISC + 16 + 15) / 16 * 16;
+  static constexpr int CBUF_BYTES = H == 64 ? 8 * QPH * CB * 8 : 0;
+  static constexpr int SMEM = OFF_CBUF + CBUF_BYTES + 1024;  // + alignment slack
   static_assert(D == 128 || D == 64, "row = one swizzle atom");
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
   static_assert(COLS % 32 == 0 && (COLS % H == 0 || H % COLS == 0), "epilogue split");
@@ -315,10 +320,31 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
           lim[ql] = pos < 0 ? -1 : pos / pool;   // s * pool <= pos  <=>  s <= pos / pool
           if constexpr (CAND) qtau[ql] = qok[ql] ? __ldg(tau + qr[ql]) : INFINITY;
         }
+        // fused selection: the warp's candidates of each query wait in shared memory (scnt of
+        // them, a warp-uniform count) and go out in one flush: one atomic reserves their slots
+        float2* cb = reinterpret_cast<float2*>(sgen + C::OFF_CBUF) + (warp - 2) * C::QPH * C::CB;
+        int scnt[C::QPH];
+#pragma unroll
+        for (int ql = 0; ql < C::QPH; ++ql) scnt[ql] = 0;
+        auto flush = [&](int ql) {
+          __syncwarp();
+          int base = 0;
+          if (lane == 0 && scnt[ql] > 0) base = atomicAdd(cnt + qr[ql], scnt[ql]);
+          base = __shfl_sync(0xffffffffu, base, 0);
+          for (int i = lane; i < scnt[ql]; i += 32)
+            if (base + i < cap) cand[qr[ql] * cap + base + i] = cb[ql * C::CB + i];
+          __syncwarp();
+          scnt[ql] = 0;
+        };
         auto store = [&](int ql, int s, float val) {
           if constexpr (CAND) {
-            cand_append(qok[ql] && s < S_max && s <= lim[ql] && val >= qtau[ql], val, s, cnt + qr[ql],
-                        cand + qr[ql] * cap, cap);
+            const bool pass = qok[ql] && s < S_max && s <= lim[ql] && val >= qtau[ql];
+            const unsigned m = __ballot_sync(0xffffffffu, pass);
+            if (m != 0u) {
+              if (pass) cb[ql * C::CB + scnt[ql] + __popc(m & ((1u << lane) - 1u))] = make_float2(val, __int_as_float(s));
+              scnt[ql] += __popc(m);
+              if (scnt[ql] > C::CB - 32) flush(ql);   // room for a full warp's worth stays
+            }
           } else {
             if (qok[ql] && s < S_max) qrow[ql][s] = (s <= lim[ql]) ? val : -INFINITY;
           }
@@ -391,6 +417,12 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
           if (more) {
             tmem_ld_wait();
             launder(v[0]);
+          }
+        }
+        if constexpr (CAND) {
+          if (ok) {
+#pragma unroll
+            for (int ql = 0; ql < C::QPH; ++ql) flush(ql);
           }
         }
       } else {

@@ -32,10 +32,13 @@ def _t_chunk(wl):
 
 
 def _sample_rows(wl, n_random=3):
+    """Query rows checked against the oracle: every sequence of a decode batch (one row each), and
+    for prefill the first rows, both sides of the 128-row tile edge, the middle, the last rows and
+    a few random ones."""
     rng = np.random.default_rng(wl.seed + 77)
     ts = sorted({0, 1, min(127, wl.T - 1), min(128, wl.T - 1), wl.T // 2, wl.T - 2, wl.T - 1,
                  *[int(x) for x in rng.integers(0, wl.T, n_random)]})
-    bs = sorted({0, wl.B - 1, int(rng.integers(0, wl.B))})
+    bs = list(range(wl.B)) if wl.T == 1 else sorted({0, wl.B - 1, int(rng.integers(0, wl.B))})
     return [(b, t) for b in bs for t in ts if 0 <= t < wl.T]
 
 
