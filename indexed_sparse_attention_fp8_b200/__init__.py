@@ -179,7 +179,7 @@ def dsa_device_status(stream=None) -> int:
 
 
 def dsa_debug_set_wait_limit(limit_ns: int) -> None:
-    """Time limit of the real kernels' bounded waits (1 us .. 2 s; 0 = the default 2 s)."""
+    """Time limit of the real kernels' bounded waits (1 ns .. 2 s; 0 = the default 2 s)."""
     _check("dsa_debug_set_wait_limit", _lib().dsa_debug_set_wait_limit(int(limit_ns)))
 
 

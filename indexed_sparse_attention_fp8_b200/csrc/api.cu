@@ -271,7 +271,7 @@ int dsa_device_status(void* stream) {
 uint64_t dsa_launch_count(void) { return g_launches; }
 
 int dsa_debug_set_wait_limit(uint64_t limit_ns) {
-  if (limit_ns != 0 && (limit_ns < 1000ull || limit_ns > 2000000000ull)) return DSA_ERR_INVALID_ARG;
+  if (limit_ns > 2000000000ull) return DSA_ERR_INVALID_ARG;
   const uint64_t v = limit_ns == 0 ? 2000000000ull : limit_ns;
   indexer_set_wait_limit(v);
   attn_tc_set_wait_limit(v);
