@@ -83,7 +83,8 @@ int dsa_debug_wait_timeout(uint64_t limit_ns, void* stream);
 
 /* Test hook for the real kernels' failure paths: sets the time limit of every bounded wait in
  * the tensor-core indexer and attention kernels on the current device (1 ns .. 2 s; 0 restores
- * the default of 2 s; at 1 ns every wait that is not ready within its first tries gives up).  Synchronous (a copy to device memory); calls whose kernels are in flight
+ * the default of 2 s; below 1 us, every wait that is not ready at its first non-blocking check
+ * gives up at once).  Synchronous (a copy to device memory); calls whose kernels are in flight
  * keep the limit they read.  With a limit shorter than a normal wait, a launch gives up early,
  * drains its copies and MMAs, frees TMEM and returns: dsa_device_status() then returns
  * DSA_ERR_TIMEOUT and that launch's outputs are incomplete; the context stays usable. */

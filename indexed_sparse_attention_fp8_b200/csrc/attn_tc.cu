@@ -175,6 +175,17 @@ __device__ __forceinline__ void mbar_arrive_cluster_after(uint32_t cluster_bar, 
                "mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];\n\t}\n" ::"r"(cluster_bar), "f"(dep)
                : "memory");
 }
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -188,8 +199,13 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 }
 // Bounded wait on a local barrier that the partner CTA completes (cluster-scope acquire).
 __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
+  if (mbar_test_wait_cluster(bar, parity)) return true;
   const uint64_t limit = *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+  if (limit < kImmediateNs) {
+    *abort = 1;
+    atomicOr(&g_status, 1u);
+    return false;
+  }
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_cluster(bar, parity)) return true;

@@ -30,8 +30,9 @@ def test_timeout_probe_rejects_bad_limits():
 
 
 def test_real_kernels_give_up_their_waits_drain_and_recover():
-    """With the wait limit of the real kernels cut to 1 ns (every wait that is not ready within its
-    first tries gives up), the tensor-core indexer's and the MLA attention's waits run out: each launch sets the status word, drains its copies and MMAs,
+    """With the wait limit of the real kernels cut to 1 ns (every wait that is not ready at its first
+    non-blocking check gives up at once), the tensor-core indexer's and the MLA attention's waits
+    run out: each launch sets the status word, drains its copies and MMAs,
     frees TMEM and returns, and dsa_device_status() reports DSA_ERR_TIMEOUT.  With the default
     limit restored, the same calls give exactly the results they gave before."""
     wl = W.WORKLOADS["prefill32k"].replace(T=256, ctx=4096)
@@ -40,7 +41,14 @@ def test_real_kernels_give_up_their_waits_drain_and_recover():
     g = torch.Generator(device="cpu").manual_seed(3)
     idx = torch.stack([torch.randperm(4096 - 256, generator=g)[: wl.topk] for _ in range(wl.T)]).to(torch.int32)
     idx = idx.view(1, wl.T, wl.topk).cuda()
-    ref_sc = dsa.dsa_index_scores(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"])
+    # score entries past a row's last visible key tile are not written: both calls start from
+    # the same sentinel so the comparison covers exactly what the indexer writes
+    S = ind["k_idx"].shape[1]
+
+    def scores():
+        sc = torch.full((1, wl.T, S), 12345.0, dtype=torch.float32, device="cuda")
+        return dsa.dsa_index_scores(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], scores=sc)
+    ref_sc = scores()
     ref_o, ref_l = dsa.dsa_sparse_attn(lay["q"], lay["kv"], idx, wl.sm_scale, wl.d_v, want_lse=True)
     assert dsa.dsa_device_status() == 0
     dsa.dsa_debug_set_wait_limit(1)
@@ -52,7 +60,7 @@ def test_real_kernels_give_up_their_waits_drain_and_recover():
     finally:
         dsa.dsa_debug_set_wait_limit(0)
     assert st_indexer == 6 and st_attn == 6                  # DSA_ERR_TIMEOUT from each kernel
-    sc = dsa.dsa_index_scores(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"])
+    sc = scores()
     o, l = dsa.dsa_sparse_attn(lay["q"], lay["kv"], idx, wl.sm_scale, wl.d_v, want_lse=True)
     assert dsa.dsa_device_status() == 0
     assert torch.equal(sc, ref_sc) and torch.equal(o, ref_o) and torch.equal(l, ref_l)
