@@ -71,10 +71,20 @@ constexpr int NBARS = 3 * NS + 6 + 2 * SMW;            // .. + s_full, s_empty, 
                                                        //    drain; x_full and x_free per softmax warp
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;       // + alignment slack
-constexpr int THREADS = 384;            // 12 warps, so up to 168 registers
-constexpr int GATHER_WARP0 = SMW;       // warps 8..10
-constexpr int GATHER_THREADS = 96;
-constexpr int MMA_WARP = 11;
+// Five warpgroups: 0-1 softmax (warps 0-7), 2 the MMA warp (8) and gather warps 9-11, 3-4 gather
+// warps 12-19.  A tile's gather is bound by how many rows are in flight at once, not by its bytes,
+// so it takes many warps; they need few registers, and the softmax warps many: the kernel starts
+// at REGS_LAUNCH per thread, warpgroup 2 drops to REGS_MID, 3-4 to REGS_LOW, and 0-1 rise to
+// REGS_HIGH, within the registers the block was launched with.
+constexpr int THREADS = 640;
+constexpr int MMA_WARP = SMW;           // warp 8
+constexpr int GATHER_WARP0 = SMW + 1;   // warps 9..19
+constexpr int GATHER_WARPS = THREADS / 32 - GATHER_WARP0;
+constexpr int GATHER_THREADS = GATHER_WARPS * 32;
+constexpr int REGS_LAUNCH = 96, REGS_MID = 72, REGS_LOW = 48, REGS_HIGH = 152;
+static_assert(THREADS == 5 * 128, "warpgroup roles");
+static_assert(2 * 128 * REGS_HIGH + 128 * REGS_MID + 2 * 128 * REGS_LOW <= THREADS * REGS_LAUNCH, "register split");
+static_assert(THREADS * REGS_LAUNCH <= 65536, "register file");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_S = 0;      // partial scores, NK columns
 constexpr uint32_t COL_Q = 64;     // this CTA's 288 q columns as packed bf16 pairs: 144 columns
@@ -231,9 +241,8 @@ __device__ __forceinline__ void cluster_sync() {
 // This CTA's q columns of the query into TMEM (bf16 pairs packed per 32-bit column), then this
 // warp's arrival on q_ready.  Warps w and w+4 share the TMEM lane quadrant w%4: each writes all
 // 32 of its heads (32x32b shape, thread = head), warp w the first 144 of the CTA's 288 q
-// columns and warp w+4 the other 144.  Out of line: it runs once per query, and inlined its
-// registers would crowd the per-tile loop.
-__device__ __noinline__ void attn_load_q(const __nv_bfloat16* __restrict__ q, int bt, int quad, int hh, int half,
+// columns and warp w+4 the other 144.
+__device__ __forceinline__ void attn_load_q(const __nv_bfloat16* __restrict__ q, int bt, int quad, int hh, int half,
                                          uint32_t tmem, uint32_t q_ready, int lane) {
   const int head = 32 * quad + lane;
   const uint4* qsrc = reinterpret_cast<const uint4*>(q + ((int64_t)bt * HQ + head) * DQK + 288 * half + 144 * hh);
@@ -260,9 +269,8 @@ __device__ __noinline__ void attn_load_q(const __nv_bfloat16* __restrict__ q, in
 
 // Epilogue of one item for this warp's 16 heads: waits for its last P.V, finishes the row sums
 // over the quad, then O / l (or the split partial and its lse) out of TMEM in the 16x256b shape:
-// per 64-column chunk, thread i writes columns 8r + 2*(i%4), +1 of its two heads.  Out of line
-// for the same reason as attn_load_q.
-__device__ __noinline__ bool attn_epilogue(int bt, int sp, int ntiles, float m0, float m1, float l0, float l1,
+// per 64-column chunk, thread i writes columns 8r + 2*(i%4), +1 of its two heads.
+__device__ __forceinline__ bool attn_epilogue(int bt, int sp, int ntiles, float m0, float m1, float l0, float l1,
                                            uint32_t g_last, bool good, int nbt, int r0, int qi, int half,
                                            uint32_t tmem, uint32_t lane_off, uint32_t pv_done, volatile int* abort,
                                            __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
@@ -325,7 +333,7 @@ struct Item {
   int bt, sp, b, kbeg, kend, ntiles;
 };
 
-__global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(1, 2, 1) __maxnreg__(REGS_LAUNCH)
 sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv, int64_t kv_rs,
                      int64_t kv_bs, int S_kv, const int32_t* __restrict__ idx, int T, int nbt, int items, int k,
                      int keys_per_split, float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
@@ -400,11 +408,13 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   cluster_sync();   // both CTAs' barriers exist (and are armed) before either signals the other
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp >= GATHER_WARP0 && warp < MMA_WARP) {
+  // The register split opens each warpgroup's branch (warpgroup-uniform, taken before any role
+  // can give up), so the compiler sizes each role's code for its own register budget.
+  if (warp >= SMW) {
+    auto gather_role = [&]() {
     // ------------------------------------------------------------ gather (cp.async)
-    // Warp gw copies rows gw, gw+3, ..: lane l moves 16-byte chunks l, l+32 of its column
-    // range, so each row is read with coalesced requests.  A tile's ids come from one
+    // Warp gw copies rows gw, gw+GATHER_WARPS, ..: lane l moves 16-byte chunks l, l+32 of its
+    // column range, so each row is read with coalesced requests.  A tile's ids come from one
     // coalesced load per warp, issued a tile ahead, and reach the rows through shuffles.
     const int gw = warp - GATHER_WARP0;
     bool ok = true;
@@ -453,8 +463,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         }
       }
       const uint32_t stage = sbase + OFF_KV + st * KV_STAGE;
-#pragma unroll 4
-      for (int r = gw; r < NK; r += 3) {
+#pragma unroll 1
+      for (int r = gw; r < NK; r += GATHER_WARPS) {
         const int key = __shfl_sync(0xffffffffu, r < 32 ? id0 : id1, r & 31);
         const int crow = __shfl_sync(0xffffffffu, r < 32 ? row0 : row1, r & 31);
         const __nv_bfloat16* src = kvb + (int64_t)(key < 0 ? 0 : crow) * kv_rs;
@@ -472,8 +482,13 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     }
     }
     cp_async_wait<0>();
-  } else if (warp == MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
+    };
+    if (warp < 12) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(REGS_MID));
+      if (warp >= GATHER_WARP0) {
+        gather_role();
+      } else {
+    // ------------------------------------------------------------ MMA issuer (warp MMA_WARP)
     // Order: S_0, S_1, then for each tile j: the first S_EARLY K-steps of S_{j+2} (as soon as the
     // softmax has read S_{j+1}), then -- once P_j is in TMEM -- P_j.V_j interleaved with the other
     // K-steps of S_{j+2}.  The tensor pipe runs the 64-key score MMAs and the MN-major P.V MMAs
@@ -566,7 +581,13 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     if (lane == 0) mma_commit(mma_drain);
     __syncwarp();
     mbar_wait_bounded(mma_drain, 0, 100000000ull);
+      }
+    } else {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(REGS_LOW));
+      gather_role();
+    }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(REGS_HIGH));
     // ------------------------------------------------------------ softmax + epilogue (warps 0-7)
     const int quad = warp & 3, hh = warp >> 2;
     const int base = 32 * quad + 16 * hh;          // first TMEM lane (head) of this warp
@@ -800,6 +821,11 @@ int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, i
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    // The warpgroups' register split draws on the registers the block is launched with: launch
+    // only a build whose register count covers it (otherwise the rising warpgroups would wait).
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, sparse_mla_tc_kernel) != cudaSuccess || fa.numRegs < REGS_LAUNCH)
+      return DSA_ERR_CUDA;
     cudaFuncSetAttribute(sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
