@@ -307,14 +307,14 @@ def run_ours(args, rank, world, dev):
     return res, wl, parts
 
 
-def breakdown(parts, ws, t_chunk, stream, dsa, reps, unfused=True):
+def breakdown(parts, ws, t_chunk, stream, dsa, reps, fused=True):
     """Average device time of each step of the group per step over `reps` steps, CUDA events on
-    `stream`, summed over this rank's parts: the pool kernel, the selection (dsa_index_select:
-    the fused indexer + top-k the group call runs), and each attention layer; with `unfused`,
-    also the indexer and the top-k as separate calls over full score rows (the unfused path,
-    for comparison)."""
+    `stream`, summed over this rank's parts: the pool kernel, the selection as the group call
+    runs it (the indexer writing full score rows, then the row top-k, per query chunk), and each
+    attention layer; with `fused`, also the fused selection (dsa_index_select) over the same
+    chunks, for comparison."""
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    tot = {"pool": 0.0, "select": 0.0, "attn": 0.0, "indexer": 0.0, "topk": 0.0}
+    tot = {"pool": 0.0, "indexer": 0.0, "topk": 0.0, "attn": 0.0, "fused_select": 0.0}
     n = {k: 0 for k in tot}
     dev = ws.device
     for p in parts:
@@ -322,10 +322,13 @@ def breakdown(parts, ws, t_chunk, stream, dsa, reps, unfused=True):
         S_eff = ind["k_idx"].shape[1] // wl.pool
         ld = (S_eff + 3) // 4 * 4
         tc_max = min(t_chunk, wl.T)
-        sel_ws = torch.empty(dsa.dsa_index_select_workspace_size(wl.B, tc_max, S_eff, wl.pool), dtype=torch.uint8,
-                             device=dev)
+        sc_buf = torch.empty(wl.B * tc_max * ld, dtype=torch.float32, device=dev)
         attn_ws = torch.empty(max(1, dsa.dsa_sparse_attn_workspace_size(wl.B, wl.T, wl.Hq, wl.d_v, wl.topk * wl.pool)),
                               dtype=torch.uint8, device=dev)
+        sel_ws = None
+        if fused:
+            sel_ws = torch.empty(dsa.dsa_index_select_workspace_size(wl.B, tc_max, S_eff, wl.pool), dtype=torch.uint8,
+                                 device=dev)
         for rep in range(reps):
             marks = []
             keys = ind["k_idx"]
@@ -337,12 +340,16 @@ def breakdown(parts, ws, t_chunk, stream, dsa, reps, unfused=True):
                 marks.append(("pool", a, b))
             for t0 in range(0, wl.T, t_chunk):
                 tc = min(t_chunk, wl.T - t0)
-                a, b = ev(), ev()
+                sc = sc_buf[: wl.B * tc * ld].view(wl.B, tc, ld)   # [B, tc, ld], batch stride tc * ld
+                a, b, c = ev(), ev(), ev()
                 a.record(stream)
-                dsa.dsa_index_select(ind["q_idx"], ind["w"], keys, ind["ctx_len"], wl.topk, pool=wl.pool, t_begin=t0,
-                                     t_count=tc, idx=g.idx, ws=sel_ws, stream=stream)
+                dsa.dsa_index_scores(ind["q_idx"], ind["w"], keys, ind["ctx_len"], pool=wl.pool, t_begin=t0,
+                                     t_count=tc, scores=sc, stream=stream)
                 b.record(stream)
-                marks.append(("select", a, b))
+                dsa.dsa_topk(sc, ind["ctx_len"], wl.T, S_eff, wl.topk, pool=wl.pool, t_begin=t0, idx=g.idx,
+                             stream=stream)
+                c.record(stream)
+                marks += [("indexer", a, b), ("topk", b, c)]
             for L in g.layers:
                 a, b = ev(), ev()
                 a.record(stream)
@@ -350,29 +357,23 @@ def breakdown(parts, ws, t_chunk, stream, dsa, reps, unfused=True):
                                     stream=stream)
                 b.record(stream)
                 marks.append(("attn", a, b))
-            if unfused and rep == 0:
-                scores = sel_ws[: wl.B * tc_max * ld * 4].view(torch.float32)
+            if fused and rep == 0:
                 for t0 in range(0, wl.T, t_chunk):
                     tc = min(t_chunk, wl.T - t0)
-                    sc = scores[: wl.B * tc * ld].view(wl.B, tc, ld)   # [B, tc, ld], batch stride tc * ld
-                    a, b, c = ev(), ev(), ev()
+                    a, b = ev(), ev()
                     a.record(stream)
-                    dsa.dsa_index_scores(ind["q_idx"], ind["w"], keys, ind["ctx_len"], pool=wl.pool, t_begin=t0,
-                                         t_count=tc, scores=sc, stream=stream)
+                    dsa.dsa_index_select(ind["q_idx"], ind["w"], keys, ind["ctx_len"], wl.topk, pool=wl.pool,
+                                         t_begin=t0, t_count=tc, idx=g.idx, ws=sel_ws, stream=stream)
                     b.record(stream)
-                    dsa.dsa_topk(sc, ind["ctx_len"], wl.T, S_eff, wl.topk, pool=wl.pool, t_begin=t0, idx=g.idx,
-                                 stream=stream)
-                    c.record(stream)
-                    marks += [("indexer", a, b), ("topk", b, c)]
+                    marks.append(("fused_select", a, b))
             torch.cuda.synchronize()
             for name, a, b in marks:
-                tot[name] += a.elapsed_time(b) / (1 if name in ("indexer", "topk") else reps)
+                tot[name] += a.elapsed_time(b) / (1 if name == "fused_select" else reps)
                 n[name] += 1
-        del sel_ws, attn_ws
-    out = {k: tot[k] for k in ("pool", "select", "attn") if n[k]}
-    if n["indexer"]:
-        out["unfused"] = {"indexer": tot["indexer"], "topk": tot["topk"]}
-    out["per_launch"] = {"select_chunk": tot["select"] / max(1, n["select"] / reps),
+        del sc_buf, attn_ws, sel_ws
+    out = {k: tot[k] for k in ("pool", "indexer", "topk", "attn", "fused_select") if n[k]}
+    out["per_launch"] = {"indexer_chunk": tot["indexer"] / max(1, n["indexer"] / reps),
+                         "topk_chunk": tot["topk"] / max(1, n["topk"] / reps),
                          "attn_layer": tot["attn"] / max(1, n["attn"] / reps)}
     return out
 
@@ -380,54 +381,54 @@ def breakdown(parts, ws, t_chunk, stream, dsa, reps, unfused=True):
 # DRAM bytes (read + write) per query, from one ncu capture with the bench's 131072-row context
 # and 2048 queries (dram__bytes_read.sum + dram__bytes_write.sum per launch / queries).
 # Per-query traffic does not depend on the number of queries, so a launch's traffic is this
-# figure times its queries.  Only kernels unchanged since that capture are listed: the indexer
-# and the top-k have changed since (their traffic is reported as None until re-captured), and
-# other contexts were not measured.
-TRAFFIC_PER_QUERY = {("prefill128k", "attn"): 587.6e3}
+# figure times its queries.  Only kernels unchanged since that capture are listed (others
+# report None), and other contexts were not measured.
+TRAFFIC_PER_QUERY = {}
 
 
 def roofline(wls, brk, pk, t_chunk):
-    """Roofline of the step with the largest share of the time; `wls` are the (sub-)workloads
-    this rank ran, whose work adds up.  The selection (fused indexer + top-k) is held against
-    the fp8 tensor roofline with the indexer's flops: its sampling pass, threshold and top-k
-    count as overhead, not as work."""
+    """Roofline of the kernel with the largest share of the time (indexer, top-k or attention,
+    as the group call runs them); `wls` are the (sub-)workloads this rank ran, whose work adds
+    up.  The fused selection, when timed, is listed too (against the indexer's roofline, its
+    sampling pass, threshold and top-k counting as overhead)."""
     wls = wls if isinstance(wls, (list, tuple)) else [wls]
     wl = wls[0]
     fp8_peak = 2.0 * pk["bf16_sus"]   # nominal fp8:bf16 ratio 2 on the measured bf16 figure
     n_layers = wl.group
-    ent = {
-        "select": {"bound": "tensor", "achieved": sum(indexer_flops(w) for w in wls) / (brk["select"] * 1e-3) / 1e12,
-                   "peak": fp8_peak, "unit": "TFLOP/s", "dtype": "fp8", "traffic": None,
-                   "peak_src": f"2 x {pk['src']} bf16 sustained",
-                   "work": "indexer flops (2*H_I*d_I per visible pair); time of the fused indexer + top-k"},
-        "attn": {"bound": "tensor",
-                 "achieved": sum(attn_flops(w) for w in wls) * n_layers / (brk["attn"] * 1e-3) / 1e12,
-                 "peak": pk["bf16_sus"], "unit": "TFLOP/s", "dtype": "bf16", "traffic": None,
-                 "peak_src": f"{pk['src']} bf16 sustained"},
-    }
     rows = sum(w.B * w.T for w in wls)
-    if rows <= 64:   # decode: HBM-bound
+    decode = rows <= 64
+    ifl = sum(indexer_flops(w) for w in wls)
+    ibytes = sum(w.B * (w.S // w.pool) * w.d_I + w.B * w.T * w.H_I * (w.d_I + 4) for w in wls)
+    topk_bytes = sum(4 * causal_pairs(w) + 4 * w.B * w.T * w.topk * w.pool for w in wls)
+
+    def idx_entry(ms, what):
+        if decode:
+            return {"bound": "hbm", "achieved": ibytes / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "traffic": None, "peak_src": f"{pk['src']} copy",
+                    "work": f"indexer key, query and weight bytes; time of {what}"}
+        return {"bound": "tensor", "achieved": ifl / (ms * 1e-3) / 1e12, "peak": fp8_peak, "unit": "TFLOP/s",
+                "dtype": "fp8", "traffic": None, "peak_src": f"2 x {pk['src']} bf16 sustained",
+                "work": f"indexer flops (2*H_I*d_I per visible pair); time of {what}"}
+    ent = {
+        "indexer": idx_entry(brk["indexer"], "the indexer"),
+        "topk": {"bound": "hbm", "achieved": topk_bytes / (brk["topk"] * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                 "unit": "GB/s", "traffic": None, "peak_src": f"{pk['src']} copy",
+                 "work": "score rows read + selected ids written"},
+    }
+    if decode:   # HBM-bound: the selected rows' bytes
         ent["attn"] = {"bound": "hbm", "achieved": sum(attn_bytes(w) for w in wls) * n_layers / (brk["attn"] * 1e-3) / 1e9,
                        "peak": pk["hbm_gbs"], "unit": "GB/s", "traffic": None, "peak_src": f"{pk['src']} copy"}
-        ent["select"] = {"bound": "hbm",
-                         "achieved": sum(w.B * (w.S // w.pool) * w.d_I + w.B * w.T * w.H_I * (w.d_I + 4) for w in wls)
-                         / (brk["select"] * 1e-3) / 1e9,
-                         "peak": pk["hbm_gbs"], "unit": "GB/s", "traffic": None, "peak_src": f"{pk['src']} copy",
-                         "work": "indexer key, query and weight bytes; time of the fused indexer + top-k"}
-    if "unfused" in brk:
-        u = brk["unfused"]
-        topk_bytes = sum(4 * causal_pairs(w) + 4 * w.B * w.T * w.topk * w.pool for w in wls)
-        ent["indexer_unfused"] = {"bound": "tensor" if rows > 64 else "hbm", "unit": "TFLOP/s" if rows > 64 else "GB/s",
-                                  "achieved": (sum(indexer_flops(w) for w in wls) / (u["indexer"] * 1e-3) / 1e12
-                                               if rows > 64 else ent["select"]["achieved"] * brk["select"] / u["indexer"]),
-                                  "peak": fp8_peak if rows > 64 else pk["hbm_gbs"], "traffic": None,
-                                  "peak_src": ent["select"]["peak_src"]}
-        ent["topk_unfused"] = {"bound": "hbm", "achieved": topk_bytes / (u["topk"] * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
-                               "unit": "GB/s", "traffic": None, "peak_src": f"{pk['src']} copy"}
-    for k, queries in (("attn", rows / len(wls)), ("select", min(t_chunk, rows))):
+    else:
+        ent["attn"] = {"bound": "tensor",
+                       "achieved": sum(attn_flops(w) for w in wls) * n_layers / (brk["attn"] * 1e-3) / 1e12,
+                       "peak": pk["bf16_sus"], "unit": "TFLOP/s", "dtype": "bf16", "traffic": None,
+                       "peak_src": f"{pk['src']} bf16 sustained"}
+    if "fused_select" in brk:
+        ent["fused_select"] = idx_entry(brk["fused_select"], "the fused indexer + top-k")
+    for k, queries in (("attn", rows / len(wls)), ("indexer", min(t_chunk, rows)), ("topk", min(t_chunk, rows))):
         per_q = TRAFFIC_PER_QUERY.get((wl.name, k))
         ent[k]["traffic"] = None if per_q is None else per_q * queries   # bytes per launch
-    top = max(("select", "attn"), key=lambda k: brk[k])
+    top = max(("indexer", "topk", "attn"), key=lambda k: brk[k])
     r = dict(ent[top])
     r["kernel"] = top
     r["frac"] = r["achieved"] / r["peak"]

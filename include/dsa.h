@@ -250,9 +250,9 @@ int dsa_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool, ui
 /* ------------------------------------------------------------------------------------
  * dsa_group_forward - one IndexShare group ("IndexShare: Amortizing the Indexer"): the
  * indexer and the top-k run ONCE, and each of the group_size attention layers reads the
- * same index buffer.  Equivalent to dsa_index_select over all queries (in query chunks sized
- * to the workspace; full score rows instead when full_scores = 1), then group_size x
- * dsa_sparse_attn.
+ * same index buffer.  Equivalent to dsa_index_scores + dsa_topk over all queries (in query
+ * chunks sized to the workspace; dsa_index_select instead when fused_select = 1), then
+ * group_size x dsa_sparse_attn.
  * With pool > 1 the indexer runs on dsa_index_pool's blocks and `topk` counts blocks
  * (idx then holds pool*topk token ids per row).  The comparator without IndexShare is
  * group_size calls with group_size = 1 and per-layer indexer tensors.
@@ -280,8 +280,9 @@ typedef struct dsa_group_args {
   int32_t* idx;            /* [B, T, topk*pool] int32 out: the shared selection */
   dsa_paging paging;       /* block_table NULL: contiguous caches; else k_idx and every
                               layer's kv (and v) are page pools sharing this table */
-  int32_t full_scores;     /* 0 (default): fused selection where the keys allow it (see
-                              dsa_index_select); 1: always full score rows + dsa_topk */
+  int32_t fused_select;    /* 0 (default): full score rows + dsa_topk, the faster path on B200
+                              (the indexer is tensor-bound, so its score rows cost little);
+                              1: fused selection where the keys allow it (dsa_index_select) */
 } dsa_group_args;
 
 /* Workspace for dsa_group_forward when the indexer is run over chunks of t_chunk queries

@@ -65,7 +65,7 @@ class GroupArgs(ctypes.Structure):
         ("kv_row_stride", _c_i64), ("kv_batch_stride", _c_i64), ("v_row_stride", _c_i64),
         ("v_batch_stride", _c_i64),
         ("Hq", ctypes.c_int32), ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32), ("sm_scale", _c_f),
-        ("idx", _c_p), ("paging", Paging), ("full_scores", ctypes.c_int32),
+        ("idx", _c_p), ("paging", Paging), ("fused_select", ctypes.c_int32),
     ]
 
 
@@ -364,7 +364,7 @@ class Group:
 
     def __init__(self, q_idx, w, k_idx, ctx_len, topk: int, layers: Sequence[dict], sm_scale: float,
                  d_v: int, pool: int = 1, idx: Optional[torch.Tensor] = None, want_lse: bool = False,
-                 paging: Optional[Paging] = None, full_scores: bool = False):
+                 paging: Optional[Paging] = None, fused_select: bool = False):
         B, T, H, D = q_idx.shape
         S = k_idx.shape[1] if paging is None else paging.pages_per_seq * paging.page_size
         L = len(layers)
@@ -413,7 +413,7 @@ class Group:
             v_row_stride=v_any.stride(1) if v_any is not None else 0,
             v_batch_stride=v_any.stride(0) if v_any is not None else 0,
             Hq=Hq, d_qk=Dqk, d_v=d_v, sm_scale=float(sm_scale), idx=_ptr(self.idx),
-            paging=paging if paging is not None else Paging(), full_scores=1 if full_scores else 0)
+            paging=paging if paging is not None else Paging(), fused_select=1 if fused_select else 0)
         self._paging = paging
         self.device = q0.device
 
@@ -428,13 +428,13 @@ class Group:
 
 def dsa_group_forward(q_idx, w, k_idx, ctx_len, topk: int, layers: Sequence[dict], sm_scale: float, d_v: int,
                       pool: int = 1, t_chunk: Optional[int] = None, ws: Optional[torch.Tensor] = None,
-                      want_lse: bool = False, paging: Optional[Paging] = None, full_scores: bool = False,
+                      want_lse: bool = False, paging: Optional[Paging] = None, fused_select: bool = False,
                       stream=None):
     """One IndexShare group: indexer + top-k once, then attention for each layer dict
     {"q", "kv", optional "v", "out", "lse"}; with `paging`, k_idx and every layer's kv (and v)
     are page pools sharing its block table.  Returns (idx, [(out, lse) per layer])."""
     g = Group(q_idx, w, k_idx, ctx_len, topk, layers, sm_scale, d_v, pool, want_lse=want_lse, paging=paging,
-              full_scores=full_scores)
+              fused_select=fused_select)
     if ws is None:
         ws = torch.empty(g.workspace_size(t_chunk or q_idx.shape[1]), dtype=torch.uint8, device=g.device)
     return g.forward(ws, stream)

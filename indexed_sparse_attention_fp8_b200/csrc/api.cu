@@ -127,8 +127,8 @@ SelectWs select_ws(int64_t rows, int S_eff, bool fused) {
 }
 
 // The fused path needs contiguous keys whose sequences hold whole sampled rows.
-bool select_fused_ok(int S_eff, const PageMap& key_pm, int full_scores) {
-  return full_scores == 0 && key_pm.bt == nullptr && S_eff >= kSampleStride && S_eff % kSampleStride == 0;
+bool select_fused_ok(int S_eff, const PageMap& key_pm, int fused_select) {
+  return fused_select != 0 && key_pm.bt == nullptr && S_eff >= kSampleStride && S_eff % kSampleStride == 0;
 }
 
 // Largest chunk of queries (<= T) whose selection workspace fits `bytes`; 0 if none does.
@@ -203,7 +203,7 @@ GroupWs group_ws(const dsa_group_args* a) {
   g.attn_bytes = round_up(attn_workspace_bytes(a->B, a->T, a->Hq, a->d_v, a->topk * a->pool), 256);
   g.fixed_bytes = g.pool_bytes + g.attn_bytes;
   const PageMap key_pm = a->pool > 1 ? PageMap{nullptr, 0, 0, 0} : page_map(&a->paging);
-  g.fused = select_fused_ok(g.S_eff, key_pm, a->full_scores);
+  g.fused = select_fused_ok(g.S_eff, key_pm, a->fused_select);
   return g;
 }
 
@@ -345,7 +345,7 @@ size_t dsa_group_workspace_size(const dsa_group_args* a, int t_chunk) {
 
 size_t dsa_index_select_workspace_size(int B, int t_chunk, int S_max, int pool) {
   if (B <= 0 || t_chunk < 1 || S_max < 1 || pool < 1) return 0;
-  return select_ws((int64_t)B * t_chunk, S_max, select_fused_ok(S_max, PageMap{nullptr, 0, 0, 0}, 0)).total();
+  return select_ws((int64_t)B * t_chunk, S_max, select_fused_ok(S_max, PageMap{nullptr, 0, 0, 0}, 1)).total();
 }
 
 int dsa_index_select(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* ctx_len, int B,
@@ -358,7 +358,7 @@ int dsa_index_select(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
   if (B == 0 || t_count == 0) return DSA_OK;
   if (!idx) return DSA_ERR_INVALID_ARG;
   const PageMap key_pm = page_map(paging);
-  const bool fused = select_fused_ok(S_max, key_pm, 0);
+  const bool fused = select_fused_ok(S_max, key_pm, 1);
   const int t_chunk = select_chunk(ws_bytes, B, t_count, S_max, fused);
   if (t_chunk < 1) return DSA_ERR_WORKSPACE_TOO_SMALL;
   if (!ws) return DSA_ERR_INVALID_ARG;

@@ -188,11 +188,11 @@ def _fused_row_bytes(S):
 
 def test_group_workspace_and_validation(lib):
     args, keep = _group_args()
-    args.full_scores = 1
+    args.fused_select = 0                                   # the default: full score rows + top-k
     one = lib.dsa_group_workspace_size(ctypes.byref(args), 1)
     big = lib.dsa_group_workspace_size(ctypes.byref(args), 1024)
     assert one == 32768 * 4 and big == 1024 * 32768 * 4     # a chunk of fp32 score rows
-    args.full_scores = 0                                    # the default: fused selection
+    args.fused_select = 1                                   # fused selection
     one = lib.dsa_group_workspace_size(ctypes.byref(args), 1)
     assert one == _fused_row_bytes(32768)
     assert lib.dsa_index_select_workspace_size(1, 1, 32768, 1) == one
@@ -202,6 +202,9 @@ def test_group_workspace_and_validation(lib):
     bad, keep2 = _group_args(topk=4096)
     assert lib.dsa_group_forward(ctypes.byref(bad), A, 1 << 40, None) == UNSUPPORTED
     pool_args, keep3 = _group_args(pool=4, topk=512, S=1048576, T=8192)
+    need = lib.dsa_group_workspace_size(ctypes.byref(pool_args), 1)
+    assert need == (1048576 // 4) * 128 + (1048576 // 4) * 4    # pooled keys + one full score row
+    pool_args.fused_select = 1
     need = lib.dsa_group_workspace_size(ctypes.byref(pool_args), 1)
     assert need == (1048576 // 4) * 128 + _fused_row_bytes(1048576 // 4)   # pooled keys + one selection row
     odd, keep4 = _group_args(pool=4, topk=512, S=1048574, T=8192)

@@ -28,18 +28,19 @@ def test_work_counts_closed_forms():
 
 def test_roofline_prefill_entries():
     wl = W.WORKLOADS["prefill128k"]
-    brk = {"select": 70.0, "attn": 451.4, "unfused": {"indexer": 89.3, "topk": 30.7},
-           "per_launch": {"select_chunk": 8.75, "attn_layer": 112.85}}
+    brk = {"indexer": 89.3, "topk": 30.7, "attn": 451.4, "fused_select": 70.0,
+           "per_launch": {"indexer_chunk": 11.2, "topk_chunk": 3.8, "attn_layer": 112.85}}
     r = bench.roofline(wl, brk, PK, 16384)
     assert r["kernel"] == "attn" and r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     flops = 128 * 2 * (576 + 512) * bench.selected_pairs(wl)
     assert r["achieved"] == pytest.approx(4 * flops / 451.4e-3 / 1e12)
     assert r["peak"] == 1382.4 and r["frac"] == pytest.approx(r["achieved"] / 1382.4)
-    assert r["traffic"] == pytest.approx(bench.TRAFFIC_PER_QUERY[("prefill128k", "attn")] * wl.B * wl.T)
-    sel, ix, tk = r["others"]["select"], r["others"]["indexer_unfused"], r["others"]["topk_unfused"]
-    assert sel["achieved"] == pytest.approx(2 * 64 * 128 * bench.causal_pairs(wl) / 70.0e-3 / 1e12)
-    assert sel["peak"] == pytest.approx(2 * 1382.4)
+    per_q = bench.TRAFFIC_PER_QUERY.get(("prefill128k", "attn"))
+    assert r["traffic"] == (None if per_q is None else pytest.approx(per_q * wl.B * wl.T))
+    ix, tk, fs = r["others"]["indexer"], r["others"]["topk"], r["others"]["fused_select"]
     assert ix["achieved"] == pytest.approx(2 * 64 * 128 * bench.causal_pairs(wl) / 89.3e-3 / 1e12)
+    assert ix["peak"] == pytest.approx(2 * 1382.4)
+    assert fs["achieved"] == pytest.approx(2 * 64 * 128 * bench.causal_pairs(wl) / 70.0e-3 / 1e12)
     assert tk["bound"] == "hbm"
     assert tk["achieved"] == pytest.approx((4 * bench.causal_pairs(wl) + 4 * wl.T * 2048) / 30.7e-3 / 1e9)
     assert tk["frac"] == pytest.approx(tk["achieved"] / 6535.7)
@@ -47,13 +48,15 @@ def test_roofline_prefill_entries():
 
 def test_roofline_decode_is_hbm_bound():
     wl = W.WORKLOADS["decode256k"]
-    brk = {"select": 0.25, "attn": 0.218, "per_launch": {"select_chunk": 0.25, "attn_layer": 0.0545}}
+    brk = {"indexer": 0.21, "topk": 0.084, "attn": 0.218,
+           "per_launch": {"indexer_chunk": 0.21, "topk_chunk": 0.084, "attn_layer": 0.0545}}
     r = bench.roofline(wl, brk, PK, 1)
-    assert r["kernel"] == "select" and r["bound"] == "hbm" and r["unit"] == "GB/s"
-    assert r["achieved"] == pytest.approx((32 * 262144 * 128 + 32 * 64 * 132) / 0.25e-3 / 1e9)
-    a = r["others"]["attn"]
-    assert a["bound"] == "hbm" and a["achieved"] == pytest.approx(4 * bench.attn_bytes(wl) / 0.218e-3 / 1e9)
-    assert r["traffic"] is None and a["traffic"] is None          # no capture at this context
+    assert r["kernel"] == "attn" and r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(4 * bench.attn_bytes(wl) / 0.218e-3 / 1e9)
+    ix = r["others"]["indexer"]
+    assert ix["bound"] == "hbm"
+    assert ix["achieved"] == pytest.approx((32 * 262144 * 128 + 32 * 64 * 132) / 0.21e-3 / 1e9)
+    assert r["traffic"] is None and ix["traffic"] is None          # no capture at this context
 
 
 def test_roofline_sums_the_work_of_shards():
@@ -63,6 +66,7 @@ def test_roofline_sums_the_work_of_shards():
     halves = [bench.box_workload(wl, b) for b in boxes]
     assert sum(bench.causal_pairs(h) for h in halves) == bench.causal_pairs(wl)
     assert sum(bench.selected_pairs(h) for h in halves) == bench.selected_pairs(wl)
-    brk = {"select": 10.0, "attn": 40.0, "per_launch": {"select_chunk": 5.0, "attn_layer": 5.0}}
+    brk = {"indexer": 8.0, "topk": 2.0, "attn": 40.0,
+           "per_launch": {"indexer_chunk": 4.0, "topk_chunk": 1.0, "attn_layer": 5.0}}
     assert bench.roofline(halves, brk, PK, 16384)["achieved"] == pytest.approx(
         bench.roofline(wl, brk, PK, 16384)["achieved"])

@@ -443,11 +443,13 @@ def test_fused_selection_equals_full_score_rows_bitwise(name, over):
     got = dsa.dsa_index_select(ind["q_idx"], ind["w"], keys, ind["ctx_len"], wl.topk, pool=wl.pool)
     ref = _unfused_ids(wl, ind, keys)
     assert torch.equal(got, ref)
-    # through the group call too, with a workspace small enough for several query chunks
-    idx, outs = dsa.dsa_group_forward(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk,
-                                      [{"q": lays[0]["q"], "kv": lays[0]["kv"], "v": lays[0]["v"]}], wl.sm_scale,
-                                      wl.d_v, pool=wl.pool, t_chunk=max(1, wl.T // 3))
-    assert torch.equal(idx, ref)
+    # through the group call too (fused and default selection), with a workspace small enough for
+    # several query chunks
+    for fused in (True, False):
+        idx, outs = dsa.dsa_group_forward(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk,
+                                          [{"q": lays[0]["q"], "kv": lays[0]["kv"], "v": lays[0]["v"]}], wl.sm_scale,
+                                          wl.d_v, pool=wl.pool, t_chunk=max(1, wl.T // 3), fused_select=fused)
+        assert torch.equal(idx, ref)
     kdec = P.Decoded(ind["k_idx"])
     kpd = P.Decoded(keys) if wl.pool > 1 else None
     idx_h = P.to_np(idx)
