@@ -128,6 +128,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
                        int pool, int t_begin, int t_count, float* __restrict__ scores, int64_t ld, PageMap pm,
                        const float* __restrict__ tau, float2* __restrict__ cand, int* __restrict__ cnt, int cap,
                        const int* __restrict__ row_flag) {
+  const uint64_t wlim = wait_limit();   // the bounded waits' time limit, read once
   using C = IdxCfg<H, D, QB>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
@@ -185,7 +186,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       ItemGeom g;
       if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g, row_flag)) continue;
       const int bs = b_cnt & 1;
-      if (!(ok = mbar_wait_warp(b_empty(bs), ((b_cnt >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
+      if (!(ok = mbar_wait_warp(b_empty(bs), ((b_cnt >> 1) & 1) ^ 1, abort, wlim))) break;
       if (lane == 0) {
         const uint32_t wbytes = (uint32_t)(g.nq * H * 4);
         mbar_arrive_expect_tx(b_full(bs), C::B_BYTES + wbytes);
@@ -195,7 +196,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       ++b_cnt;
       for (int kt = g.kt0; kt < g.kt1; ++kt) {
         const int as = a_cnt % NA;
-        if (!(ok = mbar_wait_warp(a_empty(as), ((a_cnt / NA) & 1) ^ 1, abort, kWaitLimitNs))) break;
+        if (!(ok = mbar_wait_warp(a_empty(as), ((a_cnt / NA) & 1) ^ 1, abort, wlim))) break;
         if (lane == 0) {
           // contiguous: row b*S_max + s of the cache; paged: the tile's page (a tile never
           // straddles one); a bad page id loads past the map's extent, which reads zeros
@@ -228,13 +229,13 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       ItemGeom g;
       if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g, row_flag)) continue;
       const int bs = b_cnt & 1;
-      if (!(ok = mbar_wait_warp(b_full(bs), (b_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
+      if (!(ok = mbar_wait_warp(b_full(bs), (b_cnt >> 1) & 1, abort, wlim))) break;
       const uint32_t b_addr = sbase + C::OFF_B + bs * C::B_BYTES;
       for (int kt = g.kt0; kt < g.kt1; ++kt) {
         const int as = a_cnt % NA;
         const int ab = acc_cnt & 1;
-        if (!(ok = mbar_wait_warp(a_full(as), (a_cnt / NA) & 1, abort, kWaitLimitNs))) break;
-        if (!(ok = mbar_wait_warp(acc_empty(ab), ((acc_cnt >> 1) & 1) ^ 1, abort, kWaitLimitNs))) break;
+        if (!(ok = mbar_wait_warp(a_full(as), (a_cnt / NA) & 1, abort, wlim))) break;
+        if (!(ok = mbar_wait_warp(acc_empty(ab), ((acc_cnt >> 1) & 1) ^ 1, abort, wlim))) break;
         tc_fence_after();
         if (lane == 0) {
           const uint32_t a_addr = sbase + C::OFF_A + as * C::A_BYTES;
@@ -275,7 +276,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       ItemGeom g;
       if (!item_geom(it, QB, nqb, nkc, T, t_begin, t_count, S_max, pool, ctx_len, g, row_flag)) continue;
       const int bs = b_cnt & 1;
-      if (!(ok = mbar_wait_warp(b_full(bs), (b_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
+      if (!(ok = mbar_wait_warp(b_full(bs), (b_cnt >> 1) & 1, abort, wlim))) break;
       const float* wsm = reinterpret_cast<const float*>(sgen + C::OFF_W + bs * C::W_BYTES) + half * C::COLS;
       const int ctx_b = __ldg(ctx_len + g.b);
       // H == 64: the 16x256b TMEM shape gives each thread 2 keys x 2 heads per 8-column group,
@@ -350,7 +351,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
           }
         };
         if (g.kt0 < g.kt1) {
-          if (!(ok = mbar_wait_warp(acc_full(acc_cnt & 1), (acc_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
+          if (!(ok = mbar_wait_warp(acc_full(acc_cnt & 1), (acc_cnt >> 1) & 1, abort, wlim))) break;
           tc_fence_after();
           issue(acc_cnt & 1, 0, v[0]);
           tmem_ld_wait();
@@ -370,7 +371,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
               __syncwarp();
               if (lane == 0) mbar_arrive(acc_empty(ab));
               if (more) {
-                if (!(ok = mbar_wait_warp(acc_full(ab ^ 1), ((acc_cnt + 1) >> 1) & 1, abort, kWaitLimitNs))) break;
+                if (!(ok = mbar_wait_warp(acc_full(ab ^ 1), ((acc_cnt + 1) >> 1) & 1, abort, wlim))) break;
                 tc_fence_after();
                 issue(ab ^ 1, 0, v[0]);
               }
@@ -428,7 +429,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       } else {
       for (int kt = g.kt0; kt < g.kt1; ++kt) {
         const int ab = acc_cnt & 1;
-        if (!(ok = mbar_wait_warp(acc_full(ab), (acc_cnt >> 1) & 1, abort, kWaitLimitNs))) break;
+        if (!(ok = mbar_wait_warp(acc_full(ab), (acc_cnt >> 1) & 1, abort, wlim))) break;
         tc_fence_after();
         // finished sum of query ql (local to this warp) for key s -> masked store
         auto store = [&](int ql, int s, float val) {

@@ -19,16 +19,17 @@ namespace tc {
 static __device__ unsigned int g_status;
 
 // Time limit of the kernels' bounded waits (2 s: no legal wait comes close).  A test hook may
-// shorten it (dsa_debug_set_wait_limit) to make the real kernels' waits run out; waits read it
-// only once their first check has failed.  A limit below kImmediateNs makes every wait that is
-// not ready at its first (non-blocking) check give up at once: the timer's resolution is too
-// coarse to time such limits, and a blocking try can outlast them.  One copy per translation
-// unit.
+// shorten it (dsa_debug_set_wait_limit) to make the real kernels' waits run out.  Each kernel
+// reads it once at its start (wait_limit()) and passes the value to its waits, so no wait puts a
+// memory load on its path.  A limit below kImmediateNs makes every wait that is not ready at
+// its first (non-blocking) check give up at once: the timer's resolution is too coarse to time
+// such limits, and a blocking try can outlast them.  One copy per translation unit.
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 constexpr uint64_t kImmediateNs = 1000;
 static __device__ unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
-// The limit a wait passes to mbar_wait to use g_wait_limit_ns.
-constexpr uint64_t kWaitLimitNs = 0;
+__device__ __forceinline__ uint64_t wait_limit() {
+  return *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+}
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -88,19 +89,19 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete.  Gives up after limit_ns of
-// waiting (0: the kernels' wait limit g_wait_limit_ns; below kImmediateNs: at once if the first
-// check fails), or as soon as another role of the CTA raised *abort: then sets *abort and the
-// device status word and returns false.  Never spins without bound.
+// Waits for the phase with the given parity to complete.  Gives up after limit_ns of waiting
+// (the kernel's wait_limit(); below kImmediateNs: at once if the first check fails), or as soon
+// as another role of the CTA raised *abort: then sets *abort and the device status word and
+// returns false.  Never spins without bound.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns) {
-  if (mbar_test_wait(bar, parity)) return true;
-  if (limit_ns == 0) limit_ns = *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
   if (limit_ns < kImmediateNs) {
+    if (mbar_test_wait(bar, parity)) return true;
     *abort = 1;
     atomicOr(&g_status, 1u);
     return false;
   }
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
