@@ -1,9 +1,9 @@
 """Model check of the MLA attention kernel's barrier protocol (CPU).
 
 `sparse_mla_tc_kernel` (indexed_sparse_attention_fp8_b200/csrc/attn_tc.cu) coordinates, in
-each CTA of a pair, the gather warps, the MMA-issuing warp, the 8 softmax warps (16 heads each,
-with their own exchange barriers), the tensor
-pipe and the bulk copies into the partner CTA through mbarriers only.  This model restates
+each CTA of a pair, the gather warps, the MMA-issuing warp, the 4 softmax warps (32 heads each,
+with their own exchange barriers), the tensor pipe and the bulk copies into the partner CTA
+through mbarriers only.  This model restates
 that protocol operation by operation -- every wait (barrier and parity), arrival, expect-tx,
 asynchronous completion (tensor-pipe FIFO, cp.async landings, bulk copies) -- and runs it
 under random schedules.  It checks that
@@ -21,7 +21,7 @@ import random
 import pytest
 
 NS = 4           # key-tile stages
-W = 8            # softmax warps
+W = 4            # softmax warps
 
 
 class Deadlock(Exception):
@@ -126,7 +126,7 @@ class Pair:
                 B[f"ids_ready{st}"].arrive()
 
                 def land(st=st, gg=g):
-                    R[f"kv{st}"].write(gg, 3)              # read by both K-halves of S_g and by P_g.V_g
+                    R[f"kv{st}"].write(gg, 2)              # read by S_g and by P_g.V_g
                     B[f"kv_full{st}"].arrive()
                 yield ("async", f"cp{c}", land)
                 g += 1
@@ -139,16 +139,15 @@ class Pair:
     def mma(self, c):
         B, R, O = self.cta[c]["bar"], self.cta[c]["buf"], self.cta[c]["O"]
 
-        def s_half(gg, item, second):
+        def s_run(gg, item):
             st = gg % NS
 
             def run():
                 R[f"kv{st}"].read(gg)
                 for w in range(W):
                     R[f"Q{w}"].read(item)
-                if second:                             # the last K-steps: S complete
-                    R["S"].write(gg, W)
-                    B["s_full"].arrive()
+                R["S"].write(gg, W)
+                B["s_full"].arrive()
             return run
 
         def issue_s(gg, item):
@@ -157,8 +156,7 @@ class Pair:
                 return False
             if not (yield ("wait", B["s_empty"], (gg & 1) ^ 1)):
                 return False
-            yield ("async", f"tc{c}", s_half(gg, item, False))
-            yield ("async", f"tc{c}", s_half(gg, item, True))
+            yield ("async", f"tc{c}", s_run(gg, item))
             return True
 
         def pv_run(gg, item, j):
@@ -187,22 +185,6 @@ class Pair:
             yield ("async", f"tc{c}", pv_run(gg, item, j))
             return True
 
-        def issue_s_with_pv(gs, gpv, item, j):
-            """S of tile gs: its first K-steps as soon as its stage and the S columns are free, then
-            (once P of tile gpv is in TMEM) the P.V of tile gpv interleaved with the other K-steps."""
-            st = gs % NS
-            if not (yield ("wait", B[f"kv_full{st}"], (gs // NS) & 1)):
-                return False
-            if not (yield ("wait", B["s_empty"], (gs & 1) ^ 1)):
-                return False
-            yield ("async", f"tc{c}", s_half(gs, item, False))
-            if "no_p_wait_interleave" not in self.mk:
-                if not (yield ("wait", B["p_full"], gpv & 1)):
-                    return False
-            yield ("async", f"tc{c}", pv_run(gpv, item, j))
-            yield ("async", f"tc{c}", s_half(gs, item, True))
-            return True
-
         g = nq = 0
         ok = True
         for it in self.mine():
@@ -217,13 +199,12 @@ class Pair:
             ok = yield from issue_s(g, it)
             if ok and nt > 1:
                 ok = yield from issue_s(g + 1, it)
-            for j in range(nt):
+            for j in range(nt):                        # S_{j+2} ahead of P_j.V_j
+                if ok and j + 2 < nt:
+                    ok = yield from issue_s(g + j + 2, it)
                 if not ok:
                     break
-                if j + 2 < nt:
-                    ok = yield from issue_s_with_pv(g + j + 2, g + j, it, j)
-                else:
-                    ok = yield from issue_pv(g + j, it, j)
+                ok = yield from issue_pv(g + j, it, j)
             if not ok:
                 break
             g += nt
@@ -308,7 +289,7 @@ class Pair:
             real = it is not None and ok
             nt = self.items[it] if real else 0
             if nt > 0:                                 # the next query's q into TMEM first
-                R[f"Q{w}"].write(it, 2 * nt)           # read by both K-halves of every S
+                R[f"Q{w}"].write(it, nt)               # read by every S of the item
                 B["q_ready"].arrive()
             if prev is not None:
                 ok = yield from epilogue(prev[0], prev[1], g - 1, ok)
@@ -441,7 +422,7 @@ def test_abort_path_without_a_drain_is_caught(mistake):
 
 @pytest.mark.parametrize("mistake", ["s_empty_count", "no_kv_empty_wait", "no_q_wait", "no_stage_read_wait",
                                      "no_x_free_wait", "early_x_free", "no_rearm", "no_pv_wait",
-                                     "no_epilogue_wait", "no_p_wait_interleave"])
+                                     "no_epilogue_wait"])
 def test_planted_protocol_mistake_is_caught(mistake):
     with pytest.raises((AssertionError, Deadlock)):
         _run_all(mistakes=(mistake,))
