@@ -383,7 +383,8 @@ def breakdown(parts, ws, t_chunk, stream, dsa, reps, fused=True):
 # Per-query traffic does not depend on the number of queries, so a launch's traffic is this
 # figure times its queries.  Only kernels unchanged since that capture are listed (others
 # report None), and other contexts were not measured.
-TRAFFIC_PER_QUERY = {}
+TRAFFIC_PER_QUERY = {("prefill128k", "attn"): 583.8e3, ("prefill128k", "indexer"): 509.0e3,
+                     ("prefill128k", "topk"): 574.2e3}
 
 
 def roofline(wls, brk, pk, t_chunk):
