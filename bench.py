@@ -378,13 +378,15 @@ def breakdown(parts, ws, t_chunk, stream, dsa, reps, fused=True):
     return out
 
 
-# DRAM bytes (read + write) per query, from one ncu capture with the bench's 131072-row context
-# and 2048 queries (dram__bytes_read.sum + dram__bytes_write.sum per launch / queries).
-# Per-query traffic does not depend on the number of queries, so a launch's traffic is this
-# figure times its queries.  Only kernels unchanged since that capture are listed (others
-# report None), and other contexts were not measured.
-TRAFFIC_PER_QUERY = {("prefill128k", "attn"): 583.8e3, ("prefill128k", "indexer"): 509.0e3,
-                     ("prefill128k", "topk"): 574.2e3}
+# DRAM bytes (read + write) per unit of work, from one ncu capture with the bench's 131072-row
+# context and its last 2048 queries (dram__bytes_read.sum + dram__bytes_write.sum per launch):
+# per query for the attention (each query reads its q, writes its output and gathers its own
+# 2048 key rows), per visible (query, key) pair for the indexer and the top-k (their bytes are
+# the score rows, 4 B per pair written and read back).  A launch's traffic is the figure times
+# the units it processes.  Only kernels unchanged since that capture are listed (others report
+# None), and other contexts were not measured.
+TRAFFIC_PER_UNIT = {("prefill128k", "attn"): ("query", 583.7e3), ("prefill128k", "indexer"): ("pair", 3.919),
+                    ("prefill128k", "topk"): ("pair", 4.286)}
 
 
 def roofline(wls, brk, pk, t_chunk):
@@ -426,9 +428,12 @@ def roofline(wls, brk, pk, t_chunk):
                        "peak_src": f"{pk['src']} bf16 sustained"}
     if "fused_select" in brk:
         ent["fused_select"] = idx_entry(brk["fused_select"], "the fused indexer + top-k")
-    for k, queries in (("attn", rows / len(wls)), ("indexer", min(t_chunk, rows)), ("topk", min(t_chunk, rows))):
-        per_q = TRAFFIC_PER_QUERY.get((wl.name, k))
-        ent[k]["traffic"] = None if per_q is None else per_q * queries   # bytes per launch
+    n_chunks = -(-rows // max(1, min(t_chunk, rows)))   # query chunks of the indexer and top-k
+    units = {"query": {"attn": rows / len(wls)},
+             "pair": {k: sum(causal_pairs(w) for w in wls) / n_chunks for k in ("indexer", "topk")}}
+    for k in ("attn", "indexer", "topk"):
+        unit, per = TRAFFIC_PER_UNIT.get((wl.name, k), (None, None))
+        ent[k]["traffic"] = None if per is None else per * units[unit][k]   # bytes per (average) launch
     top = max(("indexer", "topk", "attn"), key=lambda k: brk[k])
     r = dict(ent[top])
     r["kernel"] = top

@@ -35,9 +35,14 @@ def test_roofline_prefill_entries():
     flops = 128 * 2 * (576 + 512) * bench.selected_pairs(wl)
     assert r["achieved"] == pytest.approx(4 * flops / 451.4e-3 / 1e12)
     assert r["peak"] == 1382.4 and r["frac"] == pytest.approx(r["achieved"] / 1382.4)
-    per_q = bench.TRAFFIC_PER_QUERY.get(("prefill128k", "attn"))
+    unit, per_q = bench.TRAFFIC_PER_UNIT.get(("prefill128k", "attn"), (None, None))
     assert r["traffic"] == (None if per_q is None else pytest.approx(per_q * wl.B * wl.T))
     ix, tk, fs = r["others"]["indexer"], r["others"]["topk"], r["others"]["fused_select"]
+    # indexer and top-k traffic: per visible pair, times the pairs of an average 16384-query chunk
+    for name, ent in (("indexer", ix), ("topk", tk)):
+        unit, per_p = bench.TRAFFIC_PER_UNIT.get(("prefill128k", name), (None, None))
+        assert ent["traffic"] == (None if per_p is None else pytest.approx(per_p * bench.causal_pairs(wl) / 8))
+        assert unit in (None, "pair")
     assert ix["achieved"] == pytest.approx(2 * 64 * 128 * bench.causal_pairs(wl) / 89.3e-3 / 1e12)
     assert ix["peak"] == pytest.approx(2 * 1382.4)
     assert fs["achieved"] == pytest.approx(2 * 64 * 128 * bench.causal_pairs(wl) / 70.0e-3 / 1e12)

@@ -248,6 +248,60 @@ def test_topk_long_rows_exact_with_ties(reps):
         assert (np.diff(valid) > 0).all() and (got[valid.size:] == -1).all(), f"row {b}"
 
 
+def _select_rows(B, S, g):
+    """Rows of every kind the selection treats differently (fp32 scores given directly)."""
+    sc = torch.randn(B, 1, S, generator=g)
+    kinds = []
+    for b in range(B):
+        kind = b % 7
+        if kind == 1:    # small integers: thousands of keys tied at the pivot
+            sc[b, 0] = torch.randint(0, 50, (S,), generator=g).float()
+        elif kind == 2:  # all tied: the lowest ids win
+            sc[b, 0] = 0.5
+        elif kind == 3:  # sparse winners: every 7th key, far fewer than the zeros around them
+            sc[b, 0] = 0.0
+            sc[b, 0, ::7] = 1.0
+        elif kind == 4:  # ascending: every winner at the row's end (one CTA's part of a cluster)
+            sc[b, 0] = torch.arange(S, dtype=torch.float32) * 1e-3
+        elif kind == 5:  # the sampled blocks mislead the threshold: the first few sampled blocks
+            # (16 keys every sstride) hold the row's only high scores, enough of them to set the
+            # threshold above every other key, yet fewer than k keys in all
+            sstride = 16 * -(-S // (16 * 512))
+            nblk = -(-S // sstride)
+            ns = (nblk - 1) * 16 + min(16, S - (nblk - 1) * sstride)
+            r = -(-(3 * 2048 // 2) * ns // S)
+            for q in range(-(-r // 16) + 1):
+                sc[b, 0, q * sstride: q * sstride + 16] = 50.0
+        kinds.append(kind)
+    return sc, kinds
+
+
+@pytest.mark.parametrize("B,S", [(300, 20000), (6, 20000), (40, 40000), (12, 65536), (4, 131072), (2, 4500)])
+def test_topk_selection_paths_exact(B, S):
+    """The selection's every path against the oracle's sort, set for set: one CTA per row (300
+    rows), clusters of 2, 4 and 8 CTAs per row (6, 40, 12 and 4 rows), rows that fit the
+    candidate buffer whole (S = 4500), rows where the sampled threshold holds (normal, integer
+    ties, ascending: every winner in the last CTA's part) and rows where it cannot (all tied and
+    sparse winners: too many candidates; a misleading sample: too few), which take the full-row
+    path; one row of each batch sees fewer keys than k."""
+    k, T = 2048, 1
+    g = torch.Generator(device="cpu").manual_seed(11 + B)
+    sc, kinds = _select_rows(B, S, g)
+    ctx = torch.full((B,), S, dtype=torch.int32)
+    ctx[B - 1] = min(S, 1500)
+    if B > 2:
+        ctx[B - 2] = S - 777
+    idx = dsa.dsa_topk(sc.to(DEV), ctx.to(DEV), T, S, k)
+    got_all = P.to_np(idx)
+    for b in range(B):
+        n_valid = min(S, int(ctx[b]))
+        ref = O.topk_row(sc[b, 0].numpy(), n_valid, k)
+        got = got_all[b, 0]
+        valid = got[got >= 0]
+        assert np.array_equal(np.sort(valid), np.sort(ref[ref >= 0])), f"row {b} (kind {kinds[b]})"
+        assert (np.diff(valid) > 0).all() and (got[valid.size:] == -1).all(), f"row {b}"
+
+
 @pytest.mark.parametrize("name", ["tiny", "prefill32k"])
 def test_attention_ids_beyond_the_cache_are_skipped_and_flagged(name):
     """Selected ids at or beyond the cache length S_kv are skipped on the device like a -1 and
