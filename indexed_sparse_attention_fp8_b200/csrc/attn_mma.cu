@@ -311,6 +311,9 @@ sparse_attn_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16*
 __global__ void __launch_bounds__(128)
 attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int splits,
                     int64_t rows, int d_v, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  // Launched as a programmatic dependent of the attention kernel: it may start while that
+  // kernel drains, and waits here until the kernel has finished and its partials are visible.
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   const int64_t row = blockIdx.x;  // (b*T + t)*Hq + h
   float mx = -INFINITY;
   for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_lse[s * rows + row]);
@@ -338,8 +341,22 @@ attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ 
 
 int launch_attn_combine(const float* part_o, const float* part_lse, int splits, int64_t rows, int d_v,
                         uint16_t* out, float* lse, cudaStream_t stream) {
-  attn_combine_kernel<<<(unsigned)rows, 128, 0, stream>>>(part_o, part_lse, splits, rows, d_v,
-                                                         reinterpret_cast<__nv_bfloat16*>(out), lse);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)rows);
+  cfg.blockDim = dim3(128);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap its launch with the
+  attr[0].val.programmaticStreamSerializationAllowed = 1;             // attention kernel's tail
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_combine_kernel, part_o, part_lse, splits, rows, d_v,
+                                           reinterpret_cast<__nv_bfloat16*>(out), lse);
+  if (e != cudaSuccess) {
+    count_launch();
+    set_cuda_error(e);
+    return DSA_ERR_CUDA;
+  }
   return check_launch();
 }
 

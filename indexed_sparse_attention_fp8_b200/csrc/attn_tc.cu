@@ -116,6 +116,13 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
       ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
+// 32-byte global store (one whole sector per lane); the address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t a4,
+                                             uint32_t a5, uint32_t a6, uint32_t a7) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};\n" ::"l"(p), "r"(a0), "r"(a1), "r"(a2),
+               "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+               : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -204,7 +211,8 @@ __device__ __noinline__ void attn_load_q(const __nv_bfloat16* __restrict__ q, in
                                          uint32_t lane_off, uint32_t q_ready, int lane) {
   // q[head, 288*half .. +287] -> TMEM lane `head`, bf16 pairs packed per 32-bit column
   const uint4* qsrc = reinterpret_cast<const uint4*>(q + ((int64_t)bt * HQ + row) * DQK + 288 * half);
-  // two batches of loads (16 + 20 x 16 B; the rows were prefetched to L2 an item earlier)
+  // two batches of loads (16 + 20 x 16 B; the rows were asked into L2 an item earlier, or at the
+  // kernel start for a CTA's first item)
   {
     uint4 qa[16];
 #pragma unroll
@@ -253,6 +261,9 @@ __device__ __noinline__ bool attn_epilogue(int bt, int sp, int ntiles, float m_f
   const float lse_r = l_fin > 0.f ? (m_fin + log2f(l_fin)) * 0.69314718055994531f : -INFINITY;
   const bool have_o = good && ntiles > 0;
   const int64_t orow = (int64_t)bt * HQ + row;
+  // every row and column half starts a multiple of 32 B past the base: the base decides whether
+  // the 32-byte stores can be used
+  const bool wide = ((reinterpret_cast<uintptr_t>(part_o == nullptr ? (void*)out : (void*)part_o)) & 31u) == 0;
   if (part_o == nullptr) {
     __nv_bfloat16* dst = out + orow * DV + half * DVH;
 #pragma unroll 1
@@ -265,14 +276,23 @@ __device__ __noinline__ bool attn_epilogue(int bt, int sp, int ntiles, float m_f
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0.f;
       }
+      if (wide) {   // 32 B per store: each lane fills whole sectors of its row
 #pragma unroll
-      for (int i = 0; i < 32; i += 8) {
-        uint4 v;
-        v.x = pack2_bf16(o[i] * inv, o[i + 1] * inv);
-        v.y = pack2_bf16(o[i + 2] * inv, o[i + 3] * inv);
-        v.z = pack2_bf16(o[i + 4] * inv, o[i + 5] * inv);
-        v.w = pack2_bf16(o[i + 6] * inv, o[i + 7] * inv);
-        *reinterpret_cast<uint4*>(dst + c + i) = v;
+        for (int i = 0; i < 32; i += 16)
+          st_global_v8(dst + c + i, pack2_bf16(o[i] * inv, o[i + 1] * inv), pack2_bf16(o[i + 2] * inv, o[i + 3] * inv),
+                       pack2_bf16(o[i + 4] * inv, o[i + 5] * inv), pack2_bf16(o[i + 6] * inv, o[i + 7] * inv),
+                       pack2_bf16(o[i + 8] * inv, o[i + 9] * inv), pack2_bf16(o[i + 10] * inv, o[i + 11] * inv),
+                       pack2_bf16(o[i + 12] * inv, o[i + 13] * inv), pack2_bf16(o[i + 14] * inv, o[i + 15] * inv));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          uint4 v;
+          v.x = pack2_bf16(o[i] * inv, o[i + 1] * inv);
+          v.y = pack2_bf16(o[i + 2] * inv, o[i + 3] * inv);
+          v.z = pack2_bf16(o[i + 4] * inv, o[i + 5] * inv);
+          v.w = pack2_bf16(o[i + 6] * inv, o[i + 7] * inv);
+          *reinterpret_cast<uint4*>(dst + c + i) = v;
+        }
       }
     }
     if (lse != nullptr && half == 0) lse[orow] = lse_r;
@@ -289,9 +309,17 @@ __device__ __noinline__ bool attn_epilogue(int bt, int sp, int ntiles, float m_f
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0.f;
       }
+      if (wide) {
 #pragma unroll
-      for (int i = 0; i < 32; i += 4)
-        *reinterpret_cast<float4*>(dst + c + i) = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+        for (int i = 0; i < 32; i += 8)
+          st_global_v8(dst + c + i, __float_as_uint(o[i] * inv), __float_as_uint(o[i + 1] * inv),
+                       __float_as_uint(o[i + 2] * inv), __float_as_uint(o[i + 3] * inv), __float_as_uint(o[i + 4] * inv),
+                       __float_as_uint(o[i + 5] * inv), __float_as_uint(o[i + 6] * inv), __float_as_uint(o[i + 7] * inv));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(dst + c + i) = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+      }
     }
     if (half == 0) part_lse[(int64_t)sp * rows + orow] = lse_r;
   }
@@ -330,6 +358,13 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
   volatile int* abort = reinterpret_cast<volatile int*>(sgen + OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // a split-key launch's combine kernel (a programmatic dependent) may be scheduled from now on;
+  // it waits for this grid's completion before it reads anything
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  if (threadIdx.x == 0 && (int)blockIdx.x < items)   // the first item's q: to L2 while the CTA sets up
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(q + (int64_t)((int)blockIdx.x % nbt) * HQ * DQK),
+                 "r"((uint32_t)(HQ * DQK * 2))
+                 : "memory");
   const int half = (int)cluster_rank();       // 0 or 1: score columns 288*half.., output columns 256*half..
   const uint32_t partner = (uint32_t)(half ^ 1);
   // Work item it = (query bt = it % nbt, key split sp = it / nbt); the cluster takes items

@@ -11,7 +11,7 @@
 // one thread, and the per-head logits never leave the SM.
 //
 // Persistent kernel, one CTA per SM, warp-specialised:
-//   warp 0      TMA producer: key tiles (ring of NA stages), query blocks + head weights
+//   warp 0      TMA producer: key tiles (ring of C::NA stages), query blocks + head weights
 //               (2 stages), all through mbarrier transaction counts
 //   warp 1      TMEM owner and MMA issuer: d_I/32 tcgen05.mma (kind::f8f6f4, M=128, N) per
 //               key tile into one of two TMEM accumulators
@@ -32,11 +32,12 @@ using namespace tc;
 
 constexpr int KTILE = 128;        // keys per tile (MMA M)
 constexpr int KC = 32;            // key tiles per work item
-constexpr int NA = 6;             // key-tile stages
 constexpr int NUM_THREADS = 320;  // 10 warps
 
 template <int H, int D, int QB>
 struct IdxCfg {
+  // key-tile stages: decode (one query per block) streams the keys and wants many bytes in flight
+  static constexpr int NA = QB == 1 ? 9 : 6;
   static constexpr int N = QB * H;                 // MMA N: (query, head) columns
   static constexpr int A_BYTES = KTILE * D;        // one key tile
   static constexpr int B_BYTES = N * D;            // one query block
@@ -136,12 +137,12 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
   uint8_t* sgen = smem_raw + (sbase - sraw);
   const uint32_t bar0 = sbase + C::OFF_BAR;
   auto a_full = [&](int s) { return bar0 + 8u * s; };
-  auto a_empty = [&](int s) { return bar0 + 8u * (NA + s); };
-  auto b_full = [&](int s) { return bar0 + 8u * (2 * NA + s); };
-  auto b_empty = [&](int s) { return bar0 + 8u * (2 * NA + 2 + s); };
-  auto acc_full = [&](int s) { return bar0 + 8u * (2 * NA + 4 + s); };
-  auto acc_empty = [&](int s) { return bar0 + 8u * (2 * NA + 6 + s); };
-  const uint32_t mma_drain = bar0 + 8u * (2 * NA + 8);   // completes when every issued MMA has
+  auto a_empty = [&](int s) { return bar0 + 8u * (C::NA + s); };
+  auto b_full = [&](int s) { return bar0 + 8u * (2 * C::NA + s); };
+  auto b_empty = [&](int s) { return bar0 + 8u * (2 * C::NA + 2 + s); };
+  auto acc_full = [&](int s) { return bar0 + 8u * (2 * C::NA + 4 + s); };
+  auto acc_empty = [&](int s) { return bar0 + 8u * (2 * C::NA + 6 + s); };
+  const uint32_t mma_drain = bar0 + 8u * (2 * C::NA + 8);   // completes when every issued MMA has
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + C::OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(sgen + C::OFF_MISC + 4);
 
@@ -151,7 +152,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
   const int items = B * nqb * nkc;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NA; ++i) {
+    for (int i = 0; i < C::NA; ++i) {
       mbar_init(a_full(i), 1);
       mbar_init(a_empty(i), 1);
     }
@@ -195,8 +196,8 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       }
       ++b_cnt;
       for (int kt = g.kt0; kt < g.kt1; ++kt) {
-        const int as = a_cnt % NA;
-        if (!(ok = mbar_wait_warp(a_empty(as), ((a_cnt / NA) & 1) ^ 1, abort, wlim))) break;
+        const int as = a_cnt % C::NA;
+        if (!(ok = mbar_wait_warp(a_empty(as), ((a_cnt / C::NA) & 1) ^ 1, abort, wlim))) break;
         if (lane == 0) {
           // contiguous: row b*S_max + s of the cache; paged: the tile's page (a tile never
           // straddles one); a bad page id loads past the map's extent, which reads zeros
@@ -217,8 +218,8 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
     }
     // drain, whether this warp gave up or not: the copies it issued land before the CTA can leave
     // (after a normal run they landed long ago; after any role gave up some may be in flight)
-    for (uint32_t i = (a_cnt > NA ? a_cnt - NA : 0); i < a_cnt; ++i)
-      mbar_wait_bounded(a_full(i % NA), (i / NA) & 1, 100000000ull);
+    for (uint32_t i = (a_cnt > C::NA ? a_cnt - C::NA : 0); i < a_cnt; ++i)
+      mbar_wait_bounded(a_full(i % C::NA), (i / C::NA) & 1, 100000000ull);
     for (uint32_t i = (b_cnt > 2 ? b_cnt - 2 : 0); i < b_cnt; ++i)
       mbar_wait_bounded(b_full(i & 1), (i >> 1) & 1, 100000000ull);
   } else if (warp == 1) {
@@ -232,9 +233,9 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
       if (!(ok = mbar_wait_warp(b_full(bs), (b_cnt >> 1) & 1, abort, wlim))) break;
       const uint32_t b_addr = sbase + C::OFF_B + bs * C::B_BYTES;
       for (int kt = g.kt0; kt < g.kt1; ++kt) {
-        const int as = a_cnt % NA;
+        const int as = a_cnt % C::NA;
         const int ab = acc_cnt & 1;
-        if (!(ok = mbar_wait_warp(a_full(as), (a_cnt / NA) & 1, abort, wlim))) break;
+        if (!(ok = mbar_wait_warp(a_full(as), (a_cnt / C::NA) & 1, abort, wlim))) break;
         if (!(ok = mbar_wait_warp(acc_empty(ab), ((acc_cnt >> 1) & 1) ^ 1, abort, wlim))) break;
         tc_fence_after();
         if (lane == 0) {
