@@ -238,8 +238,8 @@ int dsa_sparse_attn_noalloc(const uint16_t* q, const uint16_t* kv, const uint16_
  * dsa_index_pool - IndexPool ("What changed": four indexer keys pooled into one):
  *     k_pool[b, g, :] = e4m3(((k[4g] + k[4g+1]) + (k[4g+2] + k[4g+3])) * 0.25)
  * and for pool = 2 or 8 the same mean over 2 or 8 keys (a balanced pairwise sum times
- * 1/pool; exact in fp32 before the requantisation, which is the only rounding) * with the sum in fp32 on the decoded keys and the requantisation round-to-nearest-even,
- * saturating at +-448.
+ * 1/pool).  The sum runs in fp32 on the decoded keys and is exact there, so the requantisation
+ * (round-to-nearest-even, saturating at +-448) is the only rounding.
  *   k_idx [B, S_max, d_I] e4m3 (or its page pool when paging != NULL)
  *   -> k_pool [B, S_max/pool, d_I] e4m3 (always contiguous).
  * Supported: pool in {2, 4, 8}, S_max % pool == 0, d_I % 16 == 0.
