@@ -309,7 +309,7 @@ def run_ours(args, rank, world, dev):
 
 def breakdown(parts, ws, t_chunk, stream, dsa, reps, fused=True):
     """Average device time of each step of the group per step over `reps` steps, CUDA events on
-    `stream`, summed over this rank's parts: the pool kernel, the selection as the group call
+    `stream` (the launches queued ahead of the GPU), summed over this rank's parts: the pool kernel, the selection as the group call
     runs it (the indexer writing full score rows, then the row top-k, per query chunk), and each
     attention layer; with `fused`, also the fused selection (dsa_index_select) over the same
     chunks, for comparison."""
@@ -331,6 +331,10 @@ def breakdown(parts, ws, t_chunk, stream, dsa, reps, fused=True):
                                  device=dev)
         for rep in range(reps):
             marks = []
+            # hold the stream for a few ms, so every launch below is queued before the GPU reaches
+            # it: the marks then time the kernels back to back, not the host's calls (which, for
+            # the short decode kernels, take longer than the kernels)
+            torch.cuda._sleep(5_000_000)
             keys = ind["k_idx"]
             if wl.pool > 1:
                 a, b = ev(), ev()

@@ -10,7 +10,7 @@
 // every query of the block for one key, so the weighted ReLU reduction over heads runs in
 // one thread, and the per-head logits never leave the SM.
 //
-// Persistent kernel, one CTA per SM, warp-specialised:
+// Persistent kernel, one CTA per SM (two for the one-query decode shape), warp-specialised:
 //   warp 0      TMA producer: key tiles (ring of C::NA stages), query blocks + head weights
 //               (2 stages), all through mbarrier transaction counts
 //   warp 1      TMEM owner and MMA issuer: d_I/32 tcgen05.mma (kind::f8f6f4, M=128, N) per
@@ -36,8 +36,11 @@ constexpr int NUM_THREADS = 320;  // 10 warps
 
 template <int H, int D, int QB>
 struct IdxCfg {
-  // key-tile stages: decode (one query per block) streams the keys and wants many bytes in flight
-  static constexpr int NA = QB == 1 ? 9 : 6;
+  // Decode (one query per block, N = 64): only the 4 epilogue warps of one column half have work,
+  // one per SM sub-partition, so two CTAs share each SM (4-stage key rings, 96 registers) and
+  // twice the epilogue warps hide each other's TMEM-load and reduction latency.
+  static constexpr int NA = QB == 1 ? 4 : 6;       // key-tile stages
+  static constexpr int CTAS_PER_SM = QB == 1 ? 2 : 1;
   static constexpr int N = QB * H;                 // MMA N: (query, head) columns
   static constexpr int A_BYTES = KTILE * D;        // one key tile
   static constexpr int B_BYTES = N * D;            // one query block
@@ -123,7 +126,7 @@ __device__ __forceinline__ void cand_append(bool pass, float val, int s, int* __
 // reaches tau[row]; `cnt` counts them per row.  row_flag (optional): only the work items
 // holding a flagged query run.
 template <int H, int D, int QB, bool CAND>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(NUM_THREADS, IdxCfg<H, D, QB>::CTAS_PER_SM)
 index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                        const float* __restrict__ w, const int32_t* __restrict__ ctx_len, int B, int T, int S_max,
                        int pool, int t_begin, int t_count, float* __restrict__ scores, int64_t ld, PageMap pm,
@@ -552,7 +555,7 @@ int launch_tc(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const 
   const int nqb = (t_count + QB - 1) / QB;
   const int nkc = ((S_max + KTILE - 1) / KTILE + KC - 1) / KC;
   const int64_t items = (int64_t)B * nqb * nkc;
-  const int grid = (int)std::min<int64_t>(items, num_sms());
+  const int grid = (int)std::min<int64_t>(items, (int64_t)C::CTAS_PER_SM * num_sms());
   kern<<<grid, NUM_THREADS, C::SMEM, stream>>>(mk, mq, w, ctx_len, B, T, S_max, pool, t_begin, t_count, scores, ld,
                                                pm, md.tau, md.cand, md.cnt, md.cap, md.row_flag);
   return check_launch();
