@@ -272,6 +272,7 @@ __device__ __noinline__ bool attn_epilogue(int bt, int sp, int ntiles, float m_f
       if (have_o) {
         tmem_ld32(tmem + lane_off + COL_O + c, o);
         tmem_ld_wait();
+        launder(o);
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0.f;
@@ -305,6 +306,7 @@ __device__ __noinline__ bool attn_epilogue(int bt, int sp, int ntiles, float m_f
       if (have_o) {
         tmem_ld32(tmem + lane_off + COL_O + c, o);
         tmem_ld_wait();
+        launder(o);
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0.f;
@@ -571,6 +573,8 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
       tmem_ld32(tmem + lane_off + COL_S, *reinterpret_cast<float(*)[32]>(sv));
       tmem_ld32(tmem + lane_off + COL_S + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
       tmem_ld_wait();
+      launder(*reinterpret_cast<float(*)[32]>(sv));   // no use of the scores before the wait
+      launder(*reinterpret_cast<float(*)[32]>(sv + 32));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_empty);
@@ -670,6 +674,7 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
             float o[32];
             tmem_ld32(tmem + lane_off + COL_O + c, o);
             tmem_ld_wait();
+            launder(o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
             tmem_st32(tmem + lane_off + COL_O + c, o);

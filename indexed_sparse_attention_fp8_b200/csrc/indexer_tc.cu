@@ -462,6 +462,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
           float v[2][32];
           tmem_ld32(taddr, v[0]);
           tmem_ld_wait();
+          launder(v[0]);
           uint64_t a2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
           for (int c = 0; c < C::CHUNKS; ++c) {
@@ -492,7 +493,10 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_
                 store(c * (32 / H) + qc, s, (x0 + x1) + (x2 + x3));
               }
             }
-            if (c + 1 < C::CHUNKS) tmem_ld_wait();
+            if (c + 1 < C::CHUNKS) {
+              tmem_ld_wait();
+              launder(v[(c + 1) & 1]);
+            }
           }
           tc_fence_before();
           __syncwarp();
