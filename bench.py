@@ -389,8 +389,8 @@ def breakdown(parts, ws, t_chunk, stream, dsa, reps, fused=True):
 # the score rows, 4 B per pair written and read back).  A launch's traffic is the figure times
 # the units it processes.  Only kernels unchanged since that capture are listed (others report
 # None), and other contexts were not measured.
-TRAFFIC_PER_UNIT = {("prefill128k", "attn"): ("query", 604.1e3), ("prefill128k", "indexer"): ("pair", 3.921),
-                    ("prefill128k", "topk"): ("pair", 4.286)}
+TRAFFIC_PER_UNIT = {("prefill128k", "attn"): ("query", 606.1e3), ("prefill128k", "indexer"): ("pair", 3.916),
+                    ("prefill128k", "topk"): ("pair", 4.285)}
 
 
 def roofline(wls, brk, pk, t_chunk):
