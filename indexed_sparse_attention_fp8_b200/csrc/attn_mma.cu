@@ -307,9 +307,11 @@ sparse_attn_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16*
   }
 }
 
-// Merge split-key partials: O = sum_s exp(lse_s - lse) O_s, lse = log sum_s exp(lse_s).
+// Merge split-key partials: O = sum_s exp(lse_s - lse) O_s, lse = log sum_s exp(lse_s).  The
+// partials O_s are fp32, or bf16 when bf16_parts (the MLA kernel's: half the bytes to write and
+// read back; lse_s stay fp32).
 __global__ void __launch_bounds__(128)
-attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int splits,
+attn_combine_kernel(const void* __restrict__ part_o, bool bf16_parts, const float* __restrict__ part_lse, int splits,
                     int64_t rows, int d_v, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
   // Launched as a programmatic dependent of the attention kernel: it may start while that
   // kernel drains, and waits here until the kernel has finished and its partials are visible.
@@ -328,7 +330,11 @@ attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ 
   for (int c = threadIdx.x * 2; c < d_v; c += blockDim.x * 2) {
     float2 acc = make_float2(0.f, 0.f);
     for (int s = 0; s < splits; ++s) {
-      const float2 v = *reinterpret_cast<const float2*>(part_o + (s * rows + row) * d_v + c);
+      const int64_t at = (s * rows + row) * d_v + c;
+      const float2 v = bf16_parts
+                           ? __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
+                                 reinterpret_cast<const __nv_bfloat16*>(part_o) + at))
+                           : *reinterpret_cast<const float2*>(reinterpret_cast<const float*>(part_o) + at);
       acc.x += wts[s] * v.x;
       acc.y += wts[s] * v.y;
     }
@@ -339,8 +345,8 @@ attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ 
 
 }  // namespace
 
-int launch_attn_combine(const float* part_o, const float* part_lse, int splits, int64_t rows, int d_v,
-                        uint16_t* out, float* lse, cudaStream_t stream) {
+int launch_attn_combine(const void* part_o, bool bf16_parts, const float* part_lse, int splits, int64_t rows,
+                        int d_v, uint16_t* out, float* lse, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)rows);
   cfg.blockDim = dim3(128);
@@ -350,7 +356,7 @@ int launch_attn_combine(const float* part_o, const float* part_lse, int splits, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;             // attention kernel's tail
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_combine_kernel, part_o, part_lse, splits, rows, d_v,
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_combine_kernel, part_o, bf16_parts, part_lse, splits, rows, d_v,
                                            reinterpret_cast<__nv_bfloat16*>(out), lse);
   if (e != cudaSuccess) {
     count_launch();
@@ -394,7 +400,7 @@ int launch_cfg(const uint16_t* q, const uint16_t* kv, const uint16_t* v, int64_t
       scale_log2, reinterpret_cast<__nv_bfloat16*>(out), lse, part_o, part_lse, pm);
   int st = check_launch();
   if (st != DSA_OK || splits == 1) return st;
-  return launch_attn_combine(part_o, part_lse, splits, rows, D_V, out, lse, stream);
+  return launch_attn_combine(part_o, false, part_lse, splits, rows, D_V, out, lse, stream);
 }
 
 }  // namespace

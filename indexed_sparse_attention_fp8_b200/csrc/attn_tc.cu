@@ -252,7 +252,7 @@ __device__ __noinline__ void attn_load_q(const __nv_bfloat16* __restrict__ q, in
 __device__ __noinline__ bool attn_epilogue(int bt, int sp, int ntiles, float m_fin, float l_fin, uint32_t g_last,
                                            bool good, int nbt, int row, int half, uint32_t tmem, uint32_t lane_off,
                                            uint32_t pv_done, volatile int* abort, __nv_bfloat16* __restrict__ out,
-                                           float* __restrict__ lse, float* __restrict__ part_o,
+                                           float* __restrict__ lse, __nv_bfloat16* __restrict__ part_o,
                                            float* __restrict__ part_lse) {
   if (good && ntiles > 0) good = mbar_wait(pv_done, g_last & 1, abort, wait_limit());
   good = __all_sync(0xffffffffu, good);   // the TMEM reads below are warp-collective
@@ -299,7 +299,7 @@ __device__ __noinline__ bool attn_epilogue(int bt, int sp, int ntiles, float m_f
     if (lse != nullptr && half == 0) lse[orow] = lse_r;
   } else {
     const int64_t rows = (int64_t)nbt * HQ;
-    float* dst = part_o + ((int64_t)sp * rows + orow) * DV + half * DVH;
+    __nv_bfloat16* dst = part_o + ((int64_t)sp * rows + orow) * DV + half * DVH;   // bf16 partial
 #pragma unroll 1
     for (int c = 0; c < DVH; c += 32) {
       float o[32];
@@ -313,14 +313,21 @@ __device__ __noinline__ bool attn_epilogue(int bt, int sp, int ntiles, float m_f
       }
       if (wide) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 8)
-          st_global_v8(dst + c + i, __float_as_uint(o[i] * inv), __float_as_uint(o[i + 1] * inv),
-                       __float_as_uint(o[i + 2] * inv), __float_as_uint(o[i + 3] * inv), __float_as_uint(o[i + 4] * inv),
-                       __float_as_uint(o[i + 5] * inv), __float_as_uint(o[i + 6] * inv), __float_as_uint(o[i + 7] * inv));
+        for (int i = 0; i < 32; i += 16)
+          st_global_v8(dst + c + i, pack2_bf16(o[i] * inv, o[i + 1] * inv), pack2_bf16(o[i + 2] * inv, o[i + 3] * inv),
+                       pack2_bf16(o[i + 4] * inv, o[i + 5] * inv), pack2_bf16(o[i + 6] * inv, o[i + 7] * inv),
+                       pack2_bf16(o[i + 8] * inv, o[i + 9] * inv), pack2_bf16(o[i + 10] * inv, o[i + 11] * inv),
+                       pack2_bf16(o[i + 12] * inv, o[i + 13] * inv), pack2_bf16(o[i + 14] * inv, o[i + 15] * inv));
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(dst + c + i) = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+        for (int i = 0; i < 32; i += 8) {
+          uint4 v;
+          v.x = pack2_bf16(o[i] * inv, o[i + 1] * inv);
+          v.y = pack2_bf16(o[i + 2] * inv, o[i + 3] * inv);
+          v.z = pack2_bf16(o[i + 4] * inv, o[i + 5] * inv);
+          v.w = pack2_bf16(o[i + 6] * inv, o[i + 7] * inv);
+          *reinterpret_cast<uint4*>(dst + c + i) = v;
+        }
       }
     }
     if (half == 0) part_lse[(int64_t)sp * rows + orow] = lse_r;
@@ -336,7 +343,7 @@ __global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(THREADS, 1)
 sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv, int64_t kv_rs,
                      int64_t kv_bs, int S_kv, const int32_t* __restrict__ idx, int T, int nbt, int items, int k,
                      int keys_per_split, float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-                     float* __restrict__ part_o, float* __restrict__ part_lse, PageMap pm) {
+                     __nv_bfloat16* __restrict__ part_o, float* __restrict__ part_lse, PageMap pm) {
   const uint64_t wlim = wait_limit();   // the bounded waits' time limit, read once
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
@@ -779,11 +786,12 @@ int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, i
   int kps = (k + splits - 1) / splits;
   kps = (kps + NK - 1) / NK * NK;
   const int64_t rows = (int64_t)B * T * HQ;
-  float* part_o = nullptr;
+  // split partials: O_s as bf16 (normalised, so within bf16's range), then lse_s as fp32
+  __nv_bfloat16* part_o = nullptr;
   float* part_lse = nullptr;
   if (splits > 1) {
-    part_o = reinterpret_cast<float*>(ws);
-    part_lse = part_o + (int64_t)splits * rows * DV;
+    part_o = reinterpret_cast<__nv_bfloat16*>(ws);
+    part_lse = reinterpret_cast<float*>(part_o + (int64_t)splits * rows * DV);
   }
   // persistent: one cluster (CTA pair) per two SMs, each serving items (query, key split) in turn
   const int nbt = B * T;
@@ -795,7 +803,7 @@ int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, i
       items, k, kps, sm_scale * 1.4426950408889634f, reinterpret_cast<__nv_bfloat16*>(out), lse, part_o, part_lse, pm);
   int st = check_launch();
   if (st != DSA_OK || splits == 1) return st;
-  return launch_attn_combine(part_o, part_lse, splits, rows, DV, out, lse, stream);
+  return launch_attn_combine(part_o, true, part_lse, splits, rows, DV, out, lse, stream);
 }
 
 void attn_tc_set_wait_limit(uint64_t ns) {

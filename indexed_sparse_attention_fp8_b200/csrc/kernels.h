@@ -77,8 +77,8 @@ int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, i
                          void* ws, int splits, const PageMap& pm, cudaStream_t stream);
 unsigned int attn_tc_take_status();
 // Merges split-key attention partials (normalised fp32 O and log-sum-exp per split).
-int launch_attn_combine(const float* part_o, const float* part_lse, int splits, int64_t rows, int d_v,
-                        uint16_t* out, float* lse, cudaStream_t stream);
+int launch_attn_combine(const void* part_o, bool bf16_parts, const float* part_lse, int splits, int64_t rows,
+                        int d_v, uint16_t* out, float* lse, cudaStream_t stream);
 
 // IndexPool over `pool` (2, 4 or 8) consecutive keys.
 int launch_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool, uint8_t* k_pool,
