@@ -17,8 +17,11 @@
  *   Positions   Sequence b holds ctx_len[b] keys (rows 0..ctx_len[b]-1 of its caches) and T
  *               new queries at its end: query t sits at position pos(b,t) = ctx_len[b]-T+t.
  *               A key row s (or pooled block s when pool > 1) is visible to the query iff
- *               pool*s <= pos(b,t).  ctx_len is a DEVICE array of B int32, and the caller
- *               guarantees T <= ctx_len[b] <= S_max * pool.
+ *               pool*s <= pos(b,t).  ctx_len is a DEVICE array of B int32, normally
+ *               T <= ctx_len[b] <= S_max * pool; the scoring and selection kernels also
+ *               accept values outside that range (a query at pos < 0 sees no key, and only
+ *               the S_max rows present are ever visible), which the key-sharded form below
+ *               relies on.
  *   Types       e4m3 = OCP FP8 E4M3 ("e4m3fn") codes stored as uint8, unit scale.
  *               bf16 = bfloat16 stored as uint16.  Scores and weights are IEEE fp32.
  *   Layouts     Row-major, innermost dimension last, as written in each comment.
@@ -290,6 +293,54 @@ typedef struct dsa_group_args {
  * chunk that fits in the ws_bytes it is given. */
 size_t dsa_group_workspace_size(const dsa_group_args* args, int t_chunk);
 int dsa_group_forward(const dsa_group_args* args, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * Context parallelism: the key caches sharded over ranks, rank r holding the contiguous key
+ * rows [s0_r, s0_r + len_r) of every sequence.  The pages describe no multi-GPU form; this is
+ * the exchange form of the same selection ("DeepSeek Sparse Attention", Stage 2: the top-k of
+ * the whole row) and attention ("The Time has Come": attend only to the selected tokens).  Per
+ * rank and query chunk:
+ *   1. dsa_index_scores and dsa_topk over the rank's shard (S_max = len_r), with ctx_len - s0
+ *      as the context lengths: positions and the causal rule then refer to the shard's own
+ *      rows (a shard wholly after a query's position selects nothing for it, one wholly
+ *      before it offers all its rows);
+ *   2. dsa_gather_selected: the shard's selection as (score, global id) candidates;
+ *   3. the caller all-gathers the candidates of every rank (e.g. NCCL all_gather);
+ *   4. dsa_topk_merge: the exact top-k of the union, the ids dsa_topk would give over the
+ *      whole row, identical on every rank;
+ *   5. per layer: dsa_idx_localize, then dsa_sparse_attn over the rank's rows (want lse);
+ *   6. the caller all-gathers every rank's (O, lse); dsa_attn_combine merges them.
+ * pool must be 1.  Errors and asynchrony as for the other calls.
+ * ------------------------------------------------------------------------------------ */
+
+/* Candidates of a shard's selection: for rows t_begin .. t_begin+t_count-1 of
+ * idx [B, T, k] (ids local to the shard, from dsa_topk on scores [B, t_count, ld]),
+ * cand_score/cand_id [B, t_count, k] = (scores[row][id], id + id_offset), or (-inf, -1) for a
+ * -1 entry.  Supported: 1 <= k <= 2048. */
+int dsa_gather_selected(const float* scores, int64_t ld, const int32_t* idx, int B, int T, int t_begin, int t_count,
+                        int k, int32_t id_offset, float* cand_score, int32_t* cand_id, void* stream);
+
+/* The exact top-k (ties toward lower key id, ids ascending, -1 padding) of the union of
+ * n_parts shard selections: part p is cand_score/cand_id + p * part_stride, each
+ * [B, t_count, kc] as dsa_gather_selected writes them (kc >= k).  The rows are those of
+ * queries t_begin .. of a context of ctx_len[b] keys (S_total key rows per sequence); a row with
+ * at most k visible keys selects them all.  idx [B, T, k] int32 out (rows t_begin.. written).
+ * Supported: 1 <= k <= 2048, n_parts * kc <= 16384. */
+int dsa_topk_merge(const float* cand_score, const int32_t* cand_id, int n_parts, int64_t part_stride, int kc,
+                   const int32_t* ctx_len, int B, int T, int S_total, int t_begin, int t_count, int k, int32_t* idx,
+                   void* stream);
+
+/* out[i] = idx[i] - s0 when s0 <= idx[i] < s0 + s_len, else -1 (n entries): a selection of
+ * global key ids as ids into the shard, for dsa_sparse_attn over the shard's rows. */
+int dsa_idx_localize(const int32_t* idx, int64_t n, int32_t s0, int32_t s_len, int32_t* out, void* stream);
+
+/* Merge of n_parts attention results over disjoint key sets: part_o [n_parts, rows, d_v] bf16
+ * (each normalised over its keys, as dsa_sparse_attn writes it) and part_lse [n_parts, rows]
+ * fp32 (-inf for a part with no keys) ->
+ *     out[r] = sum_p exp(lse_p - lse) part_o[p][r],  lse[r] = log sum_p exp(lse_p)
+ * as bf16 (lse may be NULL).  Supported: 1 <= n_parts <= 16, d_v even. */
+int dsa_attn_combine(const uint16_t* part_o, const float* part_lse, int n_parts, int64_t rows, int d_v, uint16_t* out,
+                     float* lse, void* stream);
 
 #ifdef __cplusplus
 }

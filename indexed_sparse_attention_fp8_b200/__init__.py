@@ -96,6 +96,12 @@ _SIGS = {
                                          ctypes.POINTER(Paging), _c_p]),
     "dsa_group_workspace_size": (_c_sz, [ctypes.POINTER(GroupArgs), _c_int]),
     "dsa_group_forward": (_c_int, [ctypes.POINTER(GroupArgs), _c_p, _c_sz, _c_p]),
+    "dsa_gather_selected": (_c_int, [_c_p, _c_i64, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, _c_p,
+                                     _c_p]),
+    "dsa_topk_merge": (_c_int, [_c_p, _c_p, _c_int, _c_i64, _c_int, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                _c_int, _c_p, _c_p]),
+    "dsa_idx_localize": (_c_int, [_c_p, _c_i64, _c_int, _c_int, _c_p, _c_p]),
+    "dsa_attn_combine": (_c_int, [_c_p, _c_p, _c_int, _c_i64, _c_int, _c_p, _c_p, _c_p]),
 }
 
 
@@ -438,3 +444,73 @@ def dsa_group_forward(q_idx, w, k_idx, ctx_len, topk: int, layers: Sequence[dict
     if ws is None:
         ws = torch.empty(g.workspace_size(t_chunk or q_idx.shape[1]), dtype=torch.uint8, device=g.device)
     return g.forward(ws, stream)
+
+
+# ---------------------------------------------------------------- context parallelism (see dsa.h)
+
+def dsa_gather_selected(scores: torch.Tensor, idx: torch.Tensor, t_begin: int, id_offset: int,
+                        cand_score: Optional[torch.Tensor] = None, cand_id: Optional[torch.Tensor] = None,
+                        stream=None):
+    """A shard's selection (rows t_begin.. of idx [B, T, k], local ids) as candidates
+    (score [B, t_count, k] f32, global id [B, t_count, k] i32), from scores [B, t_count, ld]."""
+    B, tc, ld = scores.shape
+    _, T, k = idx.shape
+    _layout("scores", scores, torch.float32, (B, tc, -1), (tc * scores.stride(1), -1, 1))
+    _layout("idx", idx, torch.int32, (B, T, k))
+    if cand_score is None:
+        cand_score = torch.empty((B, tc, k), dtype=torch.float32, device=scores.device)
+    if cand_id is None:
+        cand_id = torch.empty((B, tc, k), dtype=torch.int32, device=scores.device)
+    _layout("cand_score", cand_score, torch.float32, (B, tc, k))
+    _layout("cand_id", cand_id, torch.int32, (B, tc, k))
+    _check("dsa_gather_selected", _lib().dsa_gather_selected(_ptr(scores), scores.stride(1), _ptr(idx), B, T, t_begin,
+                                                             tc, k, id_offset, _ptr(cand_score), _ptr(cand_id),
+                                                             _stream(stream)))
+    return cand_score, cand_id
+
+
+def dsa_topk_merge(cand_score: torch.Tensor, cand_id: torch.Tensor, ctx_len: torch.Tensor, T: int, S_total: int, k: int,
+                   t_begin: int = 0, idx: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The exact top-k of the union of n_parts shard selections: cand_score / cand_id
+    [n_parts, B, t_count, kc] -> idx [B, T, k] (rows t_begin.. written)."""
+    P, B, tc, kc = cand_score.shape
+    _layout("cand_score", cand_score, torch.float32, (P, B, tc, kc))
+    _layout("cand_id", cand_id, torch.int32, (P, B, tc, kc))
+    _layout("ctx_len", ctx_len, torch.int32, (B,))
+    if idx is None:
+        idx = torch.full((B, T, k), -1, dtype=torch.int32, device=cand_score.device)
+    _layout("idx", idx, torch.int32, (B, T, k))
+    _check("dsa_topk_merge", _lib().dsa_topk_merge(_ptr(cand_score), _ptr(cand_id), P, B * tc * kc, kc, _ptr(ctx_len),
+                                                   B, T, S_total, t_begin, tc, k, _ptr(idx), _stream(stream)))
+    return idx
+
+
+def dsa_idx_localize(idx: torch.Tensor, s0: int, s_len: int, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """Global key ids -> ids into the shard [s0, s0 + s_len) (others -1), same shape."""
+    _layout("idx", idx, torch.int32, tuple(idx.shape))
+    if out is None:
+        out = torch.empty_like(idx)
+    _layout("out", out, torch.int32, tuple(idx.shape))
+    _check("dsa_idx_localize", _lib().dsa_idx_localize(_ptr(idx), idx.numel(), s0, s_len, _ptr(out), _stream(stream)))
+    return out
+
+
+def dsa_attn_combine(part_o: torch.Tensor, part_lse: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     lse: Optional[torch.Tensor] = None, want_lse: bool = False, stream=None):
+    """Merge of attention results over disjoint key sets: part_o [n, ..., d_v] bf16, part_lse
+    [n, ...] f32 -> (out [..., d_v] bf16, lse [...] f32 or None)."""
+    n, d_v = part_o.shape[0], part_o.shape[-1]
+    _layout("part_o", part_o, torch.bfloat16, tuple(part_o.shape))
+    _layout("part_lse", part_lse, torch.float32, tuple(part_o.shape[:-1]))
+    rows = part_lse[0].numel()
+    if out is None:
+        out = torch.empty(part_o.shape[1:], dtype=torch.bfloat16, device=part_o.device)
+    _layout("out", out, torch.bfloat16, tuple(part_o.shape[1:]))
+    if lse is None and want_lse:
+        lse = torch.empty(part_lse.shape[1:], dtype=torch.float32, device=part_o.device)
+    if lse is not None:
+        _layout("lse", lse, torch.float32, tuple(part_lse.shape[1:]))
+    _check("dsa_attn_combine", _lib().dsa_attn_combine(_ptr(part_o), _ptr(part_lse), n, rows, d_v, _ptr(out), _ptr(lse),
+                                                       _stream(stream)))
+    return out, lse

@@ -416,4 +416,47 @@ int dsa_group_forward(const dsa_group_args* a, void* ws, size_t ws_bytes, void* 
   return DSA_OK;
 }
 
+// ---- context parallelism (keys sharded over ranks; the exchange itself is the caller's)
+
+int dsa_gather_selected(const float* scores, int64_t ld, const int32_t* idx, int B, int T, int t_begin, int t_count,
+                        int k, int32_t id_offset, float* cand_score, int32_t* cand_id, void* stream) {
+  if (B < 0 || T < 1 || t_begin < 0 || t_count < 0 || t_begin + t_count > T || k < 1 || k > 2048 || ld < 1 ||
+      id_offset < 0)
+    return DSA_ERR_INVALID_ARG;
+  if (B == 0 || t_count == 0) return DSA_OK;
+  if (!scores || !idx || !cand_score || !cand_id) return DSA_ERR_INVALID_ARG;
+  return dsa::launch_gather_selected(scores, ld, idx, B, T, t_begin, t_count, k, id_offset, cand_score, cand_id,
+                                     static_cast<cudaStream_t>(stream));
+}
+
+int dsa_topk_merge(const float* cand_score, const int32_t* cand_id, int n_parts, int64_t part_stride, int kc,
+                   const int32_t* ctx_len, int B, int T, int S_total, int t_begin, int t_count, int k, int32_t* idx,
+                   void* stream) {
+  if (B < 0 || T < 1 || S_total < 1 || t_begin < 0 || t_count < 0 || t_begin + t_count > T || n_parts < 1 || kc < 1)
+    return DSA_ERR_INVALID_ARG;
+  if (k < 1 || k > 2048 || kc < k || (int64_t)n_parts * kc > dsa::kMergeMaxCand) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || t_count == 0) return DSA_OK;
+  if (part_stride < (int64_t)B * t_count * kc) return DSA_ERR_INVALID_ARG;
+  if (!cand_score || !cand_id || !ctx_len || !idx) return DSA_ERR_INVALID_ARG;
+  return dsa::launch_topk_merge(cand_score, cand_id, n_parts, part_stride, kc, ctx_len, B, T, S_total, t_begin,
+                                t_count, k, idx, static_cast<cudaStream_t>(stream));
+}
+
+int dsa_idx_localize(const int32_t* idx, int64_t n, int32_t s0, int32_t s_len, int32_t* out, void* stream) {
+  if (n < 0 || s0 < 0 || s_len < 0) return DSA_ERR_INVALID_ARG;
+  if (n == 0) return DSA_OK;
+  if (!idx || !out) return DSA_ERR_INVALID_ARG;
+  return dsa::launch_idx_localize(idx, n, s0, s_len, out, static_cast<cudaStream_t>(stream));
+}
+
+int dsa_attn_combine(const uint16_t* part_o, const float* part_lse, int n_parts, int64_t rows, int d_v, uint16_t* out,
+                     float* lse, void* stream) {
+  if (n_parts < 1 || n_parts > 16 || rows < 0 || d_v < 2 || (d_v & 1)) return DSA_ERR_INVALID_ARG;
+  if (rows == 0) return DSA_OK;
+  if (!part_o || !part_lse || !out) return DSA_ERR_INVALID_ARG;
+  if (!dsa::aligned16(part_o) || !dsa::aligned16(out)) return DSA_ERR_MISALIGNED;
+  return dsa::launch_attn_combine(part_o, true, part_lse, n_parts, rows, d_v, out, lse,
+                                  static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -76,9 +76,22 @@ int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, int64_t kv_rs, i
                          const int32_t* idx, int B, int T, int k, float sm_scale, uint16_t* out, float* lse,
                          void* ws, int splits, const PageMap& pm, cudaStream_t stream);
 unsigned int attn_tc_take_status();
-// Merges split-key attention partials (normalised fp32 O and log-sum-exp per split).
+// Merges split-key attention partials (normalised O, fp32 or bf16, and log-sum-exp per split).
 int launch_attn_combine(const void* part_o, bool bf16_parts, const float* part_lse, int splits, int64_t rows,
                         int d_v, uint16_t* out, float* lse, cudaStream_t stream);
+
+// Context parallelism: the exact top-k over the union of per-shard selections (n_parts lists of
+// kc (score, global id) per row, part p at part_stride elements from part 0).
+constexpr int kMergeMaxCand = 16384;   // n_parts * kc, the candidates a row's CTA holds
+int launch_topk_merge(const float* cand_score, const int32_t* cand_id, int n_parts, int64_t part_stride, int kc,
+                      const int32_t* ctx_len, int B, int T, int S_total, int t_begin, int t_count, int k, int32_t* idx,
+                      cudaStream_t stream);
+// The scores of a shard's selected keys and their global ids (local id + id_offset; -1 stays -1
+// with score -inf).
+int launch_gather_selected(const float* scores, int64_t ld, const int32_t* idx, int B, int T, int t_begin,
+                           int t_count, int k, int id_offset, float* cand_score, int32_t* cand_id, cudaStream_t stream);
+// Global key ids -> the ids within the shard [s0, s0 + s_len) (others -1).
+int launch_idx_localize(const int32_t* idx, int64_t n, int s0, int s_len, int32_t* out, cudaStream_t stream);
 
 // IndexPool over `pool` (2, 4 or 8) consecutive keys.
 int launch_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool, uint8_t* k_pool,

@@ -683,6 +683,63 @@ topk_select_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* 
   write_sorted<NT>(sel, k, n_valid, hist, tie, warp_buf, out, pool, pos);
 }
 
+// Merge of per-shard selections (context parallelism): row r of part p holds that shard's
+// selected keys as (score, global key id), ids ascending, -1 padding.  The exact top-k of the
+// union: every key a full sort over the whole row keeps is in its shard's selection (a shard
+// has at most k of them, and its own top-k keeps its lowest-indexed ties, which are the
+// lowest global ids), so the candidate selection over the union gives the same ids.
+__global__ void __launch_bounds__(TS_THREADS, 1)
+topk_merge_kernel(const float* __restrict__ cand_score, const int32_t* __restrict__ cand_id, int n_parts,
+                  int64_t part_stride, int kc, const int32_t* __restrict__ ctx_len, int T, int S_total, int t_begin,
+                  int t_count, int k, int32_t* __restrict__ idx_out) {
+  constexpr int NT = TS_THREADS;
+  __shared__ uint32_t hist[TK_BINS];
+  __shared__ int sel[TK_KMAX];
+  __shared__ int warp_buf[32];
+  __shared__ int piv[3];
+  __shared__ int counters[2];
+  __shared__ int sh_cnt;
+  extern __shared__ uint32_t cand_smem[];
+  const int cap = n_parts * kc;
+  uint32_t* ck = cand_smem;
+  int* ci = reinterpret_cast<int*>(cand_smem + cap);
+  int* tie = reinterpret_cast<int*>(cand_smem + 2 * cap);
+  const int tid = threadIdx.x;
+  const int row_id = blockIdx.x;
+  const int b = row_id / t_count;
+  const int t = t_begin + row_id % t_count;
+  const int pos = ctx_len[b] - T + t;
+  const int n_valid = pos < 0 ? 0 : min(S_total, pos + 1);
+  int32_t* out = idx_out + ((int64_t)b * T + t) * (int64_t)k;
+  if (n_valid <= k) {
+    for (int i = tid; i < k; i += NT) out[i] = i < n_valid ? i : -1;
+    return;
+  }
+  if (tid == 0) sh_cnt = 0;
+  __syncthreads();
+  for (int e0 = 0; e0 < cap; e0 += NT) {   // the same trip count in every lane of a warp
+    const int e = e0 + tid;
+    const int p = e / kc, j = e % kc;
+    int id = -1;
+    float f = 0.f;
+    if (e < cap) {
+      const int64_t at = (int64_t)p * part_stride + (int64_t)row_id * kc + j;
+      id = __ldg(cand_id + at);
+      f = __ldg(cand_score + at);
+    }
+    const int slot = warp_slot(&sh_cnt, id >= 0);
+    if (slot >= 0) {
+      ck[slot] = order_key(f);
+      ci[slot] = id;
+    }
+  }
+  __syncthreads();
+  const int ncand = sh_cnt;   // >= k: each shard kept min(k, its visible keys)
+  __syncthreads();
+  select_from_candidates<NT>(ck, ci, ncand, k, hist, sel, tie, warp_buf, piv, counters);
+  write_sorted<NT>(sel, k, n_valid, hist, tie, warp_buf, out, 1, pos);
+}
+
 __device__ __forceinline__ float from_order_key(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
@@ -868,6 +925,26 @@ int launch_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, 
     set_cuda_error(e);
     return DSA_ERR_CUDA;
   }
+  return check_launch();
+}
+
+int launch_topk_merge(const float* cand_score, const int32_t* cand_id, int n_parts, int64_t part_stride, int kc,
+                      const int32_t* ctx_len, int B, int T, int S_total, int t_begin, int t_count, int k, int32_t* idx,
+                      cudaStream_t stream) {
+  if (B * t_count == 0) return DSA_OK;
+  const int cap = n_parts * kc;
+  int cap2 = 1;
+  while (cap2 < cap) cap2 <<= 1;   // the tie list is sorted in a power-of-two buffer
+  const int smem = (2 * cap + cap2) * 4;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 3 * kMergeMaxCand * 4);
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  topk_merge_kernel<<<B * t_count, TS_THREADS, smem, stream>>>(cand_score, cand_id, n_parts, part_stride, kc, ctx_len,
+                                                               T, S_total, t_begin, t_count, k, idx);
   return check_launch();
 }
 
