@@ -316,7 +316,8 @@ int dsa_group_forward(const dsa_group_args* args, void* ws, size_t ws_bytes, voi
 /* Candidates of a shard's selection: for rows t_begin .. t_begin+t_count-1 of
  * idx [B, T, k] (ids local to the shard, from dsa_topk on scores [B, t_count, ld]),
  * cand_score/cand_id [B, t_count, k] = (scores[row][id], id + id_offset), or (-inf, -1) for a
- * -1 entry.  Supported: 1 <= k <= 2048. */
+ * -1 entry.  An id >= ld is skipped like a -1 (nothing past the score rows is read) and the
+ * next dsa_device_status() returns DSA_ERR_INDEX_RANGE.  Supported: 1 <= k <= 2048. */
 int dsa_gather_selected(const float* scores, int64_t ld, const int32_t* idx, int B, int T, int t_begin, int t_count,
                         int k, int32_t id_offset, float* cand_score, int32_t* cand_id, void* stream);
 
@@ -325,6 +326,9 @@ int dsa_gather_selected(const float* scores, int64_t ld, const int32_t* idx, int
  * [B, t_count, kc] as dsa_gather_selected writes them (kc >= k).  The rows are those of
  * queries t_begin .. of a context of ctx_len[b] keys (S_total key rows per sequence); a row with
  * at most k visible keys selects them all.  idx [B, T, k] int32 out (rows t_begin.. written).
+ * Candidate ids must be distinct within a row (disjoint shards).  An id >= the row's visible
+ * key count is skipped, a row left with fewer than k candidates is written as all -1, and
+ * either makes the next dsa_device_status() return DSA_ERR_INDEX_RANGE.
  * Supported: 1 <= k <= 2048, n_parts * kc <= 16384. */
 int dsa_topk_merge(const float* cand_score, const int32_t* cand_id, int n_parts, int64_t part_stride, int kc,
                    const int32_t* ctx_len, int B, int T, int S_total, int t_begin, int t_count, int k, int32_t* idx,

@@ -179,8 +179,10 @@ def launch_count() -> int:
 
 def dsa_device_status(stream=None) -> int:
     """Synchronises the stream and returns (and clears) the kernels' device status: 0, 6
-    (DSA_ERR_TIMEOUT) when a bounded device wait gave up, or 7 (DSA_ERR_INDEX_RANGE) when an
-    attention call met a selected id beyond its cache and skipped it."""
+    (DSA_ERR_TIMEOUT) when a bounded device wait gave up, or 7 (DSA_ERR_INDEX_RANGE) when a
+    call met an id beyond what it may read (attention: a selected id past its cache; the
+    context-parallel gather and merge: an id past the score row or the row's visible keys)
+    and skipped it."""
     return int(_lib().dsa_device_status(_stream(stream)))
 
 

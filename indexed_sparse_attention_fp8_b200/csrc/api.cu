@@ -263,7 +263,8 @@ int dsa_device_status(void* stream) {
     return DSA_ERR_CUDA;
   }
   const unsigned int st =
-      indexer_take_status() | attn_tc_take_status() | attn_mma_take_status() | pool_take_status();
+      indexer_take_status() | attn_tc_take_status() | attn_mma_take_status() | pool_take_status() |
+      cp_take_status() | merge_take_status();
   if (st & 1u) return DSA_ERR_TIMEOUT;
   if (st & 2u) return DSA_ERR_INDEX_RANGE;
   return DSA_OK;

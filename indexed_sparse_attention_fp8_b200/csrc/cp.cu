@@ -11,7 +11,11 @@
 namespace dsa {
 namespace {
 
-// One thread per selected slot: rows (b, t_begin + r) of the [B, T, k] id array.
+__device__ unsigned int g_cp_status;   // bit 1: an id at or beyond its score row's width
+
+// One thread per selected slot: rows (b, t_begin + r) of the [B, T, k] id array.  An id past
+// the score row's ld entries is skipped like a -1 and flagged, so nothing outside the score
+// rows is read.
 __global__ void gather_selected_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ idx,
                                        int T, int t_begin, int t_count, int k, int id_offset,
                                        float* __restrict__ cand_score, int32_t* __restrict__ cand_id, int64_t n) {
@@ -20,7 +24,11 @@ __global__ void gather_selected_kernel(const float* __restrict__ scores, int64_t
   const int64_t row = e / k;          // (b, r) over B * t_count rows
   const int j = (int)(e % k);
   const int64_t b = row / t_count, r = row % t_count;
-  const int id = __ldg(idx + (b * T + t_begin + r) * k + j);
+  int id = __ldg(idx + (b * T + t_begin + r) * k + j);
+  if (id >= ld) {
+    atomicOr(&g_cp_status, 2u);
+    id = -1;
+  }
   cand_id[e] = id < 0 ? -1 : id + id_offset;
   cand_score[e] = id < 0 ? -INFINITY : __ldg(scores + row * ld + id);
 }
@@ -42,6 +50,13 @@ int launch_gather_selected(const float* scores, int64_t ld, const int32_t* idx, 
   gather_selected_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(scores, ld, idx, T, t_begin, t_count, k,
                                                                           id_offset, cand_score, cand_id, n);
   return check_launch();
+}
+
+unsigned int cp_take_status() {
+  unsigned int v = 0, zero = 0;
+  cudaMemcpyFromSymbol(&v, g_cp_status, sizeof(v));
+  if (v) cudaMemcpyToSymbol(g_cp_status, &zero, sizeof(zero));
+  return v;
 }
 
 int launch_idx_localize(const int32_t* idx, int64_t n, int s0, int s_len, int32_t* out, cudaStream_t stream) {

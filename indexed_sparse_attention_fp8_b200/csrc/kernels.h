@@ -90,6 +90,8 @@ int launch_topk_merge(const float* cand_score, const int32_t* cand_id, int n_par
 // with score -inf).
 int launch_gather_selected(const float* scores, int64_t ld, const int32_t* idx, int B, int T, int t_begin,
                            int t_count, int k, int id_offset, float* cand_score, int32_t* cand_id, cudaStream_t stream);
+unsigned int cp_take_status();
+unsigned int merge_take_status();
 // Global key ids -> the ids within the shard [s0, s0 + s_len) (others -1).
 int launch_idx_localize(const int32_t* idx, int64_t n, int s0, int s_len, int32_t* out, cudaStream_t stream);
 

@@ -31,6 +31,8 @@
 namespace dsa {
 namespace {
 
+__device__ unsigned int g_merge_status;   // bit 1: a merge row whose candidates were out of range or too few
+
 constexpr int TK_THREADS = 1024;     // the fused selection's kernels
 constexpr int TK_KMAX = 2048;
 constexpr int TK_BINS = 2048;
@@ -726,6 +728,10 @@ topk_merge_kernel(const float* __restrict__ cand_score, const int32_t* __restric
       const int64_t at = (int64_t)p * part_stride + (int64_t)row_id * kc + j;
       id = __ldg(cand_id + at);
       f = __ldg(cand_score + at);
+      if (id >= n_valid) {   // not a key this row sees: skipped (the ordered write needs ids < n_valid)
+        atomicOr(&g_merge_status, 2u);
+        id = -1;
+      }
     }
     const int slot = warp_slot(&sh_cnt, id >= 0);
     if (slot >= 0) {
@@ -736,6 +742,11 @@ topk_merge_kernel(const float* __restrict__ cand_score, const int32_t* __restric
   __syncthreads();
   const int ncand = sh_cnt;   // >= k: each shard kept min(k, its visible keys)
   __syncthreads();
+  if (ncand < k) {   // only when the candidates are not shard selections of this row: no result
+    if (tid == 0) atomicOr(&g_merge_status, 2u);
+    for (int i = tid; i < k; i += NT) out[i] = -1;
+    return;
+  }
   select_from_candidates<NT>(ck, ci, ncand, k, hist, sel, tie, warp_buf, piv, counters);
   write_sorted<NT>(sel, k, n_valid, hist, tie, warp_buf, out, 1, pos);
 }
@@ -926,6 +937,13 @@ int launch_topk(const float* scores, int64_t ld, const int32_t* ctx_len, int B, 
     return DSA_ERR_CUDA;
   }
   return check_launch();
+}
+
+unsigned int merge_take_status() {
+  unsigned int v = 0, zero = 0;
+  cudaMemcpyFromSymbol(&v, g_merge_status, sizeof(v));
+  if (v) cudaMemcpyToSymbol(g_merge_status, &zero, sizeof(zero));
+  return v;
 }
 
 int launch_topk_merge(const float* cand_score, const int32_t* cand_id, int n_parts, int64_t part_stride, int kc,

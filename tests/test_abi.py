@@ -209,3 +209,32 @@ def test_group_workspace_and_validation(lib):
     assert need == (1048576 // 4) * 128 + _fused_row_bytes(1048576 // 4)   # pooled keys + one selection row
     odd, keep4 = _group_args(pool=4, topk=512, S=1048574, T=8192)
     assert lib.dsa_group_forward(ctypes.byref(odd), A, 1 << 40, None) == UNSUPPORTED
+
+
+def test_context_parallel_calls_validation(lib):
+    """The four calls around the key-sharded exchange reject bad sizes before any launch."""
+    g = lib.dsa_gather_selected   # scores, ld, idx, B, T, t_begin, t_count, k, id_offset, cs, ci, stream
+    assert g(A, 4096, A, 1, 8, 4, 8, 2048, 0, A, A, None) == INVALID      # rows past T
+    assert g(A, 4096, A, 1, 8, 0, 8, 4096, 0, A, A, None) == INVALID      # k > 2048
+    assert g(A, 4096, A, 1, 8, 0, 8, 2048, -1, A, A, None) == INVALID     # negative offset
+    assert g(None, 4096, A, 1, 8, 0, 8, 2048, 0, A, A, None) == INVALID
+    assert g(A, 4096, A, 1, 8, 0, 0, 2048, 0, A, A, None) == OK           # nothing to gather
+    m = lib.dsa_topk_merge   # cs, ci, n_parts, part_stride, kc, ctx, B, T, S, t_begin, t_count, k, idx, stream
+    stride = 8 * 2048
+    assert m(A, A, 2, stride, 2048, A, 1, 8, 9000, 0, 8, 4096, A, None) == UNSUPPORTED   # k > 2048
+    assert m(A, A, 2, stride, 1024, A, 1, 8, 9000, 0, 8, 2048, A, None) == UNSUPPORTED   # kc < k
+    assert m(A, A, 9, stride, 2048, A, 1, 8, 9000, 0, 8, 2048, A, None) == UNSUPPORTED   # 9 x 2048 > 16384
+    assert m(A, A, 2, stride - 1, 2048, A, 1, 8, 9000, 0, 8, 2048, A, None) == INVALID  # parts overlap
+    assert m(A, A, 0, stride, 2048, A, 1, 8, 9000, 0, 8, 2048, A, None) == INVALID
+    assert m(A, A, 2, stride, 2048, None, 1, 8, 9000, 0, 8, 2048, A, None) == INVALID
+    assert m(A, A, 2, stride, 2048, A, 1, 8, 9000, 0, 0, 2048, A, None) == OK           # no rows
+    loc = lib.dsa_idx_localize   # idx, n, s0, s_len, out, stream
+    assert loc(A, -1, 0, 10, A, None) == INVALID
+    assert loc(A, 10, -1, 10, A, None) == INVALID
+    assert loc(None, 10, 0, 10, A, None) == INVALID
+    assert loc(A, 0, 0, 10, A, None) == OK
+    c = lib.dsa_attn_combine   # part_o, part_lse, n_parts, rows, d_v, out, lse, stream
+    assert c(A, A, 17, 8, 512, A, None, None) == INVALID      # more than 16 parts
+    assert c(A, A, 2, 8, 511, A, None, None) == INVALID       # odd d_v
+    assert c(A + 2, A, 2, 8, 512, A, None, None) == MISALIGNED
+    assert c(A, A, 2, 0, 512, A, None, None) == OK            # no rows

@@ -108,3 +108,38 @@ def test_context_parallel_equals_one_gpu(name, over, ctx, world, t_chunk):
             msg = P.check_attn_row(P.bf16_np(o[b, t]), P.bf16_np(L["q"][b, t]), Kb, Kb[:, : wl.d_v], idx_h[b, t],
                                    wl.sm_scale, P.to_np(lse[b, t]).astype(np.float64))
             assert msg is None, f"layer {li} row {(b, t)}: {msg}"
+
+
+@pytest.mark.gpu
+def test_context_parallel_guards_skip_and_flag_bad_ids():
+    """Ids that the exchange steps may not read are skipped and reported, not read: a selected id
+    past the score row in the candidate gather; in the merge, a candidate id past the row's
+    visible keys, and a row left with fewer than k candidates (written as all -1)."""
+    import indexed_sparse_attention_fp8_b200 as dsa
+    dev = "cuda"
+    B, T, k, ld = 1, 2, 4, 64
+    scores = torch.arange(B * T * ld, dtype=torch.float32, device=dev).view(B, T, ld)
+    idx = torch.tensor([[[0, 5, 63, 64], [1, -1, 2, 10 ** 6]]], dtype=torch.int32, device=dev)
+    assert dsa.dsa_device_status() == 0
+    cs, ci = dsa.dsa_gather_selected(scores, idx, 0, 100)
+    assert dsa.dsa_device_status() == 7
+    assert ci.tolist() == [[[100, 105, 163, -1], [101, -1, 102, -1]]]
+    assert cs[0, 0, :3].tolist() == [0.0, 5.0, 63.0] and cs[0, 1, 0].item() == 65.0
+    assert torch.isinf(cs[0, 0, 3]) and torch.isinf(cs[0, 1, 3])
+    # merge: two parts of k candidates for one row at position 99 of a 100-key context
+    ctx = torch.tensor([100], dtype=torch.int32, device=dev)
+    sc = torch.tensor([[[[9.0, 8.0, 7.0, 6.0]]], [[[5.0, 4.0, 3.0, 2.0]]]], device=dev)
+    good = torch.tensor([[[[10, 20, 30, 40]]], [[[50, 60, 70, 80]]]], dtype=torch.int32, device=dev)
+    out = dsa.dsa_topk_merge(sc, good, ctx, 1, 100, k)
+    assert dsa.dsa_device_status() == 0
+    assert out.tolist() == [[[10, 20, 30, 40]]]
+    bad = good.clone()
+    bad[0, 0, 0, 1] = 100          # not a visible key (positions 0..99): skipped
+    out = dsa.dsa_topk_merge(sc, bad, ctx, 1, 100, k)
+    assert dsa.dsa_device_status() == 7
+    assert out.tolist() == [[[10, 30, 40, 50]]]
+    few = torch.full_like(good, -1)
+    few[0, 0, 0, :3] = torch.tensor([1, 2, 3], dtype=torch.int32)   # 3 < k candidates in all
+    out = dsa.dsa_topk_merge(sc, few, ctx, 1, 100, k)
+    assert dsa.dsa_device_status() == 7
+    assert out.tolist() == [[[-1, -1, -1, -1]]]
