@@ -179,12 +179,26 @@ def box_workload(wl, box):
 
 
 class Part:
-    """One box of the rank's share: its sub-workload, its input tensors and its group call."""
+    """One box of the rank's share: its sub-workload, its input tensors and its group call.
+    With IndexPool the pooled key cache is state kept beside the key cache, as a serving loop
+    keeps it: pooled once here, and each step refreshes only the blocks that hold the step's
+    T new rows (dsa_index_pool_tail) before the group call reads it."""
 
     def __init__(self, wl, box, ind, lays, dsa):
         self.wl, self.box, self.ind, self.lays = box_workload(wl, box), box, ind, lays
+        self.dsa = dsa
+        self.k_pool = dsa.dsa_index_pool(ind["k_idx"], pool=wl.pool) if wl.pool > 1 else None
         self.g = dsa.Group(ind["q_idx"], ind["w"], ind["k_idx"], ind["ctx_len"], wl.topk, lays, wl.sm_scale,
-                           wl.d_v, pool=wl.pool)
+                           wl.d_v, pool=wl.pool, k_pooled=self.k_pool)
+
+    def refresh_pool(self, stream):
+        if self.k_pool is not None:
+            self.dsa.dsa_index_pool_tail(self.ind["k_idx"], self.ind["ctx_len"], self.wl.T, self.k_pool,
+                                         pool=self.wl.pool, stream=stream)
+
+    def step(self, ws, stream):
+        self.refresh_pool(stream)
+        self.g.forward(ws, stream)
 
 
 def make_parts(wl, dev, dsa, boxes):
@@ -265,7 +279,7 @@ def run_ours(args, rank, world, dev):
 
     def step():
         for p in parts:
-            p.g.forward(ws, stream)
+            p.step(ws, stream)
 
     for _ in range(args.warmup):
         step()
@@ -309,10 +323,11 @@ def run_ours(args, rank, world, dev):
 
 def breakdown(parts, ws, t_chunk, stream, dsa, reps, fused=True):
     """Average device time of each step of the group per step over `reps` steps, CUDA events on
-    `stream` (the launches queued ahead of the GPU), summed over this rank's parts: the pool kernel, the selection as the group call
-    runs it (the indexer writing full score rows, then the row top-k, per query chunk), and each
-    attention layer; with `fused`, also the fused selection (dsa_index_select) over the same
-    chunks, for comparison."""
+    `stream` (the launches queued ahead of the GPU), summed over this rank's parts: the refresh
+    of the pooled key cache (IndexPool), the selection as the group call runs it (the indexer
+    writing full score rows, then the row top-k, per query chunk), and each attention layer;
+    with `fused`, also the fused selection (dsa_index_select) over the same chunks, for
+    comparison."""
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     tot = {"pool": 0.0, "indexer": 0.0, "topk": 0.0, "attn": 0.0, "fused_select": 0.0}
     n = {k: 0 for k in tot}
@@ -339,9 +354,10 @@ def breakdown(parts, ws, t_chunk, stream, dsa, reps, fused=True):
             if wl.pool > 1:
                 a, b = ev(), ev()
                 a.record(stream)
-                keys = dsa.dsa_index_pool(ind["k_idx"], pool=wl.pool, stream=stream)
+                p.refresh_pool(stream)
                 b.record(stream)
                 marks.append(("pool", a, b))
+                keys = p.k_pool
             for t0 in range(0, wl.T, t_chunk):
                 tc = min(t_chunk, wl.T - t0)
                 sc = sc_buf[: wl.B * tc * ld].view(wl.B, tc, ld)   # [B, tc, ld], batch stride tc * ld
@@ -389,7 +405,7 @@ def breakdown(parts, ws, t_chunk, stream, dsa, reps, fused=True):
 # the score rows, 4 B per pair written and read back).  A launch's traffic is the figure times
 # the units it processes.  Only kernels unchanged since that capture are listed (others report
 # None), and other contexts were not measured.
-TRAFFIC_PER_UNIT = {("prefill128k", "attn"): ("query", 606.1e3), ("prefill128k", "indexer"): ("pair", 3.916),
+TRAFFIC_PER_UNIT = {("prefill128k", "attn"): ("query", 603.7e3), ("prefill128k", "indexer"): ("pair", 3.922),
                     ("prefill128k", "topk"): ("pair", 4.285)}
 
 
@@ -560,7 +576,7 @@ def run_secondary(args, name, dev, steps=3, per_layer=False):
         g = parts[0].g
         t_chunk = max(1, min(wl.T, (args.score_ws_gb << 30) // (wl.B * ((wl.S // wl.pool + 3) // 4 * 4) * 4)))
         ws = torch.empty(g.workspace_size(t_chunk), dtype=torch.uint8, device=dev)
-        fn = lambda: g.forward(ws, stream)  # noqa: E731
+        fn = lambda: parts[0].step(ws, stream)  # noqa: E731
         for _ in range(max(3, args.warmup)):
             fn()
         ms = time_region(fn, steps, stream) / steps

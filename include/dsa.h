@@ -251,6 +251,22 @@ int dsa_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool, ui
                    const dsa_paging* paging, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * dsa_index_pool_tail - keeps a pooled key cache current as keys are appended (decode, chunked
+ * prefill): for every sequence b it recomputes, exactly as dsa_index_pool does, the pooled
+ * blocks that hold rows ctx_len[b]-T .. ctx_len[b]-1 (the keys this step appended; rows
+ * outside [0, S_max) are ignored) and touches no other block.  So dsa_index_pool once, then
+ * this call after every append, leaves k_pool equal to dsa_index_pool of the current cache at
+ * the cost of the new rows alone.  A block the append leaves partly filled is pooled over the
+ * rows the cache holds at that moment, as dsa_index_pool would pool it.  The method pools
+ * blocks of consecutive keys and says nothing of how a serving system keeps them; this is the
+ * plain incremental form of the same arithmetic.
+ *   ctx_len device [B] int32 (after the append); T >= 1 rows appended per sequence.
+ * Other arguments, layouts and support as for dsa_index_pool.
+ * ------------------------------------------------------------------------------------ */
+int dsa_index_pool_tail(const uint8_t* k_idx, const int32_t* ctx_len, int B, int T, int S_max, int d_I, int pool,
+                        uint8_t* k_pool, const dsa_paging* paging, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * dsa_group_forward - one IndexShare group ("IndexShare: Amortizing the Indexer"): the
  * indexer and the top-k run ONCE, and each of the group_size attention layers reads the
  * same index buffer.  Equivalent to dsa_index_scores + dsa_topk over all queries (in query
@@ -286,6 +302,10 @@ typedef struct dsa_group_args {
   int32_t fused_select;    /* 0 (default): full score rows + dsa_topk, the faster path on B200
                               (the indexer is tensor-bound, so its score rows cost little);
                               1: fused selection where the keys allow it (dsa_index_select) */
+  const uint8_t* k_pooled; /* pool > 1 only.  NULL: the call pools k_idx into its workspace;
+                              else the caller's pooled cache [B, S_max/pool, d_I] e4m3
+                              (contiguous; dsa_index_pool, then dsa_index_pool_tail after each
+                              append), which the indexer reads as is and no pooling runs */
 } dsa_group_args;
 
 /* Workspace for dsa_group_forward when the indexer is run over chunks of t_chunk queries

@@ -65,7 +65,7 @@ class GroupArgs(ctypes.Structure):
         ("kv_row_stride", _c_i64), ("kv_batch_stride", _c_i64), ("v_row_stride", _c_i64),
         ("v_batch_stride", _c_i64),
         ("Hq", ctypes.c_int32), ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32), ("sm_scale", _c_f),
-        ("idx", _c_p), ("paging", Paging), ("fused_select", ctypes.c_int32),
+        ("idx", _c_p), ("paging", Paging), ("fused_select", ctypes.c_int32), ("k_pooled", _c_p),
     ]
 
 
@@ -90,6 +90,8 @@ _SIGS = {
                                  _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p, _c_p, _c_sz, ctypes.POINTER(Paging),
                                  _c_p]),
     "dsa_index_pool": (_c_int, [_c_p, _c_int, _c_int, _c_int, _c_int, _c_p, ctypes.POINTER(Paging), _c_p]),
+    "dsa_index_pool_tail": (_c_int, [_c_p, _c_p, _c_int, _c_int, _c_int, _c_int, _c_int, _c_p, ctypes.POINTER(Paging),
+                                     _c_p]),
     "dsa_noalloc_scratch_bytes": (_c_sz, []),
     "dsa_sparse_attn_noalloc": (_c_int, [_c_p, _c_p, _c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_p, _c_int,
                                          _c_int, _c_int, _c_int, _c_int, _c_int, _c_f, _c_p, _c_p,
@@ -367,12 +369,33 @@ def dsa_index_pool(k_idx: torch.Tensor, pool: int = 4, k_pool: Optional[torch.Te
     return k_pool
 
 
+def dsa_index_pool_tail(k_idx: torch.Tensor, ctx_len: torch.Tensor, T: int, k_pool: torch.Tensor, pool: int = 4,
+                        paging: Optional[Paging] = None, B: Optional[int] = None, stream=None) -> torch.Tensor:
+    """Refresh of a pooled key cache after T keys were appended to every sequence (ctx_len
+    [B] int32 after the append): the pooled blocks holding the new rows are recomputed in
+    k_pool [B, S/pool, d_I], the rest untouched."""
+    if paging is None:
+        B, S, D = k_idx.shape
+        _layout("k_idx", k_idx, torch.uint8, (B, S, D))
+    else:
+        D = k_idx.shape[2]
+        S = paging.pages_per_seq * paging.page_size
+        B = int(B if B is not None else paging._table.shape[0])
+        _layout("k_idx", k_idx, torch.uint8, (paging.num_pages, paging.page_size, D))
+    _layout("ctx_len", ctx_len, torch.int32, (B,))
+    _layout("k_pool", k_pool, torch.uint8, (B, S // pool, D))
+    _check("dsa_index_pool_tail", _lib().dsa_index_pool_tail(_ptr(k_idx), _ptr(ctx_len), B, int(T), S, D, pool,
+                                                             _ptr(k_pool), _paging_ref(paging), _stream(stream)))
+    return k_pool
+
+
 class Group:
     """Marshalled arguments of one IndexShare group (keeps the pointer arrays alive)."""
 
     def __init__(self, q_idx, w, k_idx, ctx_len, topk: int, layers: Sequence[dict], sm_scale: float,
                  d_v: int, pool: int = 1, idx: Optional[torch.Tensor] = None, want_lse: bool = False,
-                 paging: Optional[Paging] = None, fused_select: bool = False):
+                 paging: Optional[Paging] = None, fused_select: bool = False,
+                 k_pooled: Optional[torch.Tensor] = None):
         B, T, H, D = q_idx.shape
         S = k_idx.shape[1] if paging is None else paging.pages_per_seq * paging.page_size
         L = len(layers)
@@ -388,6 +411,10 @@ class Group:
             _layout("block_table", paging._table, torch.int32, (B, -1))
         _layout("ctx_len", ctx_len, torch.int32, (B,))
         _layout("idx", idx, torch.int32, (B, T, topk * pool))
+        if k_pooled is not None:
+            if pool == 1:
+                raise ValueError("k_pooled needs pool > 1")
+            _layout("k_pooled", k_pooled, torch.uint8, (B, S // pool, D))
         v0 = layers[0].get("v")
         for l, lay in enumerate(self.layers):
             # one set of K/V strides describes every layer's caches
@@ -421,8 +448,10 @@ class Group:
             v_row_stride=v_any.stride(1) if v_any is not None else 0,
             v_batch_stride=v_any.stride(0) if v_any is not None else 0,
             Hq=Hq, d_qk=Dqk, d_v=d_v, sm_scale=float(sm_scale), idx=_ptr(self.idx),
-            paging=paging if paging is not None else Paging(), fused_select=1 if fused_select else 0)
+            paging=paging if paging is not None else Paging(), fused_select=1 if fused_select else 0,
+            k_pooled=_ptr(k_pooled))
         self._paging = paging
+        self._k_pooled = k_pooled
         self.device = q0.device
 
     def workspace_size(self, t_chunk: int) -> int:
@@ -437,12 +466,14 @@ class Group:
 def dsa_group_forward(q_idx, w, k_idx, ctx_len, topk: int, layers: Sequence[dict], sm_scale: float, d_v: int,
                       pool: int = 1, t_chunk: Optional[int] = None, ws: Optional[torch.Tensor] = None,
                       want_lse: bool = False, paging: Optional[Paging] = None, fused_select: bool = False,
-                      stream=None):
+                      k_pooled: Optional[torch.Tensor] = None, stream=None):
     """One IndexShare group: indexer + top-k once, then attention for each layer dict
     {"q", "kv", optional "v", "out", "lse"}; with `paging`, k_idx and every layer's kv (and v)
-    are page pools sharing its block table.  Returns (idx, [(out, lse) per layer])."""
+    are page pools sharing its block table; with pool > 1 and `k_pooled`, the indexer reads
+    that pooled cache (kept current by dsa_index_pool_tail) instead of pooling k_idx.
+    Returns (idx, [(out, lse) per layer])."""
     g = Group(q_idx, w, k_idx, ctx_len, topk, layers, sm_scale, d_v, pool, want_lse=want_lse, paging=paging,
-              fused_select=fused_select)
+              fused_select=fused_select, k_pooled=k_pooled)
     if ws is None:
         ws = torch.empty(g.workspace_size(t_chunk or q_idx.shape[1]), dtype=torch.uint8, device=g.device)
     return g.forward(ws, stream)

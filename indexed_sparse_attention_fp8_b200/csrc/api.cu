@@ -199,7 +199,7 @@ struct GroupWs {
 GroupWs group_ws(const dsa_group_args* a) {
   GroupWs g;
   g.S_eff = a->pool > 1 ? a->S_max / a->pool : a->S_max;
-  g.pool_bytes = a->pool > 1 ? round_up((size_t)a->B * g.S_eff * a->d_I, 256) : 0;
+  g.pool_bytes = a->pool > 1 && !a->k_pooled ? round_up((size_t)a->B * g.S_eff * a->d_I, 256) : 0;
   g.attn_bytes = round_up(attn_workspace_bytes(a->B, a->T, a->Hq, a->d_v, a->topk * a->pool), 256);
   g.fixed_bytes = g.pool_bytes + g.attn_bytes;
   const PageMap key_pm = a->pool > 1 ? PageMap{nullptr, 0, 0, 0} : page_map(&a->paging);
@@ -215,6 +215,8 @@ int check_group(const dsa_group_args* a) {
   if (a->pool > 1 && (a->S_max % a->pool)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (a->topk < 1 || a->topk > 2048) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (a->topk * a->pool > 8192) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (a->k_pooled && a->pool == 1) return DSA_ERR_INVALID_ARG;
+  if (a->k_pooled && !aligned16(a->k_pooled)) return DSA_ERR_MISALIGNED;
   const int S_eff = a->pool > 1 ? a->S_max / a->pool : a->S_max;
   const int64_t ld = (int64_t)round_up((size_t)S_eff, 4);
   int st = check_index_scores(a->q_idx, a->w, a->k_idx, a->ctx_len, a->B, a->T, S_eff, a->H_I,
@@ -337,6 +339,18 @@ int dsa_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool, ui
   return launch_index_pool(k_idx, B, S_max, d_I, pool, k_pool, page_map(paging), static_cast<cudaStream_t>(stream));
 }
 
+int dsa_index_pool_tail(const uint8_t* k_idx, const int32_t* ctx_len, int B, int T, int S_max, int d_I, int pool,
+                        uint8_t* k_pool, const dsa_paging* paging, void* stream) {
+  if (B < 0 || T < 1 || S_max < 0 || d_I <= 0) return DSA_ERR_INVALID_ARG;
+  if (pool == 1 || !pool_ok(pool) || (S_max % pool) || (d_I % 16)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (const int st = check_paging(paging, S_max)) return st;
+  if (B == 0 || S_max == 0) return DSA_OK;
+  if (!k_idx || !ctx_len || !k_pool) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(k_idx) || !aligned16(k_pool)) return DSA_ERR_MISALIGNED;
+  return launch_index_pool_tail(k_idx, ctx_len, B, T, S_max, d_I, pool, k_pool, page_map(paging),
+                                static_cast<cudaStream_t>(stream));
+}
+
 size_t dsa_group_workspace_size(const dsa_group_args* a, int t_chunk) {
   if (!a || t_chunk < 1) return 0;
   const GroupWs g = group_ws(a);
@@ -393,9 +407,13 @@ int dsa_group_forward(const dsa_group_args* a, void* ws, size_t ws_bytes, void* 
   const uint8_t* keys = a->k_idx;
   PageMap key_pm = pm;   // the indexer reads the paged keys, or the (contiguous) pooled ones
   if (a->pool > 1) {
-    st = launch_index_pool(a->k_idx, a->B, a->S_max, a->d_I, a->pool, k_pool, pm, s);
-    if (st != DSA_OK) return st;
-    keys = k_pool;
+    if (a->k_pooled) {   // the caller keeps the pooled cache current (dsa_index_pool_tail)
+      keys = a->k_pooled;
+    } else {
+      st = launch_index_pool(a->k_idx, a->B, a->S_max, a->d_I, a->pool, k_pool, pm, s);
+      if (st != DSA_OK) return st;
+      keys = k_pool;
+    }
     key_pm = PageMap{nullptr, 0, 0, 0};
   }
   // IndexShare: one indexer + one top-k over every query, in chunks that fit the workspace

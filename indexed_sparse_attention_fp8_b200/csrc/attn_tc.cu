@@ -425,9 +425,11 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
 
   if (warp >= 4 && warp < MMA_WARP) {
     // ------------------------------------------------------------ gather (cp.async)
-    // Warp gw copies rows gw, gw+3, ..: lane l moves 16-byte chunks l, l+32 of its column
-    // range, so each row is read with coalesced requests.  A tile's ids come from one
-    // coalesced load per warp, issued a tile ahead, and reach the rows through shuffles.
+    // Warp gw copies the first 32 16-byte chunks of rows gw, gw+3, .. (lane l chunk l, one
+    // coalesced request per row), and the remaining 4 (CTA 0) or 8 (CTA 1) chunks of groups of
+    // 8 or 4 rows in one request per group, so every request has all 32 lanes busy.  A tile's
+    // ids come from one coalesced load per warp, issued a tile ahead, and reach the rows
+    // through shuffles.
     const int gw = warp - 4;
     bool ok = true;
     uint32_t g = 0;   // tiles gathered so far
@@ -485,15 +487,23 @@ sparse_mla_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         const int key = __shfl_sync(0xffffffffu, r < 32 ? id0 : id1, r & 31);
         const int crow = __shfl_sync(0xffffffffu, r < 32 ? row0 : row1, r & 31);
         const __nv_bfloat16* src = kvb + (int64_t)(key < 0 ? 0 : crow) * kv_rs;
-        const int nbytes = key < 0 ? 0 : 16;
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = ch_lo + lane + 32 * cc;
-          if (c < ch_hi) {
-            const uint32_t dst = stage + ((c >> 3) - blk0) * K_BLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-            cp_async16(dst, src + c * 8, nbytes);
-          }
-        }
+        const int c = ch_lo + lane;
+        const uint32_t dst = stage + ((c >> 3) - blk0) * K_BLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+        cp_async16(dst, src + c * 8, key < 0 ? 0 : 16);
+      }
+      // the last rc = 4 (CTA 0) or 8 (CTA 1) chunks of 32/rc rows at a time: lane l takes row
+      // r0 + l/rc, chunk ch_lo + 32 + l%rc
+      const int rc_sh = half == 0 ? 2 : 3;
+      const int rpg = 32 >> rc_sh;
+      for (int grp = gw; grp < NK / rpg; grp += 3) {
+        const int r0 = grp * rpg;
+        const int r = r0 + (lane >> rc_sh);
+        const int key = __shfl_sync(0xffffffffu, r0 < 32 ? id0 : id1, (r0 & 31) + (lane >> rc_sh));
+        const int crow = __shfl_sync(0xffffffffu, r0 < 32 ? row0 : row1, (r0 & 31) + (lane >> rc_sh));
+        const __nv_bfloat16* src = kvb + (int64_t)(key < 0 ? 0 : crow) * kv_rs;
+        const int c = ch_lo + 32 + (lane & ((1 << rc_sh) - 1));
+        const uint32_t dst = stage + ((c >> 3) - blk0) * K_BLK + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+        cp_async16(dst, src + c * 8, key < 0 ? 0 : 16);
       }
       asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(kv_full(st)) : "memory");
     }

@@ -98,5 +98,7 @@ int launch_idx_localize(const int32_t* idx, int64_t n, int s0, int s_len, int32_
 // IndexPool over `pool` (2, 4 or 8) consecutive keys.
 int launch_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool, uint8_t* k_pool,
                       const PageMap& pm, cudaStream_t stream);
+int launch_index_pool_tail(const uint8_t* k_idx, const int32_t* ctx_len, int B, int T, int S_max, int d_I, int pool,
+                           uint8_t* k_pool, const PageMap& pm, cudaStream_t stream);
 
 }  // namespace dsa

@@ -23,14 +23,11 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two) {
   return __half22float2(*reinterpret_cast<const __half2*>(&h));   // e4m3 -> f16 is exact
 }
 
+// Pools group g (global over the B sequences: groups_per_seq per sequence) at 16-byte slice
+// sl: the P source rows' slices are read, and the pooled slice is written to k_pool.
 template <int P>
-__global__ void __launch_bounds__(256)
-index_pool_kernel(const uint4* __restrict__ k_idx, int64_t n_groups, int groups_per_seq, int slices,
-                  uint4* __restrict__ k_pool, PageMap pm) {
-  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (gid >= n_groups * slices) return;
-  const int64_t g = gid / slices;
-  const int sl = (int)(gid % slices);
+__device__ __forceinline__ void pool_group(const uint4* __restrict__ k_idx, int64_t g, int groups_per_seq, int slices,
+                                           int sl, uint4* __restrict__ k_pool, const PageMap& pm) {
   // first source row of the group: contiguous, or in the page of its sequence that holds it
   // (a page holds whole groups: its size is a multiple of P); a bad page id reads as zeros
   int64_t row0 = P * g;
@@ -73,7 +70,37 @@ index_pool_kernel(const uint4* __restrict__ k_idx, int64_t n_groups, int groups_
     }
     outw[wd] = packed;
   }
-  k_pool[gid] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+  k_pool[g * slices + sl] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+}
+
+// Every group of every sequence: one thread per (group, slice).
+template <int P>
+__global__ void __launch_bounds__(256)
+index_pool_kernel(const uint4* __restrict__ k_idx, int64_t n_groups, int groups_per_seq, int slices,
+                  uint4* __restrict__ k_pool, PageMap pm) {
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= n_groups * slices) return;
+  pool_group<P>(k_idx, gid / slices, groups_per_seq, slices, (int)(gid % slices), k_pool, pm);
+}
+
+// The groups holding rows ctx_len[b]-T .. ctx_len[b]-1 of each sequence b (at most `window`
+// groups per sequence; rows outside [0, S_max) ignored): one thread per (b, group, slice).
+template <int P>
+__global__ void __launch_bounds__(256)
+index_pool_tail_kernel(const uint4* __restrict__ k_idx, const int32_t* __restrict__ ctx_len, int B, int T,
+                       int groups_per_seq, int window, int slices, uint4* __restrict__ k_pool, PageMap pm) {
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (int64_t)B * window * slices) return;
+  const int sl = (int)(gid % slices);
+  const int j = (int)((gid / slices) % window);
+  const int b = (int)(gid / ((int64_t)slices * window));
+  const int S_max = groups_per_seq * P;
+  const int hi = min(__ldg(ctx_len + b), S_max);   // rows [lo, hi) were appended
+  const int lo = max(hi - T, 0);
+  if (hi <= lo) return;
+  const int g = lo / P + j;
+  if (g > (hi - 1) / P) return;
+  pool_group<P>(k_idx, (int64_t)b * groups_per_seq + g, groups_per_seq, slices, sl, k_pool, pm);
 }
 
 }  // namespace
@@ -92,6 +119,25 @@ int launch_index_pool(const uint8_t* k_idx, int B, int S_max, int d_I, int pool,
     case 2: index_pool_kernel<2><<<(unsigned)blocks, threads, 0, stream>>>(src, n_groups, S_max / 2, slices, dst, pm); break;
     case 4: index_pool_kernel<4><<<(unsigned)blocks, threads, 0, stream>>>(src, n_groups, S_max / 4, slices, dst, pm); break;
     case 8: index_pool_kernel<8><<<(unsigned)blocks, threads, 0, stream>>>(src, n_groups, S_max / 8, slices, dst, pm); break;
+    default: return DSA_ERR_UNSUPPORTED_SHAPE;
+  }
+  return check_launch();
+}
+
+int launch_index_pool_tail(const uint8_t* k_idx, const int32_t* ctx_len, int B, int T, int S_max, int d_I, int pool,
+                           uint8_t* k_pool, const PageMap& pm, cudaStream_t stream) {
+  const int slices = d_I / 16;
+  const int window = (T - 1) / pool + 2;   // groups a run of T rows can touch
+  const int64_t n = (int64_t)B * window * slices;
+  if (n == 0) return DSA_OK;
+  const int threads = 256;
+  const int64_t blocks = (n + threads - 1) / threads;
+  const uint4* src = reinterpret_cast<const uint4*>(k_idx);
+  uint4* dst = reinterpret_cast<uint4*>(k_pool);
+  switch (pool) {
+    case 2: index_pool_tail_kernel<2><<<(unsigned)blocks, threads, 0, stream>>>(src, ctx_len, B, T, S_max / 2, window, slices, dst, pm); break;
+    case 4: index_pool_tail_kernel<4><<<(unsigned)blocks, threads, 0, stream>>>(src, ctx_len, B, T, S_max / 4, window, slices, dst, pm); break;
+    case 8: index_pool_tail_kernel<8><<<(unsigned)blocks, threads, 0, stream>>>(src, ctx_len, B, T, S_max / 8, window, slices, dst, pm); break;
     default: return DSA_ERR_UNSUPPORTED_SHAPE;
   }
   return check_launch();

@@ -209,6 +209,24 @@ def test_group_workspace_and_validation(lib):
     assert need == (1048576 // 4) * 128 + _fused_row_bytes(1048576 // 4)   # pooled keys + one selection row
     odd, keep4 = _group_args(pool=4, topk=512, S=1048574, T=8192)
     assert lib.dsa_group_forward(ctypes.byref(odd), A, 1 << 40, None) == UNSUPPORTED
+    # a caller-kept pooled cache: no pooled keys in the workspace; only with pool > 1, aligned
+    pool_args.fused_select = 0
+    pool_args.k_pooled = A
+    assert lib.dsa_group_workspace_size(ctypes.byref(pool_args), 1) == (1048576 // 4) * 4
+    pool_args.k_pooled = A + 8
+    assert lib.dsa_group_forward(ctypes.byref(pool_args), A, 1 << 40, None) == MISALIGNED
+    args.k_pooled = A
+    assert lib.dsa_group_forward(ctypes.byref(args), A, 1 << 40, None) == INVALID
+
+
+def test_index_pool_tail_validation(lib):
+    f = lib.dsa_index_pool_tail   # k_idx, ctx_len, B, T, S_max, d_I, pool, k_pool, paging, stream
+    assert f(A, A, 1, 1, 16, 128, 3, A, None, None) == UNSUPPORTED     # pool factors are 2, 4 and 8
+    assert f(A, A, 1, 1, 10, 128, 4, A, None, None) == UNSUPPORTED     # S not a multiple of 4
+    assert f(A, A, 1, 0, 16, 128, 4, A, None, None) == INVALID         # nothing appended
+    assert f(A, None, 1, 1, 16, 128, 4, A, None, None) == INVALID
+    assert f(A, A, 1, 1, 16, 128, 4, A + 4, None, None) == MISALIGNED
+    assert f(A, A, 0, 1, 16, 128, 4, A, None, None) == OK              # no sequences
 
 
 def test_context_parallel_calls_validation(lib):

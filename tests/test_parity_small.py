@@ -349,6 +349,52 @@ def test_indexpool_factors_2_and_8(factor, topk):
     _check_rows(wl, ind, lays, idx, outs, [(0, t) for t in (0, 1, factor - 1, factor, 100, 255, 256, 511)])
 
 
+@pytest.mark.parametrize("factor", [2, 4, 8])
+def test_pooled_cache_tail_refresh_equals_full_pool(factor):
+    """A pooled cache kept by dsa_index_pool_tail: after keys are appended (ragged contexts, one
+    and several new rows, blocks left partly filled and then completed), the refreshed cache is
+    the full pool of the current keys bit for bit, and the oracle's; blocks away from the new
+    rows are not written."""
+    g = torch.Generator(device="cpu").manual_seed(23 + factor)
+    B, S, D = 3, 4096, 128
+    codes = torch.randint(0, 254, (B, S, D), generator=g, dtype=torch.int32)
+    k = torch.where(codes >= 0x7F, codes + 1, codes).to(torch.uint8).to(DEV)
+    ctx = torch.tensor([1000, 2049, 37], dtype=torch.int32, device=DEV)
+    kp = dsa.dsa_index_pool(k, pool=factor)
+    for T in (1, 1, 3, factor, 5 * factor + 1, 1):
+        ctx += T
+        for b in range(B):   # the append: new rows ctx-T .. ctx-1
+            c = int(ctx[b])
+            k[b, c - T:c] = torch.randint(0, 127, (T, D), generator=g, dtype=torch.int32).to(torch.uint8).to(DEV)
+        before = kp.clone()
+        dsa.dsa_index_pool_tail(k, ctx, T, kp, pool=factor)
+        full = dsa.dsa_index_pool(k, pool=factor)
+        assert torch.equal(kp, full)
+        for b in range(B):   # untouched outside the new rows' blocks
+            c = int(ctx[b])
+            lo, hi = (c - T) // factor, (c - 1) // factor + 1
+            assert torch.equal(kp[b, :lo], before[b, :lo]) and torch.equal(kp[b, hi:], before[b, hi:])
+    assert dsa.dsa_device_status() == 0
+    assert np.array_equal(P.to_np(kp), O.index_pool(P.to_np(k), pool=factor))
+
+
+def test_group_with_kept_pooled_cache_equals_pooling_in_the_call():
+    """The group call reading a caller-kept pooled cache gives the ids and outputs of the call
+    that pools the keys itself, bit for bit (decode shape, ragged contexts)."""
+    wl = W.WORKLOADS["decode256k_pool"].replace(B=3, ctx=9000)
+    ind, lays = _inputs(wl, layers=2)
+    ctx = torch.tensor([9000, 4097, 2051], dtype=torch.int32, device=DEV)
+    layers = lambda: [{"q": L["q"], "kv": L["kv"], "v": L["v"]} for L in lays]   # noqa: E731
+    idx0, outs0 = dsa.dsa_group_forward(ind["q_idx"], ind["w"], ind["k_idx"], ctx, wl.topk, layers(), wl.sm_scale,
+                                        wl.d_v, pool=wl.pool, want_lse=True)
+    kp = dsa.dsa_index_pool(ind["k_idx"], pool=wl.pool)
+    idx1, outs1 = dsa.dsa_group_forward(ind["q_idx"], ind["w"], ind["k_idx"], ctx, wl.topk, layers(), wl.sm_scale,
+                                        wl.d_v, pool=wl.pool, want_lse=True, k_pooled=kp)
+    assert torch.equal(idx0, idx1)
+    for (o0, l0), (o1, l1) in zip(outs0, outs1):
+        assert torch.equal(o0, o1) and torch.equal(l0, l1)
+
+
 def test_pooled_decode_small():
     """The decode-shaped pooled path (one query per sequence, QB=1 indexer over pooled keys,
     top-512 blocks, split-key MLA attention), at a cache size the oracle checks in seconds."""
