@@ -68,7 +68,7 @@ struct Cfg {
   static constexpr int NWARPS = NWH * NWV;
   static constexpr int THREADS = NWARPS * 32;
   static constexpr int DVW = D_V / NWV;
-  static constexpr int STAGES = 3;
+  static constexpr int STAGES = 2;   // double-buffered: the smaller footprint fits six CTAs per SM (three stages: four), which pays more than the deeper ring
   static constexpr int QCH = D_QK / 8;  // 16-byte chunks per q/K row
   static constexpr int VCH = D_V / 8;
   static constexpr int Q_BYTES = HG * D_QK * 2;
@@ -129,23 +129,56 @@ sparse_attn_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16*
     const int r = i / C::QCH, c = i % C::QCH;
     cp_async16(sbase + swz(r, c, C::QCH), qrow + (int64_t)r * D_QK + c * 8, 16);
   }
+  // A tile's selected ids are all loaded (and their page rows looked up) before the first of
+  // its row copies is issued: each copy is an asm statement the compiler keeps in order with
+  // the loads around it, so loading each id right before its copy would put one memory round
+  // trip per row into every tile.
+  constexpr int NK_IT = (C::KT * C::QCH + C::THREADS - 1) / C::THREADS;
+  constexpr int NV_IT = LATENT ? 1 : (C::KT * C::VCH + C::THREADS - 1) / C::THREADS;
   auto load_tile = [&](int tile, int stage) {
     const int p0 = kbeg + tile * C::KT;
-    for (int i = tid; i < C::KT * C::QCH; i += C::THREADS) {
-      const int r = i / C::QCH, c = i % C::QCH;
-      const int p = p0 + r;
-      const int key = cache_row(p < kend ? checked_id(__ldg(irow + p), S_kv) : -1);
-      const __nv_bfloat16* src = kvb + (int64_t)(key < 0 ? 0 : key) * kv_rs + c * 8;
-      cp_async16(sbase + C::OFF_K + stage * C::K_TILE + swz(r, c, C::QCH), src, key < 0 ? 0 : 16);
-      if (c == 0) idx_s[stage * C::KT + r] = key;
+    int krow[NK_IT], vrow[NV_IT];
+#pragma unroll
+    for (int u = 0; u < NK_IT; ++u) {
+      const int i = tid + u * C::THREADS;
+      const int p = p0 + i / C::QCH;
+      krow[u] = (i < C::KT * C::QCH && p < kend) ? __ldg(irow + p) : -1;
     }
     if constexpr (!LATENT) {
-      for (int i = tid; i < C::KT * C::VCH; i += C::THREADS) {
-        const int r = i / C::VCH, c = i % C::VCH;
-        const int p = p0 + r;
-        const int key = cache_row(p < kend ? checked_id(__ldg(irow + p), S_kv) : -1);
-        const __nv_bfloat16* src = vb + (int64_t)(key < 0 ? 0 : key) * v_rs + c * 8;
-        cp_async16(sbase + C::OFF_V + stage * C::V_TILE + swz(r, c, C::VCH), src, key < 0 ? 0 : 16);
+#pragma unroll
+      for (int u = 0; u < NV_IT; ++u) {
+        const int i = tid + u * C::THREADS;
+        const int p = p0 + i / C::VCH;
+        vrow[u] = (i < C::KT * C::VCH && p < kend) ? __ldg(irow + p) : -1;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < NK_IT; ++u) krow[u] = cache_row(checked_id(krow[u], S_kv));
+    if constexpr (!LATENT) {
+#pragma unroll
+      for (int u = 0; u < NV_IT; ++u) vrow[u] = cache_row(vrow[u] >= S_kv ? -1 : vrow[u]);   // flagged once above
+    }
+#pragma unroll
+    for (int u = 0; u < NK_IT; ++u) {
+      const int i = tid + u * C::THREADS;
+      if (i < C::KT * C::QCH) {
+        const int r = i / C::QCH, c = i % C::QCH;
+        const int key = krow[u];
+        const __nv_bfloat16* src = kvb + (int64_t)(key < 0 ? 0 : key) * kv_rs + c * 8;
+        cp_async16(sbase + C::OFF_K + stage * C::K_TILE + swz(r, c, C::QCH), src, key < 0 ? 0 : 16);
+        if (c == 0) idx_s[stage * C::KT + r] = key;
+      }
+    }
+    if constexpr (!LATENT) {
+#pragma unroll
+      for (int u = 0; u < NV_IT; ++u) {
+        const int i = tid + u * C::THREADS;
+        if (i < C::KT * C::VCH) {
+          const int r = i / C::VCH, c = i % C::VCH;
+          const int key = vrow[u];
+          const __nv_bfloat16* src = vb + (int64_t)(key < 0 ? 0 : key) * v_rs + c * 8;
+          cp_async16(sbase + C::OFF_V + stage * C::V_TILE + swz(r, c, C::VCH), src, key < 0 ? 0 : 16);
+        }
       }
     }
   };
