@@ -579,10 +579,23 @@ def run_secondary(args, name, dev, steps=3, per_layer=False):
         fn = lambda: parts[0].step(ws, stream)  # noqa: E731
         for _ in range(max(3, args.warmup)):
             fn()
+        graph = None
+        if wl.T == 1:
+            # a decode step is a short chain of launches: it runs as one CUDA graph, as a serving
+            # loop would run it, so the host's launch path does not set its pace
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                parts[0].step(ws, torch.cuda.current_stream())
+            fn = graph.replay
+            for _ in range(3):
+                fn()
         ms = time_region(fn, steps, stream) / steps
         brk = breakdown(parts, ws, t_chunk, stream, dsa, 3)
         r = {"workload": name, "value": wl.B * wl.T / (ms / 1e3), "unit": "query tok/s", "ms_per_step": ms,
-             "steps": steps, "breakdown_ms": brk, "roofline": roofline([parts[0].wl], brk, peaks(), t_chunk)}
+             "steps": steps, "cuda_graph": graph is not None, "breakdown_ms": brk,
+             "roofline": roofline([parts[0].wl], brk, peaks(), t_chunk)}
+        del graph
         del g, ws, parts
         torch.cuda.empty_cache()
         return r
