@@ -395,6 +395,41 @@ def test_group_with_kept_pooled_cache_equals_pooling_in_the_call():
         assert torch.equal(o0, o1) and torch.equal(l0, l1)
 
 
+def test_decode_step_replays_as_a_cuda_graph():
+    """A decode step (pooled-cache refresh, indexer, top-k, split-key attention and its combine
+    for two layers) captured once as a CUDA graph and replayed gives the eager step's ids,
+    outputs and lse bit for bit: no call synchronises the host or allocates while capturing."""
+    wl = W.WORKLOADS["decode256k_pool"].replace(B=3, ctx=9000)
+    ind, lays = _inputs(wl, layers=2)
+    ctx = torch.tensor([9000, 4097, 2051], dtype=torch.int32, device=DEV)
+    kp = dsa.dsa_index_pool(ind["k_idx"], pool=wl.pool)
+    layers = [{"q": L["q"], "kv": L["kv"], "v": L["v"]} for L in lays]
+    g = dsa.Group(ind["q_idx"], ind["w"], ind["k_idx"], ctx, wl.topk, layers, wl.sm_scale, wl.d_v, pool=wl.pool,
+                  want_lse=True, k_pooled=kp)
+    ws = torch.empty(g.workspace_size(wl.T), dtype=torch.uint8, device=DEV)
+
+    def step(stream):
+        dsa.dsa_index_pool_tail(ind["k_idx"], ctx, wl.T, kp, pool=wl.pool, stream=stream)
+        return g.forward(ws, stream)
+
+    idx, outs = step(torch.cuda.current_stream())
+    eager = (idx.clone(), [(o.clone(), l.clone()) for o, l in outs])
+    for o, l in outs:
+        o.zero_()
+        l.zero_()
+    idx.fill_(-7)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(torch.cuda.current_stream())
+    graph.replay()
+    torch.cuda.synchronize()
+    assert dsa.dsa_device_status() == 0
+    assert torch.equal(idx, eager[0])
+    for (o, l), (oe, le) in zip(outs, eager[1]):
+        assert torch.equal(o, oe) and torch.equal(l, le)
+
+
 def test_pooled_decode_small():
     """The decode-shaped pooled path (one query per sequence, QB=1 indexer over pooled keys,
     top-512 blocks, split-key MLA attention), at a cache size the oracle checks in seconds."""
