@@ -253,6 +253,17 @@ def job_throughput(units_per_rank_step: int, world: int, ms_per_step: float) -> 
     return units_per_rank_step * world / (ms_per_step / 1e3)
 
 
+def l2_note(wl) -> str:
+    """How the timed steps relate to the 126 MB L2: the key caches and the per-layer inputs of a
+    step either exceed it (no flush is needed between steps) or not (small profiling cases,
+    which are timed without a flush and say so)."""
+    step_bytes = (wl.B * wl.S // wl.pool * wl.d_I + wl.B * wl.T * wl.H_I * (wl.d_I + 4)
+                  + wl.group * wl.B * (wl.T * wl.Hq * wl.d_qk + wl.S * (wl.d_qk + (0 if wl.kv_latent else wl.d_v))) * 2)
+    if step_bytes > 126e6:
+        return "inputs larger than L2 (126 MB); no flush"
+    return f"inputs of {step_bytes / 1e6:.1f} MB fit in L2 (126 MB): a small profiling case, not flushed"
+
+
 def time_region(fn, steps, stream):
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
@@ -308,7 +319,7 @@ def run_ours(args, rank, world, dev):
                    "group": wl.group, "t_chunk": t_chunk,
                    "parallelism": "1 GPU" if world == 1 else
                    (f"query rows sharded zig-zag over {world} ranks" if wl.T > 1 else f"batch sharded over {world} ranks"),
-                   "l2": "inputs larger than L2 (126 MB); no flush"},
+                   "l2": l2_note(wl)},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "breakdown_ms": brk,
