@@ -77,8 +77,14 @@ struct Cfg {
   static constexpr int P_BYTES = HG * KT * 2;
   static constexpr int OFF_K = Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * K_TILE;
+  // With separate V rows, P lives in the current stage's K tile, free once the tile's scores
+  // are computed (every warp has passed the barrier after its score reads before P is
+  // written, and the next copy into that stage follows the barrier that ends the tile's P.V);
+  // the smaller footprint fits one more CTA per SM.  In the latent form K is also V: P gets its
+  // own buffer.
+  static constexpr bool P_IN_K = !LATENT && P_BYTES <= K_TILE;
   static constexpr int OFF_P = OFF_V + STAGES * V_TILE;
-  static constexpr int OFF_IDX = OFF_P + P_BYTES;
+  static constexpr int OFF_IDX = OFF_P + (P_IN_K ? 0 : P_BYTES);
   static constexpr int OFF_RED = OFF_IDX + STAGES * KT * 4;
   static constexpr int SMEM = OFF_RED + 2 * NWV * HG * 4;
   static_assert(QCH % 8 == 0 && VCH % 8 == 0, "rows must be whole 128-byte swizzle groups");
@@ -247,7 +253,7 @@ sparse_attn_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16*
       m_run[r] = mnew[r];
     }
     // ---- P = exp2(S - m), written to shared memory as bf16
-    const uint32_t pbase = sbase + C::OFF_P;
+    const uint32_t pbase = C::P_IN_K ? ks_base : sbase + C::OFF_P;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       float p[4];
