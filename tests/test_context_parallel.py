@@ -143,3 +143,155 @@ def test_context_parallel_guards_skip_and_flag_bad_ids():
     out = dsa.dsa_topk_merge(sc, few, ctx, 1, 100, k)
     assert dsa.dsa_device_status() == 7
     assert out.tolist() == [[[-1, -1, -1, -1]]]
+
+
+# ---------------------------------------------------------------- the whole key-sharded group
+# over a real process group (gloo, three CPU ranks), with a stand-in for the library whose steps
+# are the oracle's definitions: this checks group_forward's plan, its query chunks, its two
+# exchanges and its merge order, not the kernels (those are the GPU tests above).
+
+class _OracleSteps:
+    """The library's step calls, computed on the CPU from the oracle's definitions (test only)."""
+
+    def __init__(self):
+        import oracle as O
+        self.O = O
+
+    def dsa_index_scores(self, q_idx, w, k_idx, ctx_len, t_begin=0, t_count=None, stream=None):
+        O = self.O
+        B, T = q_idx.shape[:2]
+        S = k_idx.shape[1]
+        ld = (S + 3) // 4 * 4
+        out = torch.full((B, t_count, ld), float("-inf"))
+        for b in range(B):
+            kd = O.e4m3_to_f64(k_idx[b].numpy())
+            for r in range(t_count):
+                t = t_begin + r
+                pos = int(ctx_len[b]) - T + t
+                out[b, r, :S] = torch.from_numpy(O.index_scores_row(O.e4m3_to_f64(q_idx[b, t].numpy()),
+                                                                    w[b, t].numpy(), kd, pos))
+        return out
+
+    def dsa_topk(self, sc, ctx_len, T, S, k, t_begin=0, idx=None, stream=None):
+        B, tc = sc.shape[:2]
+        for b in range(B):
+            for r in range(tc):
+                pos = int(ctx_len[b]) - T + t_begin + r
+                n_valid = 0 if pos < 0 else min(S, pos + 1)
+                sel = self.O.topk_row(sc[b, r].numpy(), n_valid, k)
+                ids = np.sort(sel[sel >= 0])
+                row = np.full(k, -1, dtype=np.int32)
+                row[: ids.size] = ids
+                idx[b, t_begin + r] = torch.from_numpy(row)
+        return idx
+
+    def dsa_gather_selected(self, sc, idx, t_begin, id_offset, stream=None):
+        B, tc = sc.shape[:2]
+        sel = idx[:, t_begin:t_begin + tc].long()
+        cs = torch.where(sel >= 0, torch.gather(sc, 2, sel.clamp(min=0)), torch.tensor(float("-inf")))
+        ci = torch.where(sel >= 0, sel + id_offset, torch.tensor(-1)).to(torch.int32)
+        return cs.float(), ci
+
+    def dsa_topk_merge(self, cs, ci, ctx_len, T, S_total, k, t_begin=0, idx=None, stream=None):
+        P, B, tc, kc = cs.shape
+        for b in range(B):
+            for r in range(tc):
+                pos = int(ctx_len[b]) - T + t_begin + r
+                n_valid = 0 if pos < 0 else min(S_total, pos + 1)
+                row = np.full(k, -1, dtype=np.int32)
+                if n_valid <= k:
+                    row[:n_valid] = np.arange(n_valid)
+                else:
+                    s = cs[:, b, r].reshape(-1).double().numpy()
+                    i = ci[:, b, r].reshape(-1).numpy()
+                    keep = i >= 0
+                    s, i = s[keep], i[keep]
+                    order = np.lexsort((i, -s))[:k]
+                    row[:] = np.sort(i[order])
+                idx[b, t_begin + r] = torch.from_numpy(row)
+        return idx
+
+    def dsa_idx_localize(self, idx, s0, s_len, stream=None):
+        return torch.where((idx >= s0) & (idx < s0 + s_len), idx - s0, torch.tensor(-1, dtype=torch.int32)).to(torch.int32)
+
+    def dsa_sparse_attn(self, q, kv, idx, sm_scale, d_v, want_lse=False, stream=None):
+        O = self.O
+        B, T, Hq = q.shape[:3]
+        out = torch.empty((B, T, Hq, d_v), dtype=torch.bfloat16)
+        lse = torch.empty((B, T, Hq), dtype=torch.float32)
+        for b in range(B):
+            K = kv[b].double().numpy()
+            for t in range(T):
+                o, l = O.sparse_attn_row(q[b, t].double().numpy(), K, K[:, :d_v], idx[b, t].numpy(), sm_scale)
+                out[b, t] = torch.from_numpy(o).to(torch.bfloat16)
+                lse[b, t] = torch.from_numpy(l).float()
+        return out, lse
+
+    def dsa_attn_combine(self, part_o, part_lse, want_lse=False, stream=None):
+        lse = torch.logsumexp(part_lse.double(), dim=0)
+        wgt = torch.exp(part_lse.double() - lse).nan_to_num(0.0)
+        out = (wgt.unsqueeze(-1) * part_o.double()).sum(0)
+        return out.to(torch.bfloat16), lse.float()
+
+
+def _cp_inputs():
+    g = torch.Generator().manual_seed(31)
+    B, T, S, H, D, Hq, Dqk, Dv = 2, 6, 200, 4, 64, 4, 64, 32
+    codes = torch.randint(0, 126, (B, S, D), generator=g, dtype=torch.int32).to(torch.uint8)
+    q_idx = torch.randint(0, 126, (B, T, H, D), generator=g, dtype=torch.int32).to(torch.uint8)
+    w = torch.randn((B, T, H), generator=g) * 0.5
+    ctx = torch.tensor([200, 100], dtype=torch.int32)
+    qs = [torch.randn((B, T, Hq, Dqk), generator=g).to(torch.bfloat16) for _ in range(2)]
+    kvs = [torch.randn((B, S, Dqk), generator=g).to(torch.bfloat16) for _ in range(2)]
+    return q_idx, w, codes, ctx, qs, kvs, 16, 1.0 / 8.0, Dv
+
+
+def _cp_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        q_idx, w, codes, ctx, qs, kvs, k, sm_scale, d_v = _cp_inputs()
+        S = codes.shape[1]
+        s0, n = cp.key_shards(S, world)[rank]
+        rk = cp.Rank((s0, n), q_idx, w, codes[:, s0:s0 + n].contiguous(), ctx, [kv[:, s0:s0 + n].contiguous() for kv in kvs], S)
+        idx, outs = cp.group_forward(_OracleSteps(), rk, qs, k, sm_scale, d_v, cp.nccl_all_gather(), t_chunk=4)
+        q.put((rank, idx.numpy(), [(o.float().numpy(), l.numpy()) for o, l in outs]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_key_sharded_group_over_three_cpu_ranks_matches_the_oracle():
+    """Three gloo ranks (the last one holding no keys), two query chunks, ragged contexts (one
+    sequence's keys all on the first rank): every rank ends with the unsharded selection of the
+    oracle and its attention (bf16 parts merged by log-sum-exp)."""
+    import oracle as O
+    ctx_mp = mp.get_context("spawn")
+    q = ctx_mp.Queue()
+    port = 29700 + (os.getpid() % 1000)
+    world = 3
+    ps = [ctx_mp.Process(target=_cp_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in ps:
+        p.start()
+    got = dict((r, (i, o)) for r, i, o in (q.get(timeout=300) for _ in ps))
+    for p in ps:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert cp.key_shards(200, 3)[2][1] == 0
+    q_idx, w, codes, ctx, qs, kvs, k, sm_scale, d_v = _cp_inputs()
+    B, T = q_idx.shape[:2]
+    for b in range(B):
+        kd = O.e4m3_to_f64(codes[b].numpy())
+        layers = [{"q": qs[l][b].double().numpy(), "K": kvs[l][b].double().numpy(),
+                   "V": kvs[l][b].double().numpy()[:, :d_v]} for l in range(2)]
+        for t in range(T):
+            pos = int(ctx[b]) - T + t
+            idx_ref, outs_ref = O.group_forward_row(O.e4m3_to_f64(q_idx[b, t].numpy()), w[b, t].numpy(), kd, pos, k,
+                                                    [dict(L, q=L["q"][t]) for L in layers], sm_scale)
+            want = np.sort(idx_ref[idx_ref >= 0])
+            for r in range(world):
+                idx_r, outs_r = got[r]
+                row = idx_r[b, t]
+                assert np.array_equal(row[row >= 0], want) and (row[want.size:] == -1).all(), (r, b, t)
+                for (o, l), (oref, lref) in zip(outs_r, outs_ref):
+                    assert np.abs(o[b, t] - oref).max() <= 2e-2
+                    assert np.abs(l[b, t] - lref).max() <= 1e-3 * max(1.0, np.abs(lref).max())
