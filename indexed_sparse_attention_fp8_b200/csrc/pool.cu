@@ -95,8 +95,8 @@ index_pool_tail_kernel(const uint4* __restrict__ k_idx, const int32_t* __restric
   const int j = (int)((gid / slices) % window);
   const int b = (int)(gid / ((int64_t)slices * window));
   const int S_max = groups_per_seq * P;
-  const int hi = min(__ldg(ctx_len + b), S_max);   // rows [lo, hi) were appended
-  const int lo = max(hi - T, 0);
+  const int ctx = __ldg(ctx_len + b);
+  const int lo = max(ctx - T, 0), hi = min(ctx, S_max);   // appended rows [ctx - T, ctx) in the cache
   if (hi <= lo) return;
   const int g = lo / P + j;
   if (g > (hi - 1) / P) return;
