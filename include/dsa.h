@@ -330,6 +330,8 @@ int dsa_group_forward(const dsa_group_args* args, void* ws, size_t ws_bytes, voi
  *      whole row, identical on every rank;
  *   5. per layer: dsa_idx_localize, then dsa_sparse_attn over the rank's rows (want lse);
  *   6. the caller all-gathers every rank's (O, lse); dsa_attn_combine merges them.
+ * A rank whose shard is empty (len_r = 0) calls nothing in steps 1, 2 and 5: it contributes
+ * (-inf, -1) candidates and a part with O = 0, lse = -inf, which the merges ignore.
  * pool must be 1.  Errors and asynchrony as for the other calls.
  * ------------------------------------------------------------------------------------ */
 
