@@ -14,13 +14,17 @@ alone.  The path then has two real exchange steps, both all-gathers (NCCL over N
 Every step runs in the library's kernels (dsa.h, "Context parallelism"); this module plans the
 shards and orders the calls and the exchanges.  The steps are separate functions, so a caller can
 run them for all ranks in one process too (the tests do, joining the ranks' tensors in place of
-the all-gather).  IndexPool is not supported here (pool 1).
+the all-gather).  IndexPool is not supported here (pool 1).  The merge holds at most 16384
+candidates per row, so world * k <= 16384 (eight ranks at k = 2048).
 """
 from __future__ import annotations
 
 from typing import Callable, List, Optional, Sequence, Tuple
 
 import torch
+
+
+MERGE_MAX_CANDIDATES = 16384   # candidates per row dsa_topk_merge accepts (n_parts * kc)
 
 
 def key_shards(S: int, world: int, align: int = 128) -> List[Tuple[int, int]]:
@@ -106,7 +110,11 @@ def group_forward(dsa, rk: Rank, qs: Sequence[torch.Tensor], k: int, sm_scale: f
     for t0 in range(0, T, t_chunk):
         tc = min(t_chunk, T - t0)
         cs, ci = select_candidates(dsa, rk, k, t0, tc, idx_local, stream=stream)
-        merge_selection(dsa, all_gather(cs), all_gather(ci), rk.ctx_len, T, rk.S_total, k, t0, idx, stream=stream)
+        cs_all, ci_all = all_gather(cs), all_gather(ci)
+        if cs_all.shape[0] * k > MERGE_MAX_CANDIDATES:   # the same on every rank: all stop here
+            raise ValueError(f"{cs_all.shape[0]} ranks x k={k} candidates exceed the merge's "
+                             f"{MERGE_MAX_CANDIDATES} per row")
+        merge_selection(dsa, cs_all, ci_all, rk.ctx_len, T, rk.S_total, k, t0, idx, stream=stream)
     outs = []
     for layer, q in enumerate(qs):
         o, lse = attend_local(dsa, rk, layer, q, idx, sm_scale, d_v, stream=stream)
