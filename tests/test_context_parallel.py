@@ -295,3 +295,14 @@ def test_key_sharded_group_over_three_cpu_ranks_matches_the_oracle():
                 for (o, l), (oref, lref) in zip(outs_r, outs_ref):
                     assert np.abs(o[b, t] - oref).max() <= 2e-2
                     assert np.abs(l[b, t] - lref).max() <= 1e-3 * max(1.0, np.abs(lref).max())
+
+
+def test_group_refuses_more_candidates_than_the_merge_holds():
+    """world x k above the merge's 16384 candidates per row stops at the first exchange (the
+    check sees the gathered shape, so every rank stops at the same point)."""
+    q_idx, w, codes, ctx, qs, kvs, _, sm_scale, d_v = _cp_inputs()
+    S = codes.shape[1]
+    rk = cp.Rank((0, S), q_idx, w, codes, ctx, kvs, S)
+    nine = lambda t: torch.stack([t] * 9)   # noqa: E731  (nine ranks' worth of candidates)
+    with pytest.raises(ValueError, match="exceed"):
+        cp.group_forward(_OracleSteps(), rk, qs, 2048, sm_scale, d_v, nine, t_chunk=6)
